@@ -1,0 +1,169 @@
+"""Seeded synthetic inputs for VDA forward.
+
+This module holds no step of the method: it only draws random tensors,
+normalises key/query rows, rounds to BF16 and widens BF16 bits back to
+float64.  Both the CUDA path and the float64 oracle are fed from here, so both
+see identical input values.
+
+Workloads.  The pages measure a 768p, 14.4 s clip (the performance tables of
+the agentlenshq.com project summary and the comfyui-wiki.com news page); no
+dataset is involved.  The shapes below stand in for that clip's attention
+inputs: a 24 x 42 latent grid (n = 1008 tokens per frame), T = 45 latent
+frames, 32 heads of width 128 and 256 text tokens.
+
+Recipe (per tensor, independent stream ``PCG64(seed * 100 + index)``):
+  Q, K, K_txt : rows L2-normalised from N(0, 1)
+  V, V_txt, G : N(0, 1)  (G ~ N(0, 2), i.e. variance 2, for the mid config)
+  ill-conditioned keys: K_t = L2norm(U_t W + 0.05 E), U_t ~ N(0,1) (n x 8,
+  fresh per frame), W ~ N(0,1) (8 x d_k, one per (b, h)), E ~ N(0,1).
+Values are drawn in float32, normalised in float32, then rounded to BF16
+(round to nearest even) for BF16 workloads.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+# Stream index of every tensor; fixed so that a tensor's values do not depend
+# on which other tensors a workload draws.
+_STREAM = {"Q": 0, "K": 1, "V": 2, "G": 3, "K_txt": 4, "V_txt": 5, "U": 6, "W": 7, "E": 8}
+
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    T: int
+    n: int
+    n_txt: int
+    d_k: int
+    d_v: int
+    dtype: int
+    lam: float
+    g_std: float = 1.0
+    ill_conditioned: bool = False
+    rank: int = 8
+    noise: float = 0.05
+
+    @property
+    def units(self) -> int:
+        """(frame, head) units, the metric's counting unit."""
+        return self.B * self.H * self.T
+
+    def problem(self) -> dict:
+        return dict(B=self.B, H=self.H, T=self.T, n=self.n, n_txt=self.n_txt,
+                    d_k=self.d_k, d_v=self.d_v, dtype=self.dtype, lam=self.lam)
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", B=1, H=1, T=8, n=64, n_txt=16, d_k=64, d_v=64, dtype=DTYPE_F32, lam=1.0),
+    "mid": Workload("mid", B=1, H=8, T=16, n=256, n_txt=128, d_k=128, d_v=128, dtype=DTYPE_BF16,
+                    lam=0.5, g_std=math.sqrt(2.0)),
+    "768p": Workload("768p", B=1, H=32, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16, lam=1.0),
+    "illcond": Workload("illcond", B=1, H=32, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16,
+                        lam=0.05, ill_conditioned=True),
+    "long45": Workload("long45", B=2, H=32, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16, lam=1.0),
+    "long90": Workload("long90", B=2, H=32, T=90, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16, lam=1.0),
+    "long180": Workload("long180", B=2, H=32, T=180, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16,
+                        lam=1.0),
+}
+
+
+def _rng(seed: int, name: str) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(seed * 100 + _STREAM[name]))
+
+
+def _l2norm_rows(x: np.ndarray) -> np.ndarray:
+    nrm = np.sqrt(np.einsum("...i,...i->...", x, x, dtype=np.float32))
+    nrm = np.maximum(nrm, np.float32(1e-30))
+    return (x / nrm[..., None]).astype(np.float32)
+
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> BF16 bit patterns (uint16), round to nearest even."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def widen(x: np.ndarray, dtype: int) -> np.ndarray:
+    """Exact float64 view of an input tensor as stored (BF16 bits or float32)."""
+    if dtype == DTYPE_BF16:
+        return bf16_bits_to_f32(x).astype(np.float64)
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+@dataclasses.dataclass
+class Inputs:
+    """Host copies of one workload's inputs, as stored on the device.
+
+    BF16 tensors are uint16 bit patterns; FP32 tensors are float32.
+    """
+    workload: Workload
+    Q: np.ndarray
+    K: np.ndarray
+    V: np.ndarray
+    G: np.ndarray
+    K_txt: np.ndarray
+    V_txt: np.ndarray
+
+    def widened(self, name: str, index=None) -> np.ndarray:
+        a = getattr(self, name)
+        if index is not None:
+            a = a[index]
+        return widen(a, self.workload.dtype)
+
+    def nbytes_in(self) -> int:
+        return sum(getattr(self, k).nbytes for k in ("Q", "K", "V", "G", "K_txt", "V_txt"))
+
+
+def _normal(seed: int, name: str, shape, std: float = 1.0) -> np.ndarray:
+    x = _rng(seed, name).standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        x *= np.float32(std)
+    return x
+
+
+def _ill_keys(w: Workload, seed: int) -> np.ndarray:
+    """K_t = L2norm(U_t W + noise * E), W shared over the frames of one (b, h)."""
+    U = _normal(seed, "U", (w.B, w.H, w.T, w.n, w.rank))
+    W = _normal(seed, "W", (w.B, w.H, w.rank, w.d_k))
+    E = _normal(seed, "E", (w.B, w.H, w.T, w.n, w.d_k))
+    K = np.empty((w.B, w.H, w.T, w.n, w.d_k), dtype=np.float32)
+    for b in range(w.B):
+        for h in range(w.H):
+            K[b, h] = np.matmul(U[b, h], W[b, h]) + np.float32(w.noise) * E[b, h]
+    return _l2norm_rows(K)
+
+
+def make_inputs(w: Workload | str, seed: int = 0) -> Inputs:
+    """Draw one workload's inputs (host numpy arrays, storage dtype)."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    sh_k = (w.B, w.H, w.T, w.n, w.d_k)
+    sh_v = (w.B, w.H, w.T, w.n, w.d_v)
+    Q = _l2norm_rows(_normal(seed, "Q", sh_k))
+    K = _ill_keys(w, seed) if w.ill_conditioned else _l2norm_rows(_normal(seed, "K", sh_k))
+    V = _normal(seed, "V", sh_v)
+    G = _normal(seed, "G", sh_v, std=w.g_std)
+    K_txt = _l2norm_rows(_normal(seed, "K_txt", (w.B, w.H, w.n_txt, w.d_k)))
+    V_txt = _normal(seed, "V_txt", (w.B, w.H, w.n_txt, w.d_v))
+    if w.dtype == DTYPE_BF16:
+        conv = to_bf16_bits
+    else:
+        conv = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    return Inputs(w, conv(Q), conv(K), conv(V), conv(G), conv(K_txt), conv(V_txt))

@@ -1,0 +1,83 @@
+"""Oracle regression fixture and the seeded input generators (CPU only)."""
+import os
+
+import numpy as np
+
+from frame_wise_linear_b200 import synth
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _load_golden():
+    rows = {"frob_SF": {}, "frob_SB": {}, "O": {}}
+    with open(os.path.join(HERE, "golden", "tiny_oracle.txt")) as fh:
+        for line in fh:
+            if line.startswith("#"):
+                continue
+            p = line.split()
+            if p[0] == "frob_O":
+                rows["frob_O"] = float(p[1])
+            elif p[0] in ("frob_SF", "frob_SB"):
+                rows[p[0]][int(p[1])] = float(p[2])
+            else:
+                rows["O"][tuple(int(x) for x in p[1:-1])] = float(p[-1])
+    return rows
+
+
+def test_oracle_matches_stored_fixture():
+    import sys
+    sys.path.insert(0, os.path.join(HERE, "golden"))
+    import make_golden
+    O, st, idx = make_golden.compute()
+    g = _load_golden()
+    assert abs(np.linalg.norm(O) - g["frob_O"]) <= 1e-12 * g["frob_O"]
+    for t, v in g["frob_SF"].items():
+        assert abs(np.linalg.norm(st["SF"][t]) - v) <= 1e-12 * v
+    for t, v in g["frob_SB"].items():
+        assert abs(np.linalg.norm(st["SB"][t]) - v) <= 1e-12 * v
+    for i, v in g["O"].items():
+        assert abs(O[i] - v) <= 1e-12 * max(1.0, abs(v))
+
+
+def test_generator_is_deterministic_and_normalised():
+    a = synth.make_inputs("tiny", seed=0)
+    b = synth.make_inputs("tiny", seed=0)
+    c = synth.make_inputs("tiny", seed=1)
+    for k in ("Q", "K", "V", "G", "K_txt", "V_txt"):
+        assert np.array_equal(getattr(a, k), getattr(b, k))
+        assert not np.array_equal(getattr(a, k), getattr(c, k))
+    for k in ("Q", "K", "K_txt"):
+        nrm = np.linalg.norm(a.widened(k), axis=-1)
+        assert np.allclose(nrm, 1.0, atol=1e-6)
+    assert a.Q.dtype == np.float32 and a.Q.shape == (1, 1, 8, 64, 64)
+
+
+def test_bf16_rounding_is_nearest_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 3.0e38, 1e-40], dtype=np.float32)
+    bits = synth.to_bf16_bits(x)
+    back = synth.bf16_bits_to_f32(bits)
+    # ties go to even: 1 + 2^-8 -> 1, 1 + 3*2^-8 -> 1 + 2^-6
+    assert back[0] == 1.0 and back[1] == 1.0 and back[2] == np.float32(1.0 + 2 ** -6)
+    assert back[3] == -2.5
+    rng = np.random.default_rng(0)
+    y = rng.standard_normal(10000).astype(np.float32)
+    yb = synth.bf16_bits_to_f32(synth.to_bf16_bits(y))
+    assert np.max(np.abs(yb - y) / np.abs(y)) <= 2 ** -8
+
+
+def test_mid_workload_statistics():
+    w = synth.WORKLOADS["mid"].replace(H=2)
+    inp = synth.make_inputs(w, seed=0)
+    assert inp.Q.dtype == np.uint16 and inp.Q.shape == (1, 2, 16, 256, 128)
+    G = inp.widened("G")
+    assert abs(G.var() - 2.0) < 0.05          # G ~ N(0, 2): variance 2
+    V = inp.widened("V")
+    assert abs(V.var() - 1.0) < 0.05
+
+
+def test_ill_conditioned_keys_are_nearly_low_rank():
+    w = synth.WORKLOADS["illcond"].replace(H=1, T=2)
+    inp = synth.make_inputs(w, seed=0)
+    K = inp.widened("K")[0, 0, 0]
+    s = np.linalg.svd(K, compute_uv=False)
+    assert s[7] ** 2 > 50 and s[8] ** 2 < 0.05     # 8 dominant directions, the rest noise
