@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of VDA forward (both scan directions + gated readout) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+One step = one whole VDA forward (Gram, factor-and-solve, bidirectional scan,
+readout) over one 768p full-clip problem: B=1, H=32, T=45 frames, n=1008
+tokens (24 x 42), d_k=d_v=128, 256 text tokens, bfloat16, lambda=1, seeded
+synthetic inputs resident in HBM.  Metric: (frame, head) units per second.
+
+N > 1 (torchrun, one process per GPU): every rank runs its own problem (heads
+and batches are independent, so there is no data-path collective); the value
+is the units of all ranks over the max-over-ranks device time (weak scaling).
+
+The JSON line also carries: the roofline of the dominant kernel (timed with
+CUDA events on the launching stream, inside the timed region), the path's
+roofline fraction, an end-to-end figure through the host-buffer entry point,
+clocks sampled during the timed region, and (rank 0, N=1) the float64 CPU
+oracle timed on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "VDA frames*heads/sec (fwd+bwd) at 768p shape; % of B200 roofline"
+UNIT = "frames*heads/s"
+WORKLOAD = "768p"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# FP32 SIMT peak from unit counts and clock: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz.
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+# Kernel of each stage and the source file that defines it (for ncu traffic lookups).
+STAGE_SOURCES = {
+    "gram": "frame_wise_linear_b200/csrc/vda_simt.cu",
+    "factor": "frame_wise_linear_b200/csrc/vda_simt.cu",
+    "scan": "frame_wise_linear_b200/csrc/vda_simt.cu",
+    "readout": "frame_wise_linear_b200/csrc/vda_simt.cu",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("b200", "reference"), default="b200")
+    ap.add_argument("--workload", default=WORKLOAD, help="a name from frame_wise_linear_b200.synth.WORKLOADS")
+    ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end leg (default min(K, 10))")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Work counts (the design doc states them): algorithmic bytes / flops per launch.
+# ---------------------------------------------------------------------------
+
+def stage_work(w):
+    es = 2 if w.dtype == 1 else 4
+    bh = w.B * w.H
+    frames = bh * w.T
+    slots = bh * (w.T + 1)
+    d_k, d_v = w.d_k, w.d_v
+    return {
+        # reads K_t, V_t of every frame and the text once
+        "gram": dict(bound="hbm", bytes=(frames * w.n + bh * w.n_txt) * (d_k + d_v) * es,
+                     flops=2.0 * (frames * w.n + bh * w.n_txt) * d_k * (d_k + d_v)),
+        # Cholesky (d^3/3) + two triangular solves with d_k + d_v right-hand sides
+        "factor": dict(bound="alu", bytes=0, flops=slots * (d_k ** 3 / 3.0 + 2.0 * d_k * d_k * (d_k + d_v))),
+        # two directions, one d_k x d_k by d_k x d_v product per frame
+        "scan": dict(bound="alu", bytes=0, flops=2.0 * frames * 2.0 * d_k * d_k * d_v),
+        # reads Q_t, G_t, writes O_t
+        "readout": dict(bound="hbm", bytes=frames * w.n * (d_k + 2 * d_v) * es,
+                        flops=2.0 * frames * w.n * d_k * d_v),
+    }
+
+
+def path_roofline(w, peaks):
+    es = 2 if w.dtype == 1 else 4
+    bh = w.B * w.H
+    frames = bh * w.T
+    nbytes = frames * w.n * (2 * w.d_k + 3 * w.d_v) * es + bh * w.n_txt * (w.d_k + w.d_v) * es
+    flops = 2.0 * frames * w.n * (w.d_k * (w.d_k + w.d_v) + w.d_k * w.d_v) \
+        + 2.0 * bh * w.n_txt * w.d_k * (w.d_k + w.d_v)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    return dict(bytes=nbytes, tensor_flops=flops, t_roof_s=max(t_hbm, t_tc),
+                bound="hbm" if t_hbm >= t_tc else "tensor")
+
+
+def traffic_lookup(stage):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = os.path.join(ROOT, STAGE_SOURCES[stage])
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    with open(path) as fh:
+        for line in fh:
+            p = line.split()
+            if len(p) >= 3 and not line.startswith("#") and p[0] == stage and p[1] == digest:
+                return float(p[2])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# Clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="vda_clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.6)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"unavailable": "nvidia-smi could not be started"}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                if self.uuid and p[0] != self.uuid:
+                    continue
+                rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"unavailable": "no nvidia-smi samples for this GPU"}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_oracle_sample(w, budget_s, max_frames=None):
+    """Times the float64 oracle on whole heads (all frames) until the budget is used.
+
+    Returns (frames*heads per second, units timed, description).  Input
+    generation and widening are outside the timed part.
+    """
+    from frame_wise_linear_b200 import synth
+    from oracle import vda_oracle as vo
+    spent, units, heads = 0.0, 0, 0
+    for b in range(w.B):
+        for h in range(w.H):
+            x = synth.head_widened(w, b, h, seed=0)
+            T = w.T if max_frames is None else min(w.T, max_frames)
+            args = [x["Q"][:T], x["K"][:T], x["V"][:T], x["G"][:T], x["K_txt"], x["V_txt"], w.lam]
+            t0 = time.perf_counter()
+            vo.vda_head(*args)
+            spent += time.perf_counter() - t0
+            units += T
+            heads += 1
+            if spent >= budget_s:
+                break
+        if spent >= budget_s:
+            break
+    desc = f"{heads} head(s) x {units // max(heads, 1)} frames of the {w.name} workload (float64 oracle)"
+    return units / spent, units, desc
+
+
+# ---------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    # Size each step so the whole run stays within about two minutes.
+    from frame_wise_linear_b200 import synth
+    from oracle import vda_oracle as vo
+    x = synth.head_widened(w, 0, 0, seed=0)
+    t0 = time.perf_counter()
+    vo.vda_head(x["Q"][:2], x["K"][:2], x["V"][:2], x["G"][:2], x["K_txt"], x["V_txt"], w.lam)
+    per_frame = (time.perf_counter() - t0) / 2
+    budget = 120.0 / max(args.steps + args.warmup, 1)
+    frames = int(max(1, min(w.T, budget / max(per_frame, 1e-6))))
+    args_h = [x["Q"][:frames], x["K"][:frames], x["V"][:frames], x["G"][:frames], x["K_txt"], x["V_txt"], w.lam]
+    for _ in range(args.warmup):
+        vo.vda_head(*args_h)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vo.vda_head(*args_h)
+    dt = time.perf_counter() - t0
+    value = args.steps * frames / dt
+    sample = f"each step: head (0,0), frames 1..{frames} of the {w.name} workload (float64 oracle)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, n):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} n={w.n} d_k={w.d_k} d_v={w.d_v} "
+                        f"n_txt={w.n_txt} lambda={w.lam} {'bf16' if w.dtype == 1 else 'f32'}",
+            "B": w.B, "H": w.H, "T": w.T, "n": w.n, "n_txt": w.n_txt, "d": w.d_k,
+            "parallelism": f"independent problems on {n} GPU(s), no collective",
+            "l2": "inputs larger than L2 (1.49 GB per step vs 126 MB); no flush"}
+
+
+def run_b200(args, w):
+    import torch
+    from frame_wise_linear_b200 import build as _build
+    from frame_wise_linear_b200 import synth, vda
+
+    ws_n, rank, local = dist_env()
+    if args.gpus != ws_n:
+        if ws_n == 1 and args.gpus > 1:
+            raise SystemExit("--gpus N > 1 needs torchrun (one process per GPU)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    _build.build()
+    vda.load()
+
+    peaks, peaks_kind = load_peaks()
+    d = synth.make_inputs_torch(w, seed=rank, device=dev)
+    prob = vda.make_problem(**w.problem())
+    wsb = vda.vda_workspace_size(prob)
+    wsp = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    O = torch.empty_like(d["G"])
+    stream = torch.cuda.current_stream(dev)
+    kt = d["K_txt"] if w.n_txt else None
+    vt = d["V_txt"] if w.n_txt else None
+
+    def step(events=None):
+        if events is None:
+            vda.vda_forward(prob, d["Q"], d["K"], d["V"], d["G"], kt, vt, O, wsp, stream=stream)
+        else:
+            vda.vda_forward_timed(prob, d["Q"], d["K"], d["V"], d["G"], kt, vt, O, wsp, events, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    vda.vda_sync_status(wsp, stream=stream)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(vda.VDA_TIMED_EVENTS)]
+          for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for k in range(args.steps):
+        step(ev[k])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop()
+    vda.vda_sync_status(wsp, stream=stream)
+    ms = start.elapsed_time(end)
+    stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i, s in enumerate(vda.STAGES)}
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = ws_n * w.units / (ms_step / 1e3)
+
+    # dominant kernel roofline
+    work = stage_work(w)
+    dom = max(stage_ms, key=stage_ms.get)
+    wk = work[dom]
+    t_s = stage_ms[dom] / 1e3
+    if wk["bound"] == "hbm":
+        roof = {"kernel": dom, "bound": "hbm", "achieved": wk["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json hbm_gbs)"}
+    else:
+        roof = {"kernel": dom, "bound": "alu", "achieved": wk["flops"] / t_s / 1e12, "peak": FP32_SIMT_TFLOPS,
+                "unit": "TFLOP/s", "peak_source": "derived: 148 SMs x 128 FP32 FMA/clk x 2 x 1.965 GHz"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = traffic_lookup(dom)
+    roof["traffic"] = tr
+    pr = path_roofline(w, peaks)
+    path = {"t_roof_us": pr["t_roof_s"] * 1e6, "bound": pr["bound"], "bytes": pr["bytes"],
+            "frac": pr["t_roof_s"] / (ms_step / 1e3), "stage_ms": stage_ms}
+
+    # end-to-end through host buffers (pinned), copies inside the timed region
+    e2e_steps = args.e2e_steps if args.e2e_steps is not None else min(args.steps, 10)
+    host = {k: v.cpu().pin_memory() for k, v in d.items()}
+    Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    del d
+    wsh = torch.empty(vda.vda_host_workspace_size(prob), dtype=torch.uint8, device=dev)
+    hkt = host["K_txt"] if w.n_txt else None
+    hvt = host["V_txt"] if w.n_txt else None
+    vda.vda_forward_host(prob, host["Q"], host["K"], host["V"], host["G"], hkt, hvt, Oh, wsh, stream=stream)
+    if pg:
+        pg.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        vda.vda_forward_host(prob, host["Q"], host["K"], host["V"], host["G"], hkt, hvt, Oh, wsh, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(v.numel() * v.element_size() for k, v in host.items() if (w.n_txt or k not in ("K_txt", "V_txt")))
+    d2h = Oh.numel() * Oh.element_size()
+    e2e = {"value": ws_n * w.units / (e2e_ms / e2e_steps / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+           "api": "vda_forward_host (C ABI, pinned host buffers)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == 1 else "f32", "data": "synthetic",
+        "config": config_of(w, ws_n), "roofline": roof, "roofline_path": path, "e2e": e2e,
+        "clocks": clocks, "gpu_launches": len(vda.STAGES) * args.steps,
+    }
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        v, units, desc = cpu_oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": desc}
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    from frame_wise_linear_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_b200(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,279 @@
+// Host side of the C ABI declared in include/vda.h: argument checks,
+// workspace carve-up and the launch sequence.  No compute happens here.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "vda_internal.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+vda_status fail(vda_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+vda_status fail(vda_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+vda_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(VDA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+vda_status check_problem(const vda_problem* p) {
+  if (!p) return fail(VDA_ERR_INVALID_ARG, "problem is NULL");
+  if (p->B < 1 || p->H < 1 || p->T < 1 || p->n < 1)
+    return fail(VDA_ERR_INVALID_ARG, "B, H, T, n must be >= 1 (got %d, %d, %d, %d)", p->B, p->H,
+                p->T, p->n);
+  if (p->n_txt < 0) return fail(VDA_ERR_INVALID_ARG, "n_txt must be >= 0 (got %d)", p->n_txt);
+  if (p->d_k < 1 || p->d_v < 1)
+    return fail(VDA_ERR_INVALID_ARG, "d_k, d_v must be >= 1 (got %d, %d)", p->d_k, p->d_v);
+  if (!(p->lambda > 0.f) || !isfinite(p->lambda))
+    return fail(VDA_ERR_INVALID_ARG, "lambda must be finite and > 0 (got %g)", (double)p->lambda);
+  if (p->dtype != VDA_DTYPE_F32 && p->dtype != VDA_DTYPE_BF16)
+    return fail(VDA_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
+  if (p->dtype == VDA_DTYPE_F32) {
+    if (p->d_k % 16 || p->d_v % 16 || p->d_k > 128 || p->d_v > 128)
+      return fail(VDA_ERR_UNSUPPORTED,
+                  "float32 path supports d_k, d_v multiples of 16 up to 128 (got %d, %d)", p->d_k,
+                  p->d_v);
+  } else {
+    if (p->d_k != 128 || p->d_v != 128)
+      return fail(VDA_ERR_UNSUPPORTED, "bfloat16 path supports d_k = d_v = 128 (got %d, %d)",
+                  p->d_k, p->d_v);
+  }
+  // Index arithmetic in the kernels: slots and frames fit 32 bits, element
+  // offsets are 64-bit.
+  const long long slots = (long long)p->B * p->H * (p->T + 1);
+  if (slots > 65535LL * 64)
+    return fail(VDA_ERR_UNSUPPORTED, "B*H*(T+1) = %lld is above the supported 4194240", slots);
+  if ((long long)p->B * p->H > 65535)
+    return fail(VDA_ERR_UNSUPPORTED, "B*H = %lld is above 65535", (long long)p->B * p->H);
+  if ((long long)p->B * p->H * p->T > 65535LL * 1024)
+    return fail(VDA_ERR_UNSUPPORTED, "B*H*T is too large");
+  if (p->n > (1 << 24) || p->n_txt > (1 << 24))
+    return fail(VDA_ERR_UNSUPPORTED, "n and n_txt must be <= 2^24");
+  return VDA_OK;
+}
+
+size_t elem_size(const vda_problem& p) { return p.dtype == VDA_DTYPE_BF16 ? 2 : 4; }
+
+struct Sizes {
+  size_t q, k, v, g, kt, vt, o;
+};
+
+Sizes tensor_bytes(const vda_problem& p) {
+  const size_t es = elem_size(p);
+  const size_t fr = (size_t)p.B * p.H * p.T * p.n;
+  const size_t tx = (size_t)p.B * p.H * p.n_txt;
+  return Sizes{fr * p.d_k * es, fr * p.d_k * es, fr * p.d_v * es, fr * p.d_v * es,
+               tx * p.d_k * es, tx * p.d_v * es, fr * p.d_v * es};
+}
+
+vda_status check_pointers(const vda_problem& p, const void* Q, const void* K, const void* V,
+                          const void* G, const void* Kt, const void* Vt, const void* O) {
+  const void* req[5] = {Q, K, V, G, O};
+  const char* names[5] = {"Q", "K", "V", "G", "O"};
+  for (int i = 0; i < 5; ++i) {
+    if (!req[i]) return fail(VDA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(req[i])) return fail(VDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  if (p.n_txt > 0) {
+    if (!Kt || !Vt) return fail(VDA_ERR_INVALID_ARG, "K_txt / V_txt NULL with n_txt = %d", p.n_txt);
+    if (!aligned16(Kt) || !aligned16(Vt))
+      return fail(VDA_ERR_INVALID_ARG, "K_txt / V_txt not 16-byte aligned");
+  }
+  return VDA_OK;
+}
+
+template <typename TIn>
+vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const void* V,
+                       const void* G, const void* Kt, const void* Vt, void* O, char* ws,
+                       cudaStream_t st, float* S_fwd, float* S_bwd, cudaEvent_t const* ev) {
+  const vda::Layout L = vda::make_layout(p);
+  unsigned* err = reinterpret_cast<unsigned*>(ws + L.err);
+  float* M = reinterpret_cast<float*>(ws + L.M);
+  float* C = reinterpret_cast<float*>(ws + L.C);
+  float* SF = S_fwd ? S_fwd : reinterpret_cast<float*>(ws + L.SF);
+  float* SB = S_bwd ? S_bwd : reinterpret_cast<float*>(ws + L.SB);
+  cudaError_t e = cudaMemsetAsync(err, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  const TIn* q = static_cast<const TIn*>(Q);
+  const TIn* k = static_cast<const TIn*>(K);
+  const TIn* v = static_cast<const TIn*>(V);
+  const TIn* g = static_cast<const TIn*>(G);
+  const TIn* kt = static_cast<const TIn*>(Kt);
+  const TIn* vt = static_cast<const TIn*>(Vt);
+  auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
+  if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_gram_simt<TIn>(p, k, v, kt, vt, M, C, st)) != cudaSuccess)
+    return cuda_fail(e, "gram launch");
+  if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_factor_simt(p, M, C, err, st)) != cudaSuccess)
+    return cuda_fail(e, "factor launch");
+  if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_scan_simt(p, M, C, SF, SB, st)) != cudaSuccess)
+    return cuda_fail(e, "scan launch");
+  if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_readout_simt<TIn>(p, q, g, SF, SB, static_cast<TIn*>(O), st)) != cudaSuccess)
+    return cuda_fail(e, "readout launch");
+  if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "event record");
+  return VDA_OK;
+}
+
+vda_status forward_impl(const vda_problem* p, const void* Q, const void* K, const void* V,
+                        const void* G, const void* Kt, const void* Vt, void* O, void* workspace,
+                        size_t workspace_bytes, void* stream, float* S_fwd, float* S_bwd,
+                        cudaEvent_t const* ev = nullptr) {
+  g_msg[0] = 0;
+  vda_status s = check_problem(p);
+  if (s != VDA_OK) return s;
+  if ((s = check_pointers(*p, Q, K, V, G, Kt, Vt, O)) != VDA_OK) return s;
+  const vda::Layout L = vda::make_layout(*p);
+  if (!workspace) return fail(VDA_ERR_WORKSPACE, "workspace is NULL");
+  if ((uintptr_t)workspace & 255u) return fail(VDA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(VDA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+  if ((S_fwd && !aligned16(S_fwd)) || (S_bwd && !aligned16(S_bwd)))
+    return fail(VDA_ERR_INVALID_ARG, "S_fwd / S_bwd not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (p->dtype == VDA_DTYPE_BF16)
+    return run_forward<__nv_bfloat16>(*p, Q, K, V, G, Kt, Vt, O, ws, st, S_fwd, S_bwd, ev);
+  return run_forward<float>(*p, Q, K, V, G, Kt, Vt, O, ws, st, S_fwd, S_bwd, ev);
+}
+
+}  // namespace
+
+extern "C" {
+
+vda_status vda_workspace_size(const vda_problem* p, size_t* bytes) {
+  g_msg[0] = 0;
+  vda_status s = check_problem(p);
+  if (s != VDA_OK) return s;
+  if (!bytes) return fail(VDA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = vda::make_layout(*p).total;
+  return VDA_OK;
+}
+
+vda_status vda_forward(const vda_problem* p, const void* Q, const void* K, const void* V,
+                       const void* G, const void* K_txt, const void* V_txt, void* O,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_impl(p, Q, K, V, G, K_txt, V_txt, O, workspace, workspace_bytes, stream, nullptr,
+                      nullptr);
+}
+
+vda_status vda_forward_states(const vda_problem* p, const void* Q, const void* K, const void* V,
+                              const void* G, const void* K_txt, const void* V_txt, void* O,
+                              void* workspace, size_t workspace_bytes, void* stream,
+                              float* S_fwd, float* S_bwd) {
+  if (!S_fwd || !S_bwd) return fail(VDA_ERR_INVALID_ARG, "S_fwd / S_bwd is NULL");
+  return forward_impl(p, Q, K, V, G, K_txt, V_txt, O, workspace, workspace_bytes, stream, S_fwd,
+                      S_bwd);
+}
+
+vda_status vda_forward_timed(const vda_problem* p, const void* Q, const void* K, const void* V,
+                             const void* G, const void* K_txt, const void* V_txt, void* O,
+                             void* workspace, size_t workspace_bytes, void* stream,
+                             void* const* events, int n_events) {
+  if (!events || n_events != VDA_TIMED_EVENTS)
+    return fail(VDA_ERR_INVALID_ARG, "events must hold %d cudaEvent_t handles", VDA_TIMED_EVENTS);
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return fail(VDA_ERR_INVALID_ARG, "events[%d] is NULL", i);
+  return forward_impl(p, Q, K, V, G, K_txt, V_txt, O, workspace, workspace_bytes, stream, nullptr,
+                      nullptr, reinterpret_cast<cudaEvent_t const*>(events));
+}
+
+vda_status vda_host_workspace_size(const vda_problem* p, size_t* bytes) {
+  g_msg[0] = 0;
+  vda_status s = check_problem(p);
+  if (s != VDA_OK) return s;
+  if (!bytes) return fail(VDA_ERR_INVALID_ARG, "bytes is NULL");
+  const Sizes z = tensor_bytes(*p);
+  size_t off = 0;
+  const size_t parts[7] = {z.q, z.k, z.v, z.g, z.kt, z.vt, z.o};
+  for (size_t b : parts) off = vda::align_up(off + b, 256);
+  *bytes = off + vda::make_layout(*p).total;
+  return VDA_OK;
+}
+
+vda_status vda_forward_host(const vda_problem* p, const void* Q, const void* K, const void* V,
+                            const void* G, const void* K_txt, const void* V_txt, void* O,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  g_msg[0] = 0;
+  vda_status s = check_problem(p);
+  if (s != VDA_OK) return s;
+  if ((s = check_pointers(*p, Q, K, V, G, K_txt, V_txt, O)) != VDA_OK) return s;
+  size_t need = 0;
+  vda_host_workspace_size(p, &need);
+  if (!workspace) return fail(VDA_ERR_WORKSPACE, "workspace is NULL");
+  if ((uintptr_t)workspace & 255u) return fail(VDA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (workspace_bytes < need)
+    return fail(VDA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  const Sizes z = tensor_bytes(*p);
+  char* base = static_cast<char*>(workspace);
+  const void* src[6] = {Q, K, V, G, K_txt, V_txt};
+  const size_t len[6] = {z.q, z.k, z.v, z.g, z.kt, z.vt};
+  void* dev[7];
+  size_t off = 0;
+  for (int i = 0; i < 6; ++i) {
+    dev[i] = base + off;
+    off = vda::align_up(off + len[i], 256);
+  }
+  dev[6] = base + off;
+  off = vda::align_up(off + z.o, 256);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < 6; ++i) {
+    if (len[i] == 0) continue;
+    cudaError_t e = cudaMemcpyAsync(dev[i], src[i], len[i], cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  }
+  s = forward_impl(p, dev[0], dev[1], dev[2], dev[3], p->n_txt ? dev[4] : nullptr,
+                   p->n_txt ? dev[5] : nullptr, dev[6], base + off, workspace_bytes - off, stream,
+                   nullptr, nullptr);
+  if (s != VDA_OK) return s;
+  cudaError_t e = cudaMemcpyAsync(O, dev[6], z.o, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  return vda_sync_status(base + off, stream);
+}
+
+vda_status vda_sync_status(void* workspace, void* stream) {
+  g_msg[0] = 0;
+  if (!workspace) return fail(VDA_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  if (word) {
+    e = cudaMemset(workspace, 0, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  }
+  if (word & vda::kDevErrNotSpd) return fail(VDA_ERR_NOT_SPD, "a Cholesky pivot was not positive");
+  if (word & vda::kDevErrTimeout) return fail(VDA_ERR_TIMEOUT, "a bounded device wait gave up");
+  return VDA_OK;
+}
+
+const char* vda_status_string(vda_status s) {
+  switch (s) {
+    case VDA_OK: return "VDA_OK";
+    case VDA_ERR_INVALID_ARG: return "VDA_ERR_INVALID_ARG";
+    case VDA_ERR_UNSUPPORTED: return "VDA_ERR_UNSUPPORTED";
+    case VDA_ERR_WORKSPACE: return "VDA_ERR_WORKSPACE";
+    case VDA_ERR_CUDA: return "VDA_ERR_CUDA";
+    case VDA_ERR_NOT_SPD: return "VDA_ERR_NOT_SPD";
+    case VDA_ERR_TIMEOUT: return "VDA_ERR_TIMEOUT";
+  }
+  return "VDA_ERR_UNKNOWN";
+}
+
+const char* vda_last_error(void) { return g_msg; }
+
+}  // extern "C"

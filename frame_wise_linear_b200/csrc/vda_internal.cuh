@@ -1,0 +1,58 @@
+// Internal declarations shared by the kernels and the host API of libvda.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "vda.h"
+
+namespace vda {
+
+// Bits of the device error word (first 4 bytes of the workspace).
+enum : unsigned {
+  kDevErrNotSpd = 1u,    // a Cholesky pivot was <= 0 or not finite
+  kDevErrTimeout = 2u,   // a bounded wait gave up
+};
+
+// Workspace carve-up.  Slots: one per (b, h, t) with t = 0 for the text and
+// t = 1..T for the frames, slot = (b * H + h) * (T + 1) + t.
+//   err   : 256 bytes, the error word and reserved space
+//   M     : per slot, d_k x d_k float  (Gram A_t on the way, then lambda A_t^{-1})
+//   C     : per slot, d_k x d_v float  (B_t on the way, then A_t^{-1} B_t; S_0 at t = 0)
+//   SF,SB : per frame (b, h, t), d_k x d_v float
+struct Layout {
+  size_t err, M, C, SF, SB, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline Layout make_layout(const vda_problem& p) {
+  const size_t slots = (size_t)p.B * p.H * (p.T + 1);
+  const size_t frames = (size_t)p.B * p.H * p.T;
+  Layout L;
+  size_t off = 0;
+  L.err = off;  off += 256;
+  L.M = off;    off = align_up(off + slots * p.d_k * p.d_k * sizeof(float), 256);
+  L.C = off;    off = align_up(off + slots * p.d_k * p.d_v * sizeof(float), 256);
+  L.SF = off;   off = align_up(off + frames * p.d_k * p.d_v * sizeof(float), 256);
+  L.SB = off;   off = align_up(off + frames * p.d_k * p.d_v * sizeof(float), 256);
+  L.total = off;
+  return L;
+}
+
+// Launchers of the float32 SIMT path (vda_simt.cu).  All return the launch
+// error (cudaSuccess when enqueued).
+template <typename TIn>
+cudaError_t launch_gram_simt(const vda_problem& p, const TIn* K, const TIn* V, const TIn* Kt,
+                             const TIn* Vt, float* A, float* Bm, cudaStream_t st);
+cudaError_t launch_factor_simt(const vda_problem& p, float* M, float* C, unsigned* err,
+                               cudaStream_t st);
+cudaError_t launch_scan_simt(const vda_problem& p, const float* M, const float* C, float* SF,
+                             float* SB, cudaStream_t st);
+template <typename TIn>
+cudaError_t launch_readout_simt(const vda_problem& p, const TIn* Q, const TIn* G,
+                                const float* SF, const float* SB, TIn* O, cudaStream_t st);
+
+}  // namespace vda

@@ -11,7 +11,9 @@ dataset is involved.  The shapes below stand in for that clip's attention
 inputs: a 24 x 42 latent grid (n = 1008 tokens per frame), T = 45 latent
 frames, 32 heads of width 128 and 256 text tokens.
 
-Recipe (per tensor, independent stream ``PCG64(seed * 100 + index)``):
+Recipe (per tensor and per (b, h), an independent stream
+``PCG64(SeedSequence(seed, spawn_key=(tensor index, b, h)))``, so that any head
+can be drawn alone):
   Q, K, K_txt : rows L2-normalised from N(0, 1)
   V, V_txt, G : N(0, 1)  (G ~ N(0, 2), i.e. variance 2, for the mid config)
   ill-conditioned keys: K_t = L2norm(U_t W + 0.05 E), U_t ~ N(0,1) (n x 8,
@@ -79,8 +81,9 @@ WORKLOADS = {
 }
 
 
-def _rng(seed: int, name: str) -> np.random.Generator:
-    return np.random.Generator(np.random.PCG64(seed * 100 + _STREAM[name]))
+def _rng(seed: int, name: str, b: int, h: int) -> np.random.Generator:
+    ss = np.random.SeedSequence(seed, spawn_key=(_STREAM[name], b, h))
+    return np.random.Generator(np.random.PCG64(ss))
 
 
 def _l2norm_rows(x: np.ndarray) -> np.ndarray:
@@ -131,39 +134,87 @@ class Inputs:
         return sum(getattr(self, k).nbytes for k in ("Q", "K", "V", "G", "K_txt", "V_txt"))
 
 
-def _normal(seed: int, name: str, shape, std: float = 1.0) -> np.ndarray:
-    x = _rng(seed, name).standard_normal(size=shape, dtype=np.float32)
+def _normal(seed: int, name: str, b: int, h: int, shape, std: float = 1.0) -> np.ndarray:
+    x = _rng(seed, name, b, h).standard_normal(size=shape, dtype=np.float32)
     if std != 1.0:
         x *= np.float32(std)
     return x
 
 
-def _ill_keys(w: Workload, seed: int) -> np.ndarray:
-    """K_t = L2norm(U_t W + noise * E), W shared over the frames of one (b, h)."""
-    U = _normal(seed, "U", (w.B, w.H, w.T, w.n, w.rank))
-    W = _normal(seed, "W", (w.B, w.H, w.rank, w.d_k))
-    E = _normal(seed, "E", (w.B, w.H, w.T, w.n, w.d_k))
-    K = np.empty((w.B, w.H, w.T, w.n, w.d_k), dtype=np.float32)
-    for b in range(w.B):
-        for h in range(w.H):
-            K[b, h] = np.matmul(U[b, h], W[b, h]) + np.float32(w.noise) * E[b, h]
-    return _l2norm_rows(K)
+NAMES = ("Q", "K", "V", "G", "K_txt", "V_txt")
+
+
+def head_f32(w: Workload, b: int, h: int, seed: int = 0) -> dict:
+    """One (b, h)'s inputs in float32, before any BF16 rounding."""
+    sh_k = (w.T, w.n, w.d_k)
+    sh_v = (w.T, w.n, w.d_v)
+    Q = _l2norm_rows(_normal(seed, "Q", b, h, sh_k))
+    if w.ill_conditioned:
+        U = _normal(seed, "U", b, h, (w.T, w.n, w.rank))
+        W = _normal(seed, "W", b, h, (w.rank, w.d_k))
+        E = _normal(seed, "E", b, h, sh_k)
+        K = _l2norm_rows(np.matmul(U, W) + np.float32(w.noise) * E)
+    else:
+        K = _l2norm_rows(_normal(seed, "K", b, h, sh_k))
+    V = _normal(seed, "V", b, h, sh_v)
+    G = _normal(seed, "G", b, h, sh_v, std=w.g_std)
+    K_txt = _l2norm_rows(_normal(seed, "K_txt", b, h, (w.n_txt, w.d_k)))
+    V_txt = _normal(seed, "V_txt", b, h, (w.n_txt, w.d_v))
+    return dict(Q=Q, K=K, V=V, G=G, K_txt=K_txt, V_txt=V_txt)
+
+
+def head_inputs(w: Workload | str, b: int, h: int, seed: int = 0) -> dict:
+    """One (b, h)'s inputs in storage form (BF16 bits as uint16, or float32)."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    f = head_f32(w, b, h, seed)
+    if w.dtype == DTYPE_BF16:
+        return {k: to_bf16_bits(v) for k, v in f.items()}
+    return {k: np.ascontiguousarray(v, dtype=np.float32) for k, v in f.items()}
+
+
+def head_widened(w: Workload | str, b: int, h: int, seed: int = 0) -> dict:
+    """One (b, h)'s inputs as the exact float64 values the device sees."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    return {k: widen(v, w.dtype) for k, v in head_inputs(w, b, h, seed).items()}
 
 
 def make_inputs(w: Workload | str, seed: int = 0) -> Inputs:
-    """Draw one workload's inputs (host numpy arrays, storage dtype)."""
+    """All of a workload's inputs as host numpy arrays (storage dtype)."""
     if isinstance(w, str):
         w = WORKLOADS[w]
-    sh_k = (w.B, w.H, w.T, w.n, w.d_k)
-    sh_v = (w.B, w.H, w.T, w.n, w.d_v)
-    Q = _l2norm_rows(_normal(seed, "Q", sh_k))
-    K = _ill_keys(w, seed) if w.ill_conditioned else _l2norm_rows(_normal(seed, "K", sh_k))
-    V = _normal(seed, "V", sh_v)
-    G = _normal(seed, "G", sh_v, std=w.g_std)
-    K_txt = _l2norm_rows(_normal(seed, "K_txt", (w.B, w.H, w.n_txt, w.d_k)))
-    V_txt = _normal(seed, "V_txt", (w.B, w.H, w.n_txt, w.d_v))
-    if w.dtype == DTYPE_BF16:
-        conv = to_bf16_bits
-    else:
-        conv = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
-    return Inputs(w, conv(Q), conv(K), conv(V), conv(G), conv(K_txt), conv(V_txt))
+    st = np.uint16 if w.dtype == DTYPE_BF16 else np.float32
+    shapes = dict(Q=(w.T, w.n, w.d_k), K=(w.T, w.n, w.d_k), V=(w.T, w.n, w.d_v), G=(w.T, w.n, w.d_v),
+                  K_txt=(w.n_txt, w.d_k), V_txt=(w.n_txt, w.d_v))
+    out = {k: np.empty((w.B, w.H) + s, dtype=st) for k, s in shapes.items()}
+    for b in range(w.B):
+        for h in range(w.H):
+            for k, v in head_inputs(w, b, h, seed).items():
+                out[k][b, h] = v
+    return Inputs(w, **out)
+
+
+def make_inputs_torch(w: Workload | str, seed: int = 0, device="cuda", pin: bool = False) -> dict:
+    """All inputs as torch tensors on `device` (or pinned host memory), drawn head by head.
+
+    BF16 workloads give torch.bfloat16 tensors holding exactly the bits of
+    ``head_inputs``; the host never holds more than one head at a time
+    unless ``device`` is "cpu".
+    """
+    import torch
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    tdt = torch.bfloat16 if w.dtype == DTYPE_BF16 else torch.float32
+    shapes = dict(Q=(w.T, w.n, w.d_k), K=(w.T, w.n, w.d_k), V=(w.T, w.n, w.d_v), G=(w.T, w.n, w.d_v),
+                  K_txt=(w.n_txt, w.d_k), V_txt=(w.n_txt, w.d_v))
+    kw = dict(pin_memory=True) if (pin and str(device) == "cpu") else {}
+    out = {k: torch.empty((w.B, w.H) + s, dtype=tdt, device=device, **kw) for k, s in shapes.items()}
+    for b in range(w.B):
+        for h in range(w.H):
+            for k, v in head_inputs(w, b, h, seed).items():
+                t = torch.from_numpy(v)
+                if tdt == torch.bfloat16:
+                    t = t.view(torch.int16).view(torch.bfloat16)
+                out[k][b, h].copy_(t)
+    return out

@@ -1,0 +1,148 @@
+/*
+ * vda.h -- C ABI of libvda.so: Video Delta Attention (VDA) forward on B200.
+ *
+ * What is computed.  VDA is the linear branch of the VDN-H3 hybrid video
+ * attention.  The pages describe it in words only:
+ *   - "VDN-MiniMax-H3" (aiezz.com), section 03 (technical principles), item
+ *     "Video Delta Attention", and the same item in section 技术原理 of
+ *     "VDN-MiniMax-H3 OpenVDN 开源的视频生成加速方案" (laicaila.com): the
+ *     token-wise delta rule becomes a frame-wise joint solve through the
+ *     normal equations; non-expansive; no frame-size scaling.
+ *   - same sections, item "text dual-branch injection": the text is written
+ *     once, at initialisation, into both directional states.
+ *   - same sections, item "gate fusion": a content-dependent sigmoid gate.
+ *   - "VDN-H3: ..." (comfyui-wiki.com), section on how Video DeltaNet speeds
+ *     up H3: a bidirectional linear branch with a constant-size state.
+ * The concrete form this library computes, per (batch b, head h):
+ *     A_t = K_t^T K_t + lambda I,   B_t = K_t^T V_t            (t = 1..T)
+ *     S_0 = A_txt^{-1} B_txt        (S_0 = 0 when n_txt == 0)
+ *     S^f_t = A_t^{-1} (lambda S^f_{t-1} + B_t),  S^f_0 = S_0   (t = 1..T)
+ *     S^b_t = A_t^{-1} (lambda S^b_{t+1} + B_t),  S^b_{T+1} = S_0 (t = T..1)
+ *     O_t   = sigmoid(G_t) * (Q_t S^f_t + Q_t S^b_t)            (element-wise)
+ *
+ * Layout.  Every tensor is dense, row-major, contiguous:
+ *     Q, K : [B, H, T, n, d_k]      V, G, O : [B, H, T, n, d_v]
+ *     K_txt: [B, H, n_txt, d_k]     V_txt   : [B, H, n_txt, d_v]
+ *     S_fwd, S_bwd (states)          : [B, H, T, d_k, d_v], float32
+ * Inputs and O share one element type, vda_problem.dtype: float32 or
+ * bfloat16.  The state and every accumulation are float32; O is rounded to
+ * its type with round-to-nearest-even.
+ *
+ * Ownership.  The caller owns every buffer.  Device pointers must be CUDA
+ * device memory of the current device, 16-byte aligned.  The library
+ * allocates nothing and keeps no per-call state between calls; calls on one
+ * stream are ordered, calls on different streams must use different
+ * workspaces.  Every call that takes a stream only enqueues work on it
+ * (asynchronous), except where stated.  `stream` is a cudaStream_t passed as
+ * void* (NULL = the legacy default stream).
+ *
+ * Errors.  Argument errors are found on the host before anything is
+ * enqueued and return VDA_ERR_INVALID_ARG / VDA_ERR_UNSUPPORTED /
+ * VDA_ERR_WORKSPACE; nothing runs in that case.  A launch failure returns
+ * VDA_ERR_CUDA.  Conditions found on the device (a non-positive Cholesky
+ * pivot, which exact arithmetic rules out for lambda > 0; a bounded wait
+ * that ran out) are written to an error word in the workspace, which every
+ * vda_forward* call clears first; vda_sync_status() reads it.  There is no
+ * CPU fallback: without a usable device the calls fail.
+ */
+#ifndef VDA_H_
+#define VDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vda_status {
+  VDA_OK = 0,
+  VDA_ERR_INVALID_ARG = 1,  /* bad size, lambda, null or misaligned pointer */
+  VDA_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels support  */
+  VDA_ERR_WORKSPACE = 3,    /* workspace missing, too small or misaligned   */
+  VDA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed         */
+  VDA_ERR_NOT_SPD = 5,      /* device: a Cholesky pivot was not positive    */
+  VDA_ERR_TIMEOUT = 6       /* device: a bounded wait gave up               */
+} vda_status;
+
+typedef enum vda_dtype { VDA_DTYPE_F32 = 0, VDA_DTYPE_BF16 = 1 } vda_dtype;
+
+/* Problem sizes.  B, H, T, n >= 1; n_txt >= 0.
+ * float32: d_k, d_v multiples of 16 in [16, 128].
+ * bfloat16: d_k = d_v = 128.
+ * lambda: the ridge weight of every frame-wise solve, finite and > 0, one
+ * value shared by all batches, heads, frames and the text (the pages name no
+ * such parameter; one scalar per call is the plainest reading). */
+typedef struct vda_problem {
+  int32_t B, H, T, n, n_txt, d_k, d_v;
+  int32_t dtype; /* vda_dtype */
+  float lambda;
+} vda_problem;
+
+/* Bytes of device workspace vda_forward needs for `p` (written to *bytes).
+ * Host only, enqueues nothing.  Errors: INVALID_ARG / UNSUPPORTED as for
+ * vda_forward. */
+vda_status vda_workspace_size(const vda_problem* p, size_t* bytes);
+
+/* O = VDA(Q, K, V, G, K_txt, V_txt; lambda), the whole forward (both scan
+ * directions and the gated readout), enqueued on `stream`.
+ * Q, K, V, G, O: device pointers, layout above, element type p->dtype.
+ * K_txt, V_txt: device pointers, or NULL when p->n_txt == 0.
+ * workspace: device memory of at least vda_workspace_size() bytes, 256-byte
+ * aligned; its contents on entry do not matter and on return are the
+ * intermediates plus the error word.  Returns once the work is enqueued. */
+vda_status vda_forward(const vda_problem* p, const void* Q, const void* K, const void* V,
+                       const void* G, const void* K_txt, const void* V_txt, void* O,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* As vda_forward, and also writes the per-frame states S^f_t and S^b_t
+ * (float32, [B, H, T, d_k, d_v]) to the device buffers S_fwd, S_bwd.  Used to
+ * check the scan stage on its own. */
+vda_status vda_forward_states(const vda_problem* p, const void* Q, const void* K, const void* V,
+                              const void* G, const void* K_txt, const void* V_txt, void* O,
+                              void* workspace, size_t workspace_bytes, void* stream,
+                              float* S_fwd, float* S_bwd);
+
+/* As vda_forward, and records CUDA events on `stream` around the stages so
+ * a caller can time each kernel on the stream that runs it.  `events` holds
+ * `n_events` cudaEvent_t handles (passed as void*), created by the caller;
+ * events[0] is recorded before the first kernel and events[i] after stage i
+ * (1 = Gram, 2 = factor-and-solve, 3 = scan, 4 = readout).  n_events must be
+ * VDA_TIMED_EVENTS; elapsed time between events i-1 and i is stage i. */
+#define VDA_TIMED_EVENTS 5
+vda_status vda_forward_timed(const vda_problem* p, const void* Q, const void* K, const void* V,
+                             const void* G, const void* K_txt, const void* V_txt, void* O,
+                             void* workspace, size_t workspace_bytes, void* stream,
+                             void* const* events, int n_events);
+
+/* Bytes of device workspace vda_forward_host needs: room for the inputs and
+ * O on the device plus vda_workspace_size(). */
+vda_status vda_host_workspace_size(const vda_problem* p, size_t* bytes);
+
+/* End-to-end call on HOST buffers: copies the inputs host -> device into the
+ * workspace (one cudaMemcpyAsync per tensor), runs vda_forward, copies O
+ * device -> host, all on `stream`, then synchronises `stream` and returns the
+ * device status (as vda_sync_status).  Host buffers should be pinned
+ * (cudaHostAlloc / page-locked) for the copies to be asynchronous.  The same
+ * pointer rules hold, with host pointers in place of device ones. */
+vda_status vda_forward_host(const vda_problem* p, const void* Q, const void* K, const void* V,
+                            const void* G, const void* K_txt, const void* V_txt, void* O,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of
+ * `workspace`: VDA_OK, VDA_ERR_NOT_SPD or VDA_ERR_TIMEOUT (first one set),
+ * or VDA_ERR_CUDA if the stream reports an error.  Blocking. */
+vda_status vda_sync_status(void* workspace, void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* vda_status_string(vda_status s);
+
+/* A thread-local message describing the last error returned on this host
+ * thread ("" if none).  Valid until the next call on the same thread. */
+const char* vda_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDA_H_ */

@@ -1,0 +1,144 @@
+"""The C ABI on the host: symbols, argument checks, error codes (no GPU needed).
+
+Every call here fails its host-side checks before anything is enqueued, so no
+device pointer is ever dereferenced; the single call that passes the checks
+runs only where no CUDA device exists and must then fail loudly.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from frame_wise_linear_b200 import build, vda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return vda.load()
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(vda_[a-z_0-9]+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_symbols()
+    assert declared, "no entry points found in include/*.h"
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert declared == set(vda.SYMBOLS) | (declared - set(vda.SYMBOLS))
+    for name in vda.SYMBOLS:
+        assert name in declared, f"binding exposes {name}, which include/ does not declare"
+
+
+def _p(**kw):
+    base = dict(B=1, H=2, T=3, n=64, n_txt=8, d_k=128, d_v=128, dtype=vda.VDA_DTYPE_BF16, lam=1.0)
+    base.update(kw)
+    return vda.make_problem(**base)
+
+
+def test_workspace_size_valid(lib):
+    p = _p()
+    nb = vda.vda_workspace_size(p)
+    slots = 1 * 2 * 4
+    assert nb >= 256 + slots * 128 * 128 * 4 * 2 + 6 * 128 * 128 * 4 * 2
+    assert vda.vda_host_workspace_size(p) > nb
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(lam=0.0), vda.VDA_ERR_INVALID_ARG),
+    (dict(lam=-1.0), vda.VDA_ERR_INVALID_ARG),
+    (dict(lam=float("nan")), vda.VDA_ERR_INVALID_ARG),
+    (dict(lam=float("inf")), vda.VDA_ERR_INVALID_ARG),
+    (dict(B=0), vda.VDA_ERR_INVALID_ARG),
+    (dict(T=0), vda.VDA_ERR_INVALID_ARG),
+    (dict(n=0), vda.VDA_ERR_INVALID_ARG),
+    (dict(n_txt=-1), vda.VDA_ERR_INVALID_ARG),
+    (dict(dtype=7), vda.VDA_ERR_INVALID_ARG),
+    (dict(d_k=64, d_v=64), vda.VDA_ERR_UNSUPPORTED),            # bf16 needs 128
+    (dict(dtype=vda.VDA_DTYPE_F32, d_k=24), vda.VDA_ERR_UNSUPPORTED),
+    (dict(dtype=vda.VDA_DTYPE_F32, d_k=256), vda.VDA_ERR_UNSUPPORTED),
+    (dict(B=70000), vda.VDA_ERR_UNSUPPORTED),
+])
+def test_bad_problem_rejected(lib, kw, status):
+    p = _p(**kw)
+    out = ctypes.c_size_t(0)
+    s = lib.vda_workspace_size(ctypes.byref(p), ctypes.byref(out))
+    assert s == status, vda.vda_last_error()
+    assert vda.vda_last_error()
+    # and vda_forward rejects it before enqueuing anything
+    s = vda.vda_forward(p, 16, 16, 16, 16, 16, 16, 16, 256, stream=0, workspace_bytes=1 << 40, check=False)
+    assert s == status
+
+
+def test_null_and_misaligned_pointers(lib):
+    p = _p()
+    ok = 1 << 20
+    args = [ok] * 7
+    for i in range(7):
+        a = list(args)
+        a[i] = 0
+        s = vda.vda_forward(p, *a, ok, stream=0, workspace_bytes=1 << 40, check=False)
+        assert s == vda.VDA_ERR_INVALID_ARG, (i, vda.vda_last_error())
+        a[i] = ok + 8
+        s = vda.vda_forward(p, *a, ok, stream=0, workspace_bytes=1 << 40, check=False)
+        assert s == vda.VDA_ERR_INVALID_ARG, (i, vda.vda_last_error())
+
+
+def test_text_pointers_may_be_null_without_text(lib):
+    p = _p(n_txt=0)
+    ok = 1 << 20
+    # passes the pointer checks, fails on the workspace size instead
+    s = vda.vda_forward(p, ok, ok, ok, ok, None, None, ok, ok, stream=0, workspace_bytes=16, check=False)
+    assert s == vda.VDA_ERR_WORKSPACE
+
+
+def test_workspace_checks(lib):
+    p = _p()
+    ok = 1 << 20
+    need = vda.vda_workspace_size(p)
+    s = vda.vda_forward(p, *([ok] * 7), None, stream=0, workspace_bytes=need, check=False)
+    assert s == vda.VDA_ERR_WORKSPACE
+    s = vda.vda_forward(p, *([ok] * 7), ok + 16, stream=0, workspace_bytes=need, check=False)
+    assert s == vda.VDA_ERR_WORKSPACE
+    s = vda.vda_forward(p, *([ok] * 7), ok, stream=0, workspace_bytes=need - 1, check=False)
+    assert s == vda.VDA_ERR_WORKSPACE
+    s = vda.vda_forward_states(p, *([ok] * 7), ok, None, ok, stream=0, workspace_bytes=need, check=False)
+    assert s == vda.VDA_ERR_INVALID_ARG
+    need_h = vda.vda_host_workspace_size(p)
+    s = vda.vda_forward_host(p, *([ok] * 7), ok, stream=0, workspace_bytes=need_h - 1, check=False)
+    assert s == vda.VDA_ERR_WORKSPACE
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert vda.vda_status_string(code).startswith("VDA_")
+    assert vda.vda_status_string(99) == "VDA_ERR_UNKNOWN"
+
+
+def _has_cuda():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.mark.skipif(_has_cuda(), reason="only meaningful where no CUDA device exists")
+def test_no_device_fails_loudly(lib):
+    """With every check passed and no GPU, the call reports a CUDA error: no CPU fallback."""
+    p = _p()
+    ok = 1 << 20
+    need = vda.vda_workspace_size(p)
+    s = vda.vda_forward(p, *([ok] * 7), ok, stream=0, workspace_bytes=need, check=False)
+    assert s == vda.VDA_ERR_CUDA
