@@ -41,7 +41,7 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 # Kernel of each stage and the source file that defines it (for ncu traffic lookups).
 STAGE_SOURCES = {
-    "gram": "frame_wise_linear_b200/csrc/vda_simt.cu",
+    "gram": "frame_wise_linear_b200/csrc/vda_gram_tc.cu",
     "factor": "frame_wise_linear_b200/csrc/vda_simt.cu",
     "scan": "frame_wise_linear_b200/csrc/vda_simt.cu",
     "readout": "frame_wise_linear_b200/csrc/vda_simt.cu",
@@ -322,6 +322,10 @@ def run_b200(args, w):
     sampler.start()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(vda.VDA_TIMED_EVENTS)]
           for _ in range(args.steps)]
+    for e_step in ev:          # torch creates the CUDA event on its first record
+        for e in e_step:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     if pg:

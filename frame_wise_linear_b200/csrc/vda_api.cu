@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <type_traits>
+
 #include "vda_internal.cuh"
 
 namespace {
@@ -112,8 +114,13 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
   const TIn* vt = static_cast<const TIn*>(Vt);
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
   if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "event record");
-  if ((e = vda::launch_gram_simt<TIn>(p, k, v, kt, vt, M, C, st)) != cudaSuccess)
-    return cuda_fail(e, "gram launch");
+  if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
+    if ((e = vda::launch_gram_tc(p, k, v, kt, vt, M, C, err, st)) != cudaSuccess)
+      return cuda_fail(e, "gram launch");
+  } else {
+    if ((e = vda::launch_gram_simt<TIn>(p, k, v, kt, vt, M, C, st)) != cudaSuccess)
+      return cuda_fail(e, "gram launch");
+  }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
   if ((e = vda::launch_factor_simt(p, M, C, err, st)) != cudaSuccess)
     return cuda_fail(e, "factor launch");

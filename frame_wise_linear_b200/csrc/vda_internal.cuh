@@ -1,6 +1,7 @@
 // Internal declarations shared by the kernels and the host API of libvda.so.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -54,5 +55,20 @@ cudaError_t launch_scan_simt(const vda_problem& p, const float* M, const float* 
 template <typename TIn>
 cudaError_t launch_readout_simt(const vda_problem& p, const TIn* Q, const TIn* G,
                                 const float* SF, const float* SB, TIn* O, cudaStream_t st);
+
+// Tensor-core Gram (vda_gram_tc.cu): bf16 inputs, d_k = d_v = 128.  Writes
+// the same A and B slots as launch_gram_simt.
+cudaError_t launch_gram_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                           const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* A, float* Bm,
+                           unsigned* err, cudaStream_t st);
+
+// Tensor-core readout (vda_readout_tc.cu): bf16 Q, G, O, d_k = d_v = 128.
+cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,
+                              const float* SF, const float* SB, __nv_bfloat16* O, unsigned* err,
+                              cudaStream_t st);
+
+// TMA descriptor of a [items][rows][128] bf16 tensor, boxes of 64 features x
+// box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
+bool make_bf16_rows_map(CUtensorMap* m, const void* ptr, int rows, int items, int box_rows);
 
 }  // namespace vda
