@@ -128,8 +128,13 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
   if ((e = vda::launch_scan_simt(p, M, C, SF, SB, st)) != cudaSuccess)
     return cuda_fail(e, "scan launch");
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "event record");
-  if ((e = vda::launch_readout_simt<TIn>(p, q, g, SF, SB, static_cast<TIn*>(O), st)) != cudaSuccess)
-    return cuda_fail(e, "readout launch");
+  if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
+    if ((e = vda::launch_readout_tc(p, q, g, SF, SB, static_cast<TIn*>(O), err, st)) != cudaSuccess)
+      return cuda_fail(e, "readout launch");
+  } else {
+    if ((e = vda::launch_readout_simt<TIn>(p, q, g, SF, SB, static_cast<TIn*>(O), st)) != cudaSuccess)
+      return cuda_fail(e, "readout launch");
+  }
   if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "event record");
   return VDA_OK;
 }

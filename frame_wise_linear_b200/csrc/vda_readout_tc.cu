@@ -1,0 +1,318 @@
+// Gated readout on tcgen05 tensor cores:
+//     O_t = sigmoid(G_t) * (Q_t (S^f_t + S^b_t))
+// ("VDN-MiniMax-H3" (aiezz.com), section 03, gate fusion item: a
+// content-dependent sigmoid gate on the branch output).  bfloat16 Q, G, O,
+// d = 128; the states are float32.
+//
+// Precision: Q is exact in bf16; S = S^f + S^b is split as S_hi + S_lo (two
+// bf16 terms, about 16 significant bits) and the product takes two MMA passes,
+// Q S_hi + Q S_lo, accumulated in float32.
+//
+// Design (persistent, one CTA per SM, 6 warps), work = 128-row tiles of every
+// frame, a contiguous range of tiles per CTA:
+//   warp 0      TMA producer: Q tiles (3-stage ring) and G tiles (2-stage ring),
+//               each tile as two 64-feature boxes with the 128-byte swizzle.
+//   warp 1      TMEM (2 x 128 columns) and the MMAs (one thread).
+//   warps 2..5  at each new frame: S = S^f + S^b split into bf16 hi/lo in
+//               shared memory (the MMA B operand); per tile: TMEM -> registers,
+//               gate from the G tile, O written over the G tile in shared
+//               memory, then one TMA store of the O tile.
+// Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
+// bit of the error word and the CTA winds down.
+#include "sm100.cuh"
+#include "vda_internal.cuh"
+
+namespace vda {
+namespace {
+
+using namespace sm100;
+
+constexpr int kQStages = 3;
+constexpr int kGStages = 2;
+constexpr int kRows = 128;                   // tokens per tile
+constexpr int kBox = kRows * 64 * 2;         // 128 rows x 64 features bf16: 16 KB
+constexpr int kTile = 2 * kBox;              // 32 KB
+constexpr int kSig = 2 * kTile;              // S_hi and S_lo, 32 KB each
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
+
+struct ReadoutTcParams {
+  CUtensorMap mQ, mG, mO;
+  const float* SF;
+  const float* SB;
+  unsigned* err;
+  int units;       // B*H*T frames
+  int tiles_per_unit;
+};
+
+struct Shared {
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t g_full[kGStages], g_empty[kGStages];
+  uint64_t t_full[2], t_empty[2];
+  uint64_t sig_full, sig_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool aborted(Shared& sh) { return *reinterpret_cast<volatile int*>(&sh.abort) != 0; }
+__device__ __forceinline__ void set_abort(Shared& sh, unsigned* err) {
+  atomicOr(err, kDevErrTimeout);
+  *reinterpret_cast<volatile int*>(&sh.abort) = 1;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_constant__ ReadoutTcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sig = base;                              // S_hi | S_lo
+  uint8_t* qbuf = base + kSig;                      // kQStages tiles
+  uint8_t* gbuf = qbuf + kQStages * kTile;          // kGStages tiles (G in, O out)
+  Shared& sh = *reinterpret_cast<Shared*>(gbuf + kGStages * kTile);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const long long total = (long long)p.units * p.tiles_per_unit;
+  const int t_begin = (int)(total * blockIdx.x / gridDim.x);
+  const int t_end = (int)(total * (blockIdx.x + 1) / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&sh.q_full[i], 1);
+      mbar_init(&sh.q_empty[i], 1);
+    }
+    for (int i = 0; i < kGStages; ++i) {
+      mbar_init(&sh.g_full[i], 1);
+      mbar_init(&sh.g_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.t_full[i], 1);
+      mbar_init(&sh.t_empty[i], 128);
+    }
+    mbar_init(&sh.sig_full, 128);
+    mbar_init(&sh.sig_empty, 1);
+    mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.mQ);
+    tma_prefetch_desc(&p.mG);
+    tma_prefetch_desc(&p.mO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int qs = 0, gs = 0;
+      uint32_t qph = 0, gph = 0;
+      int q_issued = 0, g_issued = 0;
+      for (int tile = t_begin; tile < t_end && !aborted(sh); ++tile) {
+        const int u = tile / p.tiles_per_unit;
+        const int y = (tile % p.tiles_per_unit) * kRows;
+        if (!mbar_wait(&sh.q_empty[qs], qph ^ 1)) {
+          set_abort(sh, p.err);
+          break;
+        }
+        mbar_expect_tx(&sh.q_full[qs], kTile);
+        tma_load_3d(qbuf + qs * kTile, &p.mQ, &sh.q_full[qs], 0, y, u, pol);
+        tma_load_3d(qbuf + qs * kTile + kBox, &p.mQ, &sh.q_full[qs], 64, y, u, pol);
+        ++q_issued;
+        if (++qs == kQStages) { qs = 0; qph ^= 1; }
+        if (!mbar_wait(&sh.g_empty[gs], gph ^ 1)) {
+          set_abort(sh, p.err);
+          break;
+        }
+        mbar_expect_tx(&sh.g_full[gs], kTile);
+        tma_load_3d(gbuf + gs * kTile, &p.mG, &sh.g_full[gs], 0, y, u, pol);
+        tma_load_3d(gbuf + gs * kTile + kBox, &p.mG, &sh.g_full[gs], 64, y, u, pol);
+        ++g_issued;
+        if (++gs == kGStages) { gs = 0; gph ^= 1; }
+      }
+      if (aborted(sh)) {  // let the loads still in flight land before exit
+        for (int c = q_issued > kQStages ? q_issued - kQStages : 0; c < q_issued; ++c)
+          mbar_wait(&sh.q_full[c % kQStages], (c / kQStages) & 1);
+        for (int c = g_issued > kGStages ? g_issued - kGStages : 0; c < g_issued; ++c)
+          mbar_wait(&sh.g_full[c % kGStages], (c / kGStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int qs = 0, tb = 0;
+      uint32_t qph = 0, tph = 0, sph = 0;
+      int cur_u = -1;
+      const uint32_t qaddr = smem_u32(qbuf);
+      const uint32_t saddr = smem_u32(sig);
+      for (int tile = t_begin; tile < t_end && !aborted(sh); ++tile) {
+        const int u = tile / p.tiles_per_unit;
+        if (u != cur_u) {
+          if (!mbar_wait(&sh.sig_full, sph)) { set_abort(sh, p.err); break; }
+          sph ^= 1;
+          cur_u = u;
+        }
+        if (!mbar_wait(&sh.t_empty[tb], tph ^ 1)) { set_abort(sh, p.err); break; }
+        if (!mbar_wait(&sh.q_full[qs], qph)) { set_abort(sh, p.err); break; }
+        tc_fence_after();
+        const uint32_t d = tmem + tb * 128;
+        const uint32_t qa = qaddr + qs * kTile;
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            // A: Q tile, K-major; 16 features = 32 bytes inside a 128-byte row.
+            const uint64_t a = smem_desc(qa + (k / 4) * kBox + (k % 4) * 32, 16, 1024, kSwizzle128B);
+            // B: S_hi or S_lo, MN-major; 16 rows of 128 bytes per k-step,
+            // 64-column blocks 16 KB apart.
+            const uint64_t b = smem_desc(saddr + pass * kTile + k * 16 * 128, kBox, 1024, kSwizzle128B);
+            mma_bf16_ss(d, a, b, kIdesc, (pass | k) ? 1u : 0u);
+          }
+        }
+        mma_commit(&sh.q_empty[qs]);
+        mma_commit(&sh.t_full[tb]);
+        const bool last_of_unit = (tile + 1 == t_end) || ((tile + 1) / p.tiles_per_unit != u);
+        if (last_of_unit) mma_commit(&sh.sig_empty);
+        if (++qs == kQStages) { qs = 0; qph ^= 1; }
+        tb ^= 1;
+        if (tb == 0) tph ^= 1;
+      }
+      mma_commit(&sh.drain);
+      mbar_wait(&sh.drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ S prep + epilogue
+    const int et = threadIdx.x - 64;          // 0..127
+    const int quarter = warp % 4;
+    const int row = quarter * 32 + lane;      // tile row this thread owns in TMEM
+    int gs = 0, tb = 0, cur_u = -1;
+    uint32_t gph = 0, tph = 0, seph = 0;
+    for (int tile = t_begin; tile < t_end; ++tile) {
+      const int u = tile / p.tiles_per_unit;
+      const int y = (tile % p.tiles_per_unit) * kRows;
+      if (__any_sync(0xffffffffu, aborted(sh))) break;
+      if (u != cur_u) {
+        const bool ok = mbar_wait(&sh.sig_empty, seph ^ 1);
+        if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
+        seph ^= 1;
+        // Row `et` of S = S^f + S^b, split into hi/lo bf16, MN-major swizzled.
+        const float4* f = reinterpret_cast<const float4*>(p.SF + ((size_t)u * 128 + et) * 128);
+        const float4* b = reinterpret_cast<const float4*>(p.SB + ((size_t)u * 128 + et) * 128);
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {   // 8 columns per step
+          const float4 f0 = __ldg(f + 2 * c), f1 = __ldg(f + 2 * c + 1);
+          const float4 b0 = __ldg(b + 2 * c), b1 = __ldg(b + 2 * c + 1);
+          const float x[8] = {f0.x + b0.x, f0.y + b0.y, f0.z + b0.z, f0.w + b0.w,
+                              f1.x + b1.x, f1.y + b1.y, f1.z + b1.z, f1.w + b1.w};
+          float hi[8], lo[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
+            lo[i] = x[i] - hi[i];
+          }
+          const uint32_t off = (c / 8) * kBox + sw128(et, c % 8);
+          *reinterpret_cast<uint4*>(sig + off) =
+              make_uint4(pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]),
+                         pack_bf16(hi[6], hi[7]));
+          *reinterpret_cast<uint4*>(sig + kTile + off) =
+              make_uint4(pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]),
+                         pack_bf16(lo[6], lo[7]));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&sh.sig_full);
+        cur_u = u;
+      }
+      bool ok = mbar_wait(&sh.t_full[tb], tph);
+      ok = ok && mbar_wait(&sh.g_full[gs], gph);
+      if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
+      tc_fence_after();
+      uint8_t* gt = gbuf + gs * kTile;
+      const uint32_t taddr = tmem + tb * 128 + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {           // 32 output columns per step
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_ld_wait();
+        uint8_t* rowp = gt + (c / 2) * kBox;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {          // 8 columns = one 16-byte chunk
+          const uint32_t off = sw128(row, (c % 2) * 4 + q);
+          const uint4 gv = *reinterpret_cast<const uint4*>(rowp + off);
+          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+          uint32_t ow[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(&gw[e]);
+            const float g0 = __low2float(g2), g1 = __high2float(g2);
+            const float d0 = __uint_as_float(r[q * 8 + 2 * e]), d1 = __uint_as_float(r[q * 8 + 2 * e + 1]);
+            ow[e] = pack_bf16(__fdividef(d0, 1.f + __expf(-g0)), __fdividef(d1, 1.f + __expf(-g1)));
+          }
+          *reinterpret_cast<uint4*>(rowp + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sh.t_empty[tb]);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (et == 0) {
+        tma_store_3d(&p.mO, gt, 0, y, u);
+        tma_store_3d(&p.mO, gt + kBox, 64, y, u);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(&sh.g_empty[gs]);
+      }
+      if (++gs == kGStages) { gs = 0; gph ^= 1; }
+      tb ^= 1;
+      if (tb == 0) tph ^= 1;
+    }
+    if (et == 0) bulk_wait<0>();               // O stores complete before exit
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,
+                              const float* SF, const float* SB, __nv_bfloat16* O, unsigned* err,
+                              cudaStream_t st) {
+  ReadoutTcParams prm;
+  memset(&prm, 0, sizeof(prm));
+  const int units = p.B * p.H * p.T;
+  if (!make_bf16_rows_map(&prm.mQ, Q, p.n, units, kRows) || !make_bf16_rows_map(&prm.mG, G, p.n, units, kRows) ||
+      !make_bf16_rows_map(&prm.mO, O, p.n, units, kRows))
+    return cudaErrorInvalidValue;
+  prm.SF = SF;
+  prm.SB = SB;
+  prm.err = err;
+  prm.units = units;
+  prm.tiles_per_unit = (p.n + kRows - 1) / kRows;
+  const size_t smem = 1024 + kSig + (kQStages + kGStages) * kTile + sizeof(Shared);
+  cudaError_t e = cudaFuncSetAttribute(readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tiles = (long long)units * prm.tiles_per_unit;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  readout_tc_kernel<<<grid, kThreads, smem, st>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace vda

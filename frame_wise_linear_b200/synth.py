@@ -72,6 +72,8 @@ WORKLOADS = {
     "mid": Workload("mid", B=1, H=8, T=16, n=256, n_txt=128, d_k=128, d_v=128, dtype=DTYPE_BF16,
                     lam=0.5, g_std=math.sqrt(2.0)),
     "768p": Workload("768p", B=1, H=32, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16, lam=1.0),
+    # The 768p shapes with 8 heads: 372 MB of inputs (above L2) for profiler captures.
+    "768p_h8": Workload("768p_h8", B=1, H=8, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16, lam=1.0),
     "illcond": Workload("illcond", B=1, H=32, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16,
                         lam=0.05, ill_conditioned=True),
     "long45": Workload("long45", B=2, H=32, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16, lam=1.0),
