@@ -163,6 +163,10 @@ vda_status forward_impl(const vda_problem* p, const void* Q, const void* K, cons
 
 }  // namespace
 
+namespace vda {
+void set_error_message(const char* msg) { snprintf(g_msg, sizeof(g_msg), "%s", msg); }
+}  // namespace vda
+
 extern "C" {
 
 vda_status vda_workspace_size(const vda_problem* p, size_t* bytes) {

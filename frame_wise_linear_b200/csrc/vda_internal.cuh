@@ -71,4 +71,7 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
 bool make_bf16_rows_map(CUtensorMap* m, const void* ptr, int rows, int items, int box_rows);
 
+// Replaces the thread-local message vda_last_error() returns (vda_api.cu).
+void set_error_message(const char* msg);
+
 }  // namespace vda

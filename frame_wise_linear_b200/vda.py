@@ -38,6 +38,7 @@ SYMBOLS = (
     "vda_forward_timed",
     "vda_host_workspace_size",
     "vda_forward_host",
+    "vda_forward_noalloc",
     "vda_sync_status",
     "vda_status_string",
     "vda_last_error",
@@ -86,6 +87,8 @@ def load(path: str | None = None):
         lib.vda_forward_states.restype = st
         lib.vda_forward_timed.argtypes = fwd + [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
         lib.vda_forward_timed.restype = st
+        lib.vda_forward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.vda_forward_noalloc.restype = st
         lib.vda_sync_status.argtypes = [vp, vp]
         lib.vda_sync_status.restype = st
         lib.vda_status_string.argtypes = [st]
@@ -197,6 +200,23 @@ def vda_forward_host(problem, Q, K, V, G, K_txt, V_txt, O, workspace, stream=Non
                                 _stream(stream))
     if check:
         _check(s, "vda_forward_host")
+    return s
+
+
+VDA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def vda_forward_noalloc(problem, Q, K, V, G, K_txt, V_txt, O, stream=None, check=True) -> int:
+    """Forward on the library's own static scratch, for callers that cannot allocate.
+
+    Same results as vda_forward; no workspace argument.  Problems needing more
+    than VDA_NOALLOC_SCRATCH_BYTES of workspace are rejected; calls that
+    overlap on the GPU share the scratch and race.
+    """
+    s = load().vda_forward_noalloc(ctypes.byref(problem), _ptr(Q), _ptr(K), _ptr(V), _ptr(G),
+                                   _ptr(K_txt), _ptr(V_txt), _ptr(O), _stream(stream))
+    if check:
+        _check(s, "vda_forward_noalloc")
     return s
 
 

@@ -129,6 +129,38 @@ vda_status vda_forward_host(const vda_problem* p, const void* Q, const void* K, 
                             const void* G, const void* K_txt, const void* V_txt, void* O,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Forward for callers that cannot allocate device memory.  Some callers own
+ * no device allocator of their own or may not call one: code running under a
+ * framework whose memory manager owns the whole device (a caching allocator,
+ * or a fixed per-process budget that cudaMalloc would overrun), and callers on
+ * a latency-critical path, where cudaMalloc/cudaFree would synchronise the
+ * device.  They can neither hand vda_forward a workspace nor let the library
+ * allocate one.
+ * This call computes exactly what vda_forward computes, but its workspace is
+ * a scratch array inside the library: a file-scope device array of
+ * VDA_NOALLOC_SCRATCH_BYTES (64 MiB) that every GPU which loads the library
+ * holds until the process exits.  It allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.  The caller still owns Q, K, V, G,
+ * K_txt, V_txt and O (device pointers, same rules as vda_forward).
+ * Limits and caveats:
+ *   - problems whose vda_workspace_size() exceeds the scratch are rejected
+ *     with VDA_ERR_WORKSPACE before anything is enqueued (for example the
+ *     mid workload, 8 heads x 16 frames, fits; 32 heads x 45 frames does not);
+ *   - the first call on a device looks up the scratch's device address (with
+ *     that device current); make that first call before any stream capture;
+ *   - every call on a device shares the one scratch, which keeps the last
+ *     call's contents (each call clears what must start at zero): calls that
+ *     overlap on the GPU, on different streams or from different threads,
+ *     race and give wrong results;
+ *   - the device error word lives in the scratch, so device-side conditions
+ *     (VDA_ERR_NOT_SPD, VDA_ERR_TIMEOUT) are not reported by this call; host
+ *     side argument errors are, as for vda_forward.
+ * The pages describe no such entry point: it has no counterpart there. */
+#define VDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+vda_status vda_forward_noalloc(const vda_problem* p, const void* Q, const void* K, const void* V,
+                               const void* G, const void* K_txt, const void* V_txt, void* O,
+                               void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of
  * `workspace`: VDA_OK, VDA_ERR_NOT_SPD or VDA_ERR_TIMEOUT (first one set),
  * or VDA_ERR_CUDA if the stream reports an error.  Blocking. */
