@@ -42,8 +42,8 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # Kernel of each stage and the source file that defines it (for ncu traffic lookups).
 STAGE_SOURCES = {
     "gram": "frame_wise_linear_b200/csrc/vda_gram_tc.cu",
-    "factor": "frame_wise_linear_b200/csrc/vda_simt.cu",
-    "scan": "frame_wise_linear_b200/csrc/vda_simt.cu",
+    "factor": "frame_wise_linear_b200/csrc/vda_factor.cu",
+    "scan": "frame_wise_linear_b200/csrc/vda_scan_tc.cu",
     "readout": "frame_wise_linear_b200/csrc/vda_readout_tc.cu",
 }
 
@@ -84,8 +84,8 @@ def stage_work(w):
         # reads K_t, V_t of every frame and the text once
         "gram": dict(bound="hbm", bytes=(frames * w.n + bh * w.n_txt) * (d_k + d_v) * es,
                      flops=2.0 * (frames * w.n + bh * w.n_txt) * d_k * (d_k + d_v)),
-        # Cholesky (d^3/3) + two triangular solves with d_k + d_v right-hand sides
-        "factor": dict(bound="alu", bytes=0, flops=slots * (d_k ** 3 / 3.0 + 2.0 * d_k * d_k * (d_k + d_v))),
+        # lambda A^{-1} by the symmetric sweep: d^3/2 FMA = d^3 flops per slot
+        "factor": dict(bound="alu", bytes=0, flops=slots * float(d_k) ** 3),
         # two directions, one d_k x d_k by d_k x d_v product per frame
         "scan": dict(bound="alu", bytes=0, flops=2.0 * frames * 2.0 * d_k * d_k * d_v),
         # reads Q_t, G_t, writes O_t

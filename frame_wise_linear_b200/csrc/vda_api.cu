@@ -122,11 +122,14 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
       return cuda_fail(e, "gram launch");
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
-  if ((e = vda::launch_factor_simt(p, M, C, err, st)) != cudaSuccess)
-    return cuda_fail(e, "factor launch");
+  constexpr bool kBf16 = std::is_same<TIn, __nv_bfloat16>::value;
+  if ((e = vda::launch_factor(p, M, err, kBf16, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
-  if ((e = vda::launch_scan_simt(p, M, C, SF, SB, st)) != cudaSuccess)
-    return cuda_fail(e, "scan launch");
+  if constexpr (kBf16) {
+    if ((e = vda::launch_scan_tc(p, M, C, SF, SB, err, st)) != cudaSuccess) return cuda_fail(e, "scan launch");
+  } else {
+    if ((e = vda::launch_scan_simt(p, M, C, SF, SB, st)) != cudaSuccess) return cuda_fail(e, "scan launch");
+  }
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "event record");
   if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
     if ((e = vda::launch_readout_tc(p, q, g, SF, SB, static_cast<TIn*>(O), err, st)) != cudaSuccess)

@@ -20,8 +20,8 @@ enum : unsigned {
 // Workspace carve-up.  Slots: one per (b, h, t) with t = 0 for the text and
 // t = 1..T for the frames, slot = (b * H + h) * (T + 1) + t.
 //   err   : 256 bytes, the error word and reserved space
-//   M     : per slot, d_k x d_k float  (Gram A_t on the way, then lambda A_t^{-1})
-//   C     : per slot, d_k x d_v float  (B_t on the way, then A_t^{-1} B_t; S_0 at t = 0)
+//   M     : per slot, d_k x d_k float  (Gram A_t, then M_t = lambda A_t^{-1})
+//   C     : per slot, d_k x d_v float  (B_t = K_t^T V_t)
 //   SF,SB : per frame (b, h, t), d_k x d_v float
 struct Layout {
   size_t err, M, C, SF, SB, total;
@@ -48,13 +48,22 @@ inline Layout make_layout(const vda_problem& p) {
 template <typename TIn>
 cudaError_t launch_gram_simt(const vda_problem& p, const TIn* K, const TIn* V, const TIn* Kt,
                              const TIn* Vt, float* A, float* Bm, cudaStream_t st);
-cudaError_t launch_factor_simt(const vda_problem& p, float* M, float* C, unsigned* err,
-                               cudaStream_t st);
-cudaError_t launch_scan_simt(const vda_problem& p, const float* M, const float* C, float* SF,
+cudaError_t launch_scan_simt(const vda_problem& p, const float* M, const float* Bm, float* SF,
                              float* SB, cudaStream_t st);
 template <typename TIn>
 cudaError_t launch_readout_simt(const vda_problem& p, const TIn* Q, const TIn* G,
                                 const float* SF, const float* SB, TIn* O, cudaStream_t st);
+
+// Factor step (vda_factor.cu): overwrites each slot's A_t in M with
+// M_t = lambda A_t^{-1}, as float32 row-major or, with split_bf16 (d_k = 128),
+// as bf16 hi and lo halves in the K-major 128-byte-swizzled MMA operand image
+// (32 KB each, same 64 KB per slot).
+cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool split_bf16, cudaStream_t st);
+
+// Tensor-core scan (vda_scan_tc.cu): bf16 path, d_k = d_v = 128; M in the
+// split layout above, B_t float32 in the C region.
+cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
+                           unsigned* err, cudaStream_t st);
 
 // Tensor-core Gram (vda_gram_tc.cu): bf16 inputs, d_k = d_v = 128.  Writes
 // the same A and B slots as launch_gram_simt.

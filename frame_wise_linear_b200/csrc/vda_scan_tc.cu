@@ -1,0 +1,252 @@
+// Bidirectional scan on tcgen05 tensor cores (bf16 path, d_k = d_v = 128).
+//
+// "VDN-H3" (comfyui-wiki.com), section on how Video DeltaNet speeds up H3: a
+// bidirectional linear branch carries context through a constant-size state;
+// "VDN-MiniMax-H3" (aiezz.com), section 03: the text is written once into
+// both directional states.  Per (b, h) and direction, every step is
+//     X = S_prev + B_t / lambda,    S_t = M_t X          (M_t = lambda A_t^{-1})
+// starting from S_prev = 0 on the text slot (which gives S_0), then frames
+// 1..T (forward) or T..1 (backward).  S^f_t / S^b_t are written as float32.
+//
+// Precision: M_t arrives as bf16 hi + lo (written by the factor step in the
+// MMA operand layout); X is split the same way; the product takes three MMA
+// passes, M_hi X_hi + M_hi X_lo + M_lo X_hi, accumulated in float32 (the
+// dropped M_lo X_lo term is below 2^-16 relative).  ||M_t||_2 <= 1, so the
+// per-step error does not grow along the chain.
+//
+// The recurrence is independent per column of S, so each chain is split over
+// kSplit CTAs of N = 128 / kSplit columns.  CTA layout (160 threads):
+//   warps 0..3  own TMEM lanes = rows of S: build X (row m) in shared memory,
+//               then read S_t back from TMEM and store it;
+//   warp 4      one thread: bulk-copies M_t (64 KB) into a 2-stage ring ahead
+//               of time and issues the 24 MMAs of each step.
+// Every wait is bounded; a timeout sets the error bit and the CTA winds down.
+#include "sm100.cuh"
+#include "vda_internal.cuh"
+
+namespace vda {
+namespace {
+
+using namespace sm100;
+
+constexpr int kSplit = 2;
+constexpr int N = 128 / kSplit;              // columns of S per CTA
+constexpr int kThreads = 160;
+constexpr int kMBytes = 65536;               // M_t hi | lo
+constexpr int kXHalf = (N / 64) * 16384;     // X hi (or lo): N/64 blocks of 128 rows x 128 B
+constexpr uint32_t kIdesc = idesc_bf16_f32(128, N, /*a MN*/ false, /*b MN*/ true);
+
+struct ScanTcParams {
+  const uint8_t* M;     // per slot 64 KB: M hi (32 KB) | M lo (32 KB)
+  const float* Bm;      // per slot 128 x 128 float
+  float* SF;
+  float* SB;
+  unsigned* err;
+  int T;
+  float lam;
+};
+
+struct Shared {
+  uint64_t m_full[2], m_empty[2];
+  uint64_t x_full, d_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool aborted(Shared& sh) { return *reinterpret_cast<volatile int*>(&sh.abort) != 0; }
+__device__ __forceinline__ void set_abort(Shared& sh, unsigned* err) {
+  atomicOr(err, kDevErrTimeout);
+  *reinterpret_cast<volatile int*>(&sh.abort) = 1;
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_constant__ ScanTcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* mring = base;                     // 2 x 64 KB
+  uint8_t* xbuf = base + 2 * kMBytes;        // X hi | X lo
+  Shared& sh = *reinterpret_cast<Shared*>(xbuf + 2 * kXHalf);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int c0 = blockIdx.x * N;             // first column of S handled here
+  const int dir = blockIdx.y;
+  const int bh = blockIdx.z;
+  const int T = p.T;
+  const size_t slot0 = (size_t)bh * (T + 1);
+  auto slot_of = [&](int s) -> size_t { return slot0 + (s == 0 ? 0 : (dir == 0 ? s : T + 1 - s)); };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.m_full[i], 1);
+      mbar_init(&sh.m_empty[i], 1);
+    }
+    mbar_init(&sh.x_full, 128);
+    mbar_init(&sh.d_full, 1);
+    mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&sh.tmem_base, N);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------------------------------------------- loads + MMAs
+      auto issue_load = [&](int s) {
+        const int st = s & 1;
+        const uint8_t* src = p.M + slot_of(s) * (size_t)kMBytes;
+        mbar_expect_tx(&sh.m_full[st], kMBytes);
+        bulk_load(mring + st * kMBytes, src, kMBytes / 2, &sh.m_full[st]);
+        bulk_load(mring + st * kMBytes + kMBytes / 2, src + kMBytes / 2, kMBytes / 2, &sh.m_full[st]);
+      };
+      int issued = 0;
+      issue_load(0);
+      ++issued;
+      if (T >= 1) {
+        issue_load(1);
+        ++issued;
+      }
+      const uint32_t maddr = smem_u32(mring);
+      const uint32_t xaddr = smem_u32(xbuf);
+      for (int s = 0; s <= T; ++s) {
+        const int st = s & 1;
+        if (!mbar_wait(&sh.m_full[st], (s >> 1) & 1) || !mbar_wait(&sh.x_full, s & 1)) {
+          set_abort(sh, p.err);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ma = maddr + st * kMBytes;
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass) {
+          const uint32_t a_off = pass == 2 ? kMBytes / 2 : 0;      // M lo on the last pass
+          const uint32_t b_off = pass == 1 ? kXHalf : 0;           // X lo on the second pass
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t a = smem_desc(ma + a_off + (k / 4) * 16384 + (k % 4) * 32, 16, 1024, kSwizzle128B);
+            const uint64_t b = smem_desc(xaddr + b_off + k * 16 * 128, 16384, 1024, kSwizzle128B);
+            mma_bf16_ss(tmem, a, b, kIdesc, (pass | k) ? 1u : 0u);
+          }
+        }
+        mma_commit(&sh.d_full);
+        mma_commit(&sh.m_empty[st]);
+        if (s + 2 <= T) {
+          // refill this stage with step s + 2 once its MMAs have read it
+          if (!mbar_wait(&sh.m_empty[st], (s >> 1) & 1)) {
+            set_abort(sh, p.err);
+            break;
+          }
+          issue_load(s + 2);
+          ++issued;
+        }
+      }
+      if (aborted(sh)) {  // copies still in flight land before exit
+        for (int s = issued > 2 ? issued - 2 : 0; s < issued; ++s) mbar_wait(&sh.m_full[s & 1], (s >> 1) & 1);
+      }
+      mma_commit(&sh.drain);
+      mbar_wait(&sh.drain, 0);
+    }
+  } else {
+    // ---------------------------------------------------- rows of S (warps 0..3)
+    const int m = warp * 32 + lane;          // row of S = TMEM lane
+    const float inv_lam = 1.f / p.lam;
+    float srow[N];
+#pragma unroll
+    for (int j = 0; j < N; ++j) srow[j] = 0.f;
+    for (int s = 0; s <= T; ++s) {
+      const size_t slot = slot_of(s);
+      // X row m = S row m + B_t row m / lambda, split into hi / lo, MN-major swizzled.
+      const float4* brow = reinterpret_cast<const float4*>(p.Bm + (slot * 128 + m) * 128 + c0);
+#pragma unroll
+      for (int q = 0; q < N / 8; ++q) {
+        const float4 b0 = __ldg(brow + 2 * q), b1 = __ldg(brow + 2 * q + 1);
+        const float x[8] = {srow[8 * q + 0] + b0.x * inv_lam, srow[8 * q + 1] + b0.y * inv_lam,
+                            srow[8 * q + 2] + b0.z * inv_lam, srow[8 * q + 3] + b0.w * inv_lam,
+                            srow[8 * q + 4] + b1.x * inv_lam, srow[8 * q + 5] + b1.y * inv_lam,
+                            srow[8 * q + 6] + b1.z * inv_lam, srow[8 * q + 7] + b1.w * inv_lam};
+        float h[8], l[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          h[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
+          l[i] = x[i] - h[i];
+        }
+        const uint32_t off = (q / 8) * 16384u + sw128(m, q % 8);
+        *reinterpret_cast<uint4*>(xbuf + off) =
+            make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(h[4], h[5]), pack_bf16(h[6], h[7]));
+        *reinterpret_cast<uint4*>(xbuf + kXHalf + off) =
+            make_uint4(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]), pack_bf16(l[4], l[5]), pack_bf16(l[6], l[7]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sh.x_full);
+      if (__any_sync(0xffffffffu, aborted(sh))) break;
+      const bool ok = mbar_wait(&sh.d_full, s & 1);
+      if (!__all_sync(0xffffffffu, ok)) {
+        set_abort(sh, p.err);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+      for (int c = 0; c < N / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) srow[c * 32 + j] = __uint_as_float(r[j]);
+      }
+      if (s > 0) {
+        const int t = dir == 0 ? s : T + 1 - s;
+        float* out = (dir == 0 ? p.SF : p.SB) + (((size_t)bh * T + (t - 1)) * 128 + m) * 128 + c0;
+#pragma unroll
+        for (int j = 0; j < N; j += 4)
+          *reinterpret_cast<float4*>(out + j) = make_float4(srow[j], srow[j + 1], srow[j + 2], srow[j + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) tmem_dealloc(tmem, N);
+}
+
+}  // namespace
+
+cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
+                           unsigned* err, cudaStream_t st) {
+  ScanTcParams prm;
+  prm.M = reinterpret_cast<const uint8_t*>(M);
+  prm.Bm = Bm;
+  prm.SF = SF;
+  prm.SB = SB;
+  prm.err = err;
+  prm.T = p.T;
+  prm.lam = p.lambda;
+  const size_t smem = 1024 + 2 * kMBytes + 2 * kXHalf + sizeof(Shared);
+  cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(kSplit, 2, p.B * p.H);
+  scan_tc_kernel<<<grid, kThreads, smem, st>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace vda

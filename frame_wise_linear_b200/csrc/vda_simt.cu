@@ -1,11 +1,13 @@
 // Float32 SIMT kernels for every step of VDA forward.
 //
 // These serve float32 inputs (any d_k, d_v multiple of 16 up to 128), where
-// the result must hold float32 accuracy end to end.  Steps, per (b, h):
+// the result must hold float32 accuracy end to end.  Steps, per (b, h), besides
+// the factor step (vda_factor.cu, shared with the bf16 path):
 //   gram    : A_t = K_t^T K_t + lambda I, B_t = K_t^T V_t (frames and text)
-//   factor  : Cholesky A_t = L L^T; M_t = lambda A_t^{-1}, C_t = A_t^{-1} B_t
-//   scan    : S^f_t = M_t S^f_{t-1} + C_t forward, S^b_t = M_t S^b_{t+1} + C_t
-//             backward, both seeded by S_0 = C_0 (the text slot)
+//   scan    : S^f_t = M_t (S^f_{t-1} + B_t / lambda) forward and
+//             S^b_t = M_t (S^b_{t+1} + B_t / lambda) backward, with
+//             M_t = lambda A_t^{-1} from the factor step (vda_factor.cu); both
+//             start from S_0 = M_0 (B_txt / lambda), the text slot
 //   readout : O_t = sigmoid(G_t) * (Q_t (S^f_t + S^b_t))
 // The equations follow "VDN-MiniMax-H3" (aiezz.com) section 03, items Video
 // Delta Attention, text dual-branch injection and gate fusion.
@@ -105,131 +107,71 @@ __global__ void __launch_bounds__(kThreads) gram_simt_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// factor: one block per slot.  Right-looking Cholesky of A in shared memory,
-// then forward and backward substitution with the right-hand sides
-// [lambda I | B], one thread per right-hand-side column.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads) factor_simt_kernel(float* __restrict__ M,
-                                                               float* __restrict__ C, int dk,
-                                                               int dv, float lam,
-                                                               unsigned* __restrict__ err) {
-  extern __shared__ float smem[];
-  const int ldl = dk + 1;
-  const int ncol = dk + dv;
-  float* sL = smem;               // dk x ldl
-  float* sZ = smem + dk * ldl;    // dk x ncol
-  const int slot = blockIdx.x;
-  const int tid = threadIdx.x;
-  float* Ap = M + (size_t)slot * dk * dk;
-  float* Bp = C + (size_t)slot * dk * dv;
-  for (int e = tid; e < dk * dk; e += kThreads) sL[(e / dk) * ldl + (e % dk)] = Ap[e];
-  for (int e = tid; e < dk * ncol; e += kThreads) {
-    const int i = e / ncol, c = e % ncol;
-    sZ[e] = c < dk ? (i == c ? lam : 0.f) : Bp[(size_t)i * dv + (c - dk)];
-  }
-  __syncthreads();
-
-  bool bad = false;
-  for (int j = 0; j < dk; ++j) {
-    float djj = sL[j * ldl + j];
-    if (!(djj > 0.f) || !isfinite(djj)) {
-      bad = true;
-      djj = 1.f;
-    }
-    const float ljj = sqrtf(djj);
-    for (int i = j + 1 + tid; i < dk; i += kThreads) sL[i * ldl + j] /= ljj;
-    __syncthreads();
-    if (tid == 0) sL[j * ldl + j] = ljj;
-    const int m = dk - j - 1;
-    for (int e = tid; e < m * m; e += kThreads) {
-      const int ii = e / m, kk = e % m;
-      if (kk <= ii) {
-        const int i = j + 1 + ii, k = j + 1 + kk;
-        sL[i * ldl + k] -= sL[i * ldl + j] * sL[k * ldl + j];
-      }
-    }
-    __syncthreads();
-  }
-  if (bad && tid == 0) atomicOr(err, kDevErrNotSpd);
-
-  if (tid < ncol) {
-    const int c = tid;
-    for (int i = 0; i < dk; ++i) {  // L Y = Z
-      float z = sZ[i * ncol + c];
-      for (int k = 0; k < i; ++k) z = fmaf(-sL[i * ldl + k], sZ[k * ncol + c], z);
-      sZ[i * ncol + c] = z / sL[i * ldl + i];
-    }
-    for (int i = dk - 1; i >= 0; --i) {  // L^T X = Y
-      float z = sZ[i * ncol + c];
-      for (int k = i + 1; k < dk; ++k) z = fmaf(-sL[k * ldl + i], sZ[k * ncol + c], z);
-      sZ[i * ncol + c] = z / sL[i * ldl + i];
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < dk * ncol; e += kThreads) {
-    const int i = e / ncol, c = e % ncol;
-    if (c < dk) Ap[(size_t)i * dk + c] = sZ[e];
-    else Bp[(size_t)i * dv + (c - dk)] = sZ[e];
-  }
-}
-
-// ---------------------------------------------------------------------------
-// scan: one block per (column slice of 16, direction, b*h).  The recurrence
-// is independent per column of S, so slices need no communication.
+// scan: one block per (column slice of 16, direction, b*h).  Every step is
+//     X = S_prev + B_t / lambda,   S = M_t X          (M_t = lambda A_t^{-1})
+// which equals A_t^{-1} (lambda S_prev + B_t).  The text slot (t = 0) runs it
+// from S_prev = 0 to give S_0.  The recurrence is independent per column of
+// S, so slices need no communication.
 // ---------------------------------------------------------------------------
 constexpr int kScanCols = 16;
 
 __global__ void __launch_bounds__(kThreads) scan_simt_kernel(const float* __restrict__ M,
-                                                             const float* __restrict__ C,
+                                                             const float* __restrict__ Bm,
                                                              float* __restrict__ SF,
                                                              float* __restrict__ SB, int T,
-                                                             int dk, int dv) {
+                                                             int dk, int dv, float lam) {
   extern __shared__ float smem[];
   const int ldm = dk + 1;
-  float* sM = smem;              // dk x ldm
-  float* sS = smem + dk * ldm;   // dk x kScanCols
+  float* sM = smem;                          // dk x ldm
+  float* sX = smem + dk * ldm;               // dk x kScanCols
   const int c0 = blockIdx.x * kScanCols;
   const int dir = blockIdx.y;
   const int bh = blockIdx.z;
   const int tid = threadIdx.x;
   const size_t base = (size_t)bh * (T + 1);
   float* out = dir == 0 ? SF : SB;
-
-  for (int e = tid; e < dk * kScanCols; e += kThreads) {
-    const int i = e / kScanCols, c = e % kScanCols;
-    sS[e] = C[base * dk * dv + (size_t)i * dv + c0 + c];  // S_0
-  }
+  const float inv_lam = 1.f / lam;
   constexpr int kPer = (128 * kScanCols) / kThreads;  // outputs per thread at most
-  for (int step = 0; step < T; ++step) {
-    const int t = dir == 0 ? step + 1 : T - step;
+  float res[kPer];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) res[r] = 0.f;       // S_prev = 0 before the text
+
+  for (int step = 0; step <= T; ++step) {
+    const int t = step == 0 ? 0 : (dir == 0 ? step : T + 1 - step);
     const float* Mp = M + (base + t) * dk * dk;
-    const float* Cp = C + (base + t) * dk * dv;
+    const float* Bp = Bm + (base + t) * dk * dv;
     for (int e = tid; e < dk * dk; e += kThreads) sM[(e / dk) * ldm + (e % dk)] = Mp[e];
-    __syncthreads();
-    float res[kPer];
 #pragma unroll
     for (int r = 0; r < kPer; ++r) {
       const int e = tid + r * kThreads;
-      res[r] = 0.f;
       if (e < dk * kScanCols) {
         const int i = e / kScanCols, c = e % kScanCols;
-        float acc = Cp[(size_t)i * dv + c0 + c];
-        for (int k = 0; k < dk; ++k) acc = fmaf(sM[i * ldm + k], sS[k * kScanCols + c], acc);
+        sX[e] = res[r] + Bp[(size_t)i * dv + c0 + c] * inv_lam;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int e = tid + r * kThreads;
+      if (e < dk * kScanCols) {
+        const int i = e / kScanCols, c = e % kScanCols;
+        float acc = 0.f;
+        for (int k = 0; k < dk; ++k) acc = fmaf(sM[i * ldm + k], sX[k * kScanCols + c], acc);
         res[r] = acc;
       }
     }
     __syncthreads();
-    float* op = out + ((size_t)bh * T + (t - 1)) * dk * dv;
+    if (step > 0) {
+      float* op = out + ((size_t)bh * T + (t - 1)) * dk * dv;
 #pragma unroll
-    for (int r = 0; r < kPer; ++r) {
-      const int e = tid + r * kThreads;
-      if (e < dk * kScanCols) {
-        const int i = e / kScanCols, c = e % kScanCols;
-        sS[e] = res[r];
-        op[(size_t)i * dv + c0 + c] = res[r];
+      for (int r = 0; r < kPer; ++r) {
+        const int e = tid + r * kThreads;
+        if (e < dk * kScanCols) {
+          const int i = e / kScanCols, c = e % kScanCols;
+          op[(size_t)i * dv + c0 + c] = res[r];
+        }
       }
     }
-    __syncthreads();
   }
 }
 
@@ -304,25 +246,14 @@ cudaError_t launch_gram_simt(const vda_problem& p, const TIn* K, const TIn* V, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_factor_simt(const vda_problem& p, float* M, float* C, unsigned* err,
-                               cudaStream_t st) {
-  const size_t smem = ((size_t)p.d_k * (p.d_k + 1) + (size_t)p.d_k * (p.d_k + p.d_v)) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(factor_simt_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  const unsigned slots = (unsigned)(p.B * p.H * (p.T + 1));
-  factor_simt_kernel<<<slots, kThreads, smem, st>>>(M, C, p.d_k, p.d_v, p.lambda, err);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_scan_simt(const vda_problem& p, const float* M, const float* C, float* SF,
+cudaError_t launch_scan_simt(const vda_problem& p, const float* M, const float* Bm, float* SF,
                              float* SB, cudaStream_t st) {
   const size_t smem = ((size_t)p.d_k * (p.d_k + 1) + (size_t)p.d_k * kScanCols) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.d_v / kScanCols, 2, p.B * p.H);
-  scan_simt_kernel<<<grid, kThreads, smem, st>>>(M, C, SF, SB, p.T, p.d_k, p.d_v);
+  scan_simt_kernel<<<grid, kThreads, smem, st>>>(M, Bm, SF, SB, p.T, p.d_k, p.d_v, p.lambda);
   return cudaGetLastError();
 }
 
