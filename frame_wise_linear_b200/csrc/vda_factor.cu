@@ -15,54 +15,26 @@
 // row/column k zeroed first, a -= x (p x)^T.  n^3/2 FMA on the lower triangle.
 //
 // Layout: one CTA per slot, 160 threads; thread t owns one 8x8 block (R, C),
-// R >= C, of the lower triangle in registers (136 blocks for d = 128).  Per
-// pivot, the owners of column k publish it (double-buffered) and one barrier
-// separates pivots.  A non-positive or non-finite pivot sets the NOT_SPD bit.
-#include "sm100.cuh"
-#include "vda_internal.cuh"
+// R >= C, of the lower triangle in registers (136 blocks for d = 128).  Pivots
+// go in pairs: the owners publish columns k and k + 1 (double-buffered), one
+// barrier per pair, and every thread derives the second pivot's column from
+// the two published ones.  A non-positive or non-finite pivot sets the
+// NOT_SPD bit.
+#include "vda_sweep.cuh"
 
 namespace vda {
 namespace {
 
 constexpr int kThreads = 160;
 
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Writes 8 consecutive k-values of row m of M as bf16 hi and lo chunks of the
-// K-major, 128-byte-swizzled MMA operand image (two 64-column halves of 16 KB).
-__device__ __forceinline__ void store_split_chunk(uint8_t* hi, uint8_t* lo, int m, int kchunk, const float (&v)[8]) {
-  float h[8], l[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    h[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
-    l[i] = v[i] - h[i];
-  }
-  const uint32_t off = (kchunk / 8) * 16384u + sm100::sw128(m, kchunk % 8);
-  *reinterpret_cast<uint4*>(hi + off) = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
-  *reinterpret_cast<uint4*>(lo + off) = make_uint4(pack2(l[0], l[1]), pack2(l[2], l[3]), pack2(l[4], l[5]), pack2(l[6], l[7]));
-}
-
 template <int D, bool kSplitOut>
-__global__ void __launch_bounds__(kThreads) factor_sweep_kernel(float* __restrict__ Mreg, float lam,
-                                                                unsigned* __restrict__ err) {
-  constexpr int NB = D / 8;
-  constexpr int NBLK = NB * (NB + 1) / 2;
-  __shared__ float xs[2][D];
-  __shared__ float pinv[2];
+__global__ void __launch_bounds__(kThreads, 3) factor_sweep_kernel(float* __restrict__ Mreg, float lam,
+                                                                   unsigned* __restrict__ err) {
+  // xs[b][0] = column k, xs[b][1] = column k + 1, both before the pair of pivots.
+  __shared__ __align__(16) float xs[2][2][D];
 
-  const int tid = threadIdx.x;
-  const bool active = tid < NBLK;
-  // block (R, C) of the lower triangle, enumerated row by row
-  int R = 0, C = 0;
-  if (active) {
-    int r = 0;
-    while ((r + 1) * (r + 2) / 2 <= tid) ++r;
-    R = r;
-    C = tid - r * (r + 1) / 2;
-  }
+  int R, C;
+  const bool active = sweep::block_of<D>(threadIdx.x, R, C);
   float* A = Mreg + (size_t)blockIdx.x * D * D;
 
   float a[8][8];
@@ -75,72 +47,7 @@ __global__ void __launch_bounds__(kThreads) factor_sweep_kernel(float* __restric
       a[r][4] = v1.x; a[r][5] = v1.y; a[r][6] = v1.z; a[r][7] = v1.w;
     }
   }
-  bool bad = false;
-
-  // Publishes column k (pre-update values of the next pivot) into buffer b.
-  auto publish = [&](int K, auto kk_c, int b) {
-    constexpr int kk = decltype(kk_c)::value;
-    if (!active) return;
-    if (C == K) {
-#pragma unroll
-      for (int r = 0; r < 8; ++r) xs[b][8 * R + r] = a[r][kk];
-    }
-    if (R == K && C < K) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) xs[b][8 * C + c] = a[kk][c];
-    }
-    if (R == K && C == K) {
-      const float piv = a[kk][kk];
-      if (!(piv > 0.f) || !isfinite(piv)) bad = true;
-      pinv[b] = 1.f / piv;
-      xs[b][8 * K + kk] = -1.f;
-    }
-  };
-
-  publish(0, std::integral_constant<int, 0>{}, 0);
-  int buf = 0;
-#pragma unroll 1
-  for (int K = 0; K < NB; ++K) {
-    auto step = [&](auto kk_c) {
-      constexpr int kk = decltype(kk_c)::value;
-      __syncthreads();
-      if (active) {
-        const float p = pinv[buf];
-        float xr[8], yc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          xr[i] = xs[buf][8 * R + i];
-          yc[i] = p * xs[buf][8 * C + i];
-        }
-        if (R == K) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) a[kk][c] = 0.f;
-        }
-        if (C == K) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r) a[r][kk] = 0.f;
-        }
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-xr[r], yc[c], a[r][c]);
-      }
-      buf ^= 1;
-      if constexpr (kk < 7) {
-        publish(K, std::integral_constant<int, kk + 1>{}, buf);
-      } else {
-        if (K + 1 < NB) publish(K + 1, std::integral_constant<int, 0>{}, buf);
-      }
-    };
-    step(std::integral_constant<int, 0>{});
-    step(std::integral_constant<int, 1>{});
-    step(std::integral_constant<int, 2>{});
-    step(std::integral_constant<int, 3>{});
-    step(std::integral_constant<int, 4>{});
-    step(std::integral_constant<int, 5>{});
-    step(std::integral_constant<int, 6>{});
-    step(std::integral_constant<int, 7>{});
-  }
+  const bool bad = sweep::invert<D>(a, R, C, active, xs, [] { __syncthreads(); });
   if (bad) atomicOr(err, kDevErrNotSpd);
   if (!active) return;
 
@@ -151,39 +58,9 @@ __global__ void __launch_bounds__(kThreads) factor_sweep_kernel(float* __restric
     for (int c = 0; c < 8; ++c) a[r][c] *= -lam;
 
   if constexpr (kSplitOut) {
-    uint8_t* hi = reinterpret_cast<uint8_t*>(A);
-    uint8_t* lo = hi + 32768;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      float v[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) v[c] = a[r][c];
-      store_split_chunk(hi, lo, 8 * R + r, C, v);
-    }
-    if (R != C) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float v[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) v[r] = a[r][c];
-        store_split_chunk(hi, lo, 8 * C + c, R, v);
-      }
-    }
+    sweep::store_split(a, R, C, reinterpret_cast<uint8_t*>(A));
   } else {
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      float* row = A + (size_t)(8 * R + r) * D + 8 * C;
-      *reinterpret_cast<float4*>(row) = make_float4(a[r][0], a[r][1], a[r][2], a[r][3]);
-      *reinterpret_cast<float4*>(row + 4) = make_float4(a[r][4], a[r][5], a[r][6], a[r][7]);
-    }
-    if (R != C) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float* row = A + (size_t)(8 * C + c) * D + 8 * R;
-        *reinterpret_cast<float4*>(row) = make_float4(a[0][c], a[1][c], a[2][c], a[3][c]);
-        *reinterpret_cast<float4*>(row + 4) = make_float4(a[4][c], a[5][c], a[6][c], a[7][c]);
-      }
-    }
+    sweep::store_f32<D>(a, R, C, A);
   }
 }
 

@@ -65,6 +65,12 @@ cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool sp
 cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
                            unsigned* err, cudaStream_t st);
 
+// Gram and factor fused (vda_gram_factor_tc.cu): bf16, d_k = d_v = 128.
+// Writes M_t (split layout, as launch_factor with split_bf16) and B_t.
+cudaError_t launch_gram_factor_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                                  const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* M, float* Bm,
+                                  unsigned* err, cudaStream_t st);
+
 // Tensor-core Gram (vda_gram_tc.cu): bf16 inputs, d_k = d_v = 128.  Writes
 // the same A and B slots as launch_gram_simt.
 cudaError_t launch_gram_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,

@@ -13,10 +13,12 @@
 //   warp 0      TMA producer: Q tiles (3-stage ring) and G tiles (2-stage ring),
 //               each tile as two 64-feature boxes with the 128-byte swizzle.
 //   warp 1      TMEM (2 x 128 columns) and the MMAs (one thread).
-//   warps 2..5  at each new frame: S = S^f + S^b split into bf16 hi/lo in
+//   warps 2..9  at each new frame: S = S^f + S^b split into bf16 hi/lo in
 //               shared memory (the MMA B operand); per tile: TMEM -> registers,
 //               gate from the G tile, O written over the G tile in shared
-//               memory, then one TMA store of the O tile.
+//               memory, then a TMA store per 64-column half.  Warps 2..5 take
+//               columns 0..63 and warps 6..9 columns 64..127 (two warps per
+//               TMEM lane quarter).
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
@@ -33,7 +35,7 @@ constexpr int kRows = 128;                   // tokens per tile
 constexpr int kBox = kRows * 64 * 2;         // 128 rows x 64 features bf16: 16 KB
 constexpr int kTile = 2 * kBox;              // 32 KB
 constexpr int kSig = 2 * kTile;              // S_hi and S_lo, 32 KB each
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;              // 2 control warps + 8 epilogue warps
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
 
@@ -88,13 +90,13 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     }
     for (int i = 0; i < kGStages; ++i) {
       mbar_init(&sh.g_full[i], 1);
-      mbar_init(&sh.g_empty[i], 1);
+      mbar_init(&sh.g_empty[i], 2);   // one arrival per stored half
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.t_full[i], 1);
-      mbar_init(&sh.t_empty[i], 128);
+      mbar_init(&sh.t_empty[i], 256);
     }
-    mbar_init(&sh.sig_full, 128);
+    mbar_init(&sh.sig_full, 256);
     mbar_init(&sh.sig_empty, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -195,9 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     }
   } else {
     // ------------------------------------------------------------ S prep + epilogue
-    const int et = threadIdx.x - 64;          // 0..127
-    const int quarter = warp % 4;
+    const int et = threadIdx.x - 64;          // 0..255
+    const int quarter = warp % 4;             // TMEM lanes this warp may access
+    const int half = (warp - 2) / 4;          // column half 0..63 or 64..127
     const int row = quarter * 32 + lane;      // tile row this thread owns in TMEM
+    const int srow_i = et % 128;              // row of S this thread prepares
+    const int shalf = et / 128;               // and which 64 of its columns
     int gs = 0, tb = 0, cur_u = -1;
     uint32_t gph = 0, tph = 0, seph = 0;
     for (int tile = t_begin; tile < t_end; ++tile) {
@@ -208,13 +213,20 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
         const bool ok = mbar_wait(&sh.sig_empty, seph ^ 1);
         if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
         seph ^= 1;
-        // Row `et` of S = S^f + S^b, split into hi/lo bf16, MN-major swizzled.
-        const float4* f = reinterpret_cast<const float4*>(p.SF + ((size_t)u * 128 + et) * 128);
-        const float4* b = reinterpret_cast<const float4*>(p.SB + ((size_t)u * 128 + et) * 128);
-#pragma unroll 4
-        for (int c = 0; c < 16; ++c) {   // 8 columns per step
-          const float4 f0 = __ldg(f + 2 * c), f1 = __ldg(f + 2 * c + 1);
-          const float4 b0 = __ldg(b + 2 * c), b1 = __ldg(b + 2 * c + 1);
+        // S = S^f + S^b, row srow_i, columns 64*shalf .. +63: split into hi/lo
+        // bf16, MN-major swizzled (the MMA B operand).
+        const float4* f = reinterpret_cast<const float4*>(p.SF + ((size_t)u * 128 + srow_i) * 128 + 64 * shalf);
+        const float4* b = reinterpret_cast<const float4*>(p.SB + ((size_t)u * 128 + srow_i) * 128 + 64 * shalf);
+        float4 fv[16], bv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          fv[c] = __ldg(f + c);
+          bv[c] = __ldg(b + c);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {   // 8 columns per chunk
+          const float4 f0 = fv[2 * c], f1 = fv[2 * c + 1];
+          const float4 b0 = bv[2 * c], b1 = bv[2 * c + 1];
           const float x[8] = {f0.x + b0.x, f0.y + b0.y, f0.z + b0.z, f0.w + b0.w,
                               f1.x + b1.x, f1.y + b1.y, f1.z + b1.z, f1.w + b1.w};
           float hi[8], lo[8];
@@ -223,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
             hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
             lo[i] = x[i] - hi[i];
           }
-          const uint32_t off = (c / 8) * kBox + sw128(et, c % 8);
+          const uint32_t off = shalf * kBox + sw128(srow_i, c);
           *reinterpret_cast<uint4*>(sig + off) =
               make_uint4(pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]),
                          pack_bf16(hi[6], hi[7]));
@@ -240,16 +252,16 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
       tc_fence_after();
       uint8_t* gt = gbuf + gs * kTile;
-      const uint32_t taddr = tmem + tb * 128 + ((uint32_t)(quarter * 32) << 16);
+      uint8_t* rowp = gt + half * kBox;
+      const uint32_t taddr = tmem + tb * 128 + half * 64 + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {           // 32 output columns per step
+      for (int c = 0; c < 2; ++c) {           // 32 output columns per step
         uint32_t r[32];
         tmem_ld_32x32b_x32(taddr + c * 32, r);
         tmem_ld_wait();
-        uint8_t* rowp = gt + (c / 2) * kBox;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {          // 8 columns = one 16-byte chunk
-          const uint32_t off = sw128(row, (c % 2) * 4 + q);
+          const uint32_t off = sw128(row, c * 4 + q);
           const uint4 gv = *reinterpret_cast<const uint4*>(rowp + off);
           const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
           uint32_t ow[4];
@@ -266,10 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       tc_fence_before();
       mbar_arrive(&sh.t_empty[tb]);
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (et == 0) {
-        tma_store_3d(&p.mO, gt, 0, y, u);
-        tma_store_3d(&p.mO, gt + kBox, 64, y, u);
+      named_bar_sync(1 + half, 128);
+      if (et % 128 == 0) {   // first thread of each half stores that half
+        tma_store_3d(&p.mO, rowp, 64 * half, y, u);
         bulk_commit();
         bulk_wait_read<0>();
         mbar_arrive(&sh.g_empty[gs]);
@@ -278,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       tb ^= 1;
       if (tb == 0) tph ^= 1;
     }
-    if (et == 0) bulk_wait<0>();               // O stores complete before exit
+    if (et % 128 == 0) bulk_wait<0>();         // O stores complete before exit
   }
 
   tc_fence_before();

@@ -168,25 +168,33 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     // ---------------------------------------------------- rows of S (warps 0..3)
     const int m = warp * 32 + lane;          // row of S = TMEM lane
     const float inv_lam = 1.f / p.lam;
-    float srow[N];
+    float srow[N], brow[N];
 #pragma unroll
     for (int j = 0; j < N; ++j) srow[j] = 0.f;
+    // B_t row m of the first step; each later row is fetched while the
+    // previous step's MMAs run.
+    auto fetch_b = [&](int s) {
+      const float4* src = reinterpret_cast<const float4*>(p.Bm + (slot_of(s) * 128 + m) * 128 + c0);
+#pragma unroll
+      for (int q = 0; q < N / 4; ++q) {
+        const float4 v = __ldg(src + q);
+        brow[4 * q] = v.x;
+        brow[4 * q + 1] = v.y;
+        brow[4 * q + 2] = v.z;
+        brow[4 * q + 3] = v.w;
+      }
+    };
+    fetch_b(0);
     for (int s = 0; s <= T; ++s) {
-      const size_t slot = slot_of(s);
       // X row m = S row m + B_t row m / lambda, split into hi / lo, MN-major swizzled.
-      const float4* brow = reinterpret_cast<const float4*>(p.Bm + (slot * 128 + m) * 128 + c0);
 #pragma unroll
       for (int q = 0; q < N / 8; ++q) {
-        const float4 b0 = __ldg(brow + 2 * q), b1 = __ldg(brow + 2 * q + 1);
-        const float x[8] = {srow[8 * q + 0] + b0.x * inv_lam, srow[8 * q + 1] + b0.y * inv_lam,
-                            srow[8 * q + 2] + b0.z * inv_lam, srow[8 * q + 3] + b0.w * inv_lam,
-                            srow[8 * q + 4] + b1.x * inv_lam, srow[8 * q + 5] + b1.y * inv_lam,
-                            srow[8 * q + 6] + b1.z * inv_lam, srow[8 * q + 7] + b1.w * inv_lam};
         float h[8], l[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          h[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
-          l[i] = x[i] - h[i];
+          const float x = fmaf(brow[8 * q + i], inv_lam, srow[8 * q + i]);
+          h[i] = __bfloat162float(__float2bfloat16_rn(x));
+          l[i] = x - h[i];
         }
         const uint32_t off = (q / 8) * 16384u + sw128(m, q % 8);
         *reinterpret_cast<uint4*>(xbuf + off) =
@@ -197,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sh.x_full);
+      if (s + 1 <= T) fetch_b(s + 1);
       if (__any_sync(0xffffffffu, aborted(sh))) break;
       const bool ok = mbar_wait(&sh.d_full, s & 1);
       if (!__all_sync(0xffffffffu, ok)) {

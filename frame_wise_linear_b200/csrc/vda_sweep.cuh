@@ -1,0 +1,229 @@
+// The symmetric sweep operator on a d x d SPD matrix held as 8x8 register
+// blocks of its lower triangle (one block per thread), shared by the
+// stand-alone factor kernel and the fused Gram + factor kernel.
+//
+// Sweeping pivot k maps a_kk -> -1/a_kk, a_ik -> a_ik/a_kk and
+// a_ij -> a_ij - a_ik a_kj / a_kk (in-place Gauss-Jordan with diagonal pivots,
+// which are the positive LDL^T pivots of an SPD matrix); after all pivots the
+// matrix is -A^{-1}.  Each pivot is one symmetric rank-1 update: with
+// x = column k (x_k := -1), p = 1/a_kk and row/column k zeroed, a -= x (p x)^T.
+// Pivots go in pairs: the owners publish columns k and k + 1, one barrier per
+// pair, and every thread derives the second pivot's column from the two.
+#pragma once
+
+#include "sm100.cuh"
+#include "vda_internal.cuh"
+
+namespace vda {
+namespace sweep {
+
+// Block (R, C), R >= C, of the lower triangle owned by thread `tid` (blocks
+// enumerated row by row); false for threads past the last block.
+template <int D>
+__device__ __forceinline__ bool block_of(int tid, int& R, int& C) {
+  constexpr int NB = D / 8;
+  R = C = 0;
+  if (tid >= NB * (NB + 1) / 2) return false;
+  int r = 0;
+  while ((r + 1) * (r + 2) / 2 <= tid) ++r;
+  R = r;
+  C = tid - r * (r + 1) / 2;
+  return true;
+}
+
+// Runs all D pivots on `a` (this thread's block).  `xs` is shared scratch of
+// [2][2][D] floats (16-byte aligned); `sync` is a barrier over all threads
+// taking part (inactive ones included).  Returns true if a pivot was not
+// positive and finite.  On return a holds this block of -A^{-1}.
+template <int D, typename Sync>
+__device__ __forceinline__ bool invert(float (&a)[8][8], int R, int C, bool active, float (*xs)[2][D], Sync sync) {
+  constexpr int NB = D / 8;
+  bool bad = false;
+
+  // Publishes columns k and k + 1 = 8K + kk, 8K + kk + 1 (current values) into buffer b.
+  auto publish = [&](int K, auto kk_c, int b) {
+    constexpr int kk = decltype(kk_c)::value;
+    if (!active) return;
+    if (C == K) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        xs[b][0][8 * R + r] = a[r][kk];
+        xs[b][1][8 * R + r] = a[r][kk + 1];
+      }
+    }
+    if (R == K && C < K) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        xs[b][0][8 * C + c] = a[kk][c];
+        xs[b][1][8 * C + c] = a[kk + 1][c];
+      }
+    }
+  };
+  auto load8 = [&](const float* src, float (&v)[8]) {
+    const float4 lo = *reinterpret_cast<const float4*>(src);
+    const float4 hi = *reinterpret_cast<const float4*>(src + 4);
+    v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+    v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+  };
+
+  publish(0, std::integral_constant<int, 0>{}, 0);
+  int buf = 0;
+#pragma unroll 1
+  for (int K = 0; K < NB; ++K) {
+    // Two pivots k = 8K + kk and k + 1 per barrier.  With u, v the columns
+    // before both: pivot k uses x = u (x_k = -1), p1 = 1/u_k; column k + 1
+    // after it is v' = v - u p1 u_{k+1} (v'_k = p1 u_{k+1}); pivot k + 1 uses
+    // y = v' (y_{k+1} = -1), p2 = 1/v'_{k+1}.
+    auto pair = [&](auto kk_c) {
+      constexpr int kk = decltype(kk_c)::value;
+      sync();
+      const float uk = xs[buf][0][8 * K + kk];
+      const float uk1 = xs[buf][0][8 * K + kk + 1];
+      const float vk1 = xs[buf][1][8 * K + kk + 1];
+      const float p1 = 1.f / uk;
+      const float g = p1 * uk1;                 // v' = v - u g
+      const float piv2 = vk1 - uk1 * g;
+      const float p2 = 1.f / piv2;
+      if (active) {
+        if (R == K && C == K && (!(uk > 0.f) || !isfinite(uk) || !(piv2 > 0.f) || !isfinite(piv2))) bad = true;
+        float ur[8], uc[8];
+        load8(&xs[buf][0][8 * R], ur);
+        load8(&xs[buf][0][8 * C], uc);
+        // ---- pivot k
+        {
+          float xr[8], yc[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            xr[i] = ur[i];
+            yc[i] = uc[i];
+          }
+          if (R == K) xr[kk] = -1.f;
+          if (C == K) yc[kk] = -1.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) yc[i] *= p1;
+          if (R == K) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a[kk][c] = 0.f;
+          }
+          if (C == K) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) a[r][kk] = 0.f;
+          }
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-xr[r], yc[c], a[r][c]);
+        }
+        // ---- pivot k + 1
+        {
+          float vr[8], vc[8];
+          load8(&xs[buf][1][8 * R], vr);
+          load8(&xs[buf][1][8 * C], vc);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            vr[i] = fmaf(-ur[i], g, vr[i]);
+            vc[i] = fmaf(-uc[i], g, vc[i]);
+          }
+          if (R == K) {
+            vr[kk] = g;
+            vr[kk + 1] = -1.f;
+          }
+          if (C == K) {
+            vc[kk] = g;
+            vc[kk + 1] = -1.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) vc[i] *= p2;
+          if (R == K) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a[kk + 1][c] = 0.f;
+          }
+          if (C == K) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) a[r][kk + 1] = 0.f;
+          }
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-vr[r], vc[c], a[r][c]);
+        }
+      }
+      buf ^= 1;
+      if constexpr (kk + 2 < 8) {
+        publish(K, std::integral_constant<int, kk + 2>{}, buf);
+      } else {
+        if (K + 1 < NB) publish(K + 1, std::integral_constant<int, 0>{}, buf);
+      }
+    };
+    pair(std::integral_constant<int, 0>{});
+    pair(std::integral_constant<int, 2>{});
+    pair(std::integral_constant<int, 4>{});
+    pair(std::integral_constant<int, 6>{});
+  }
+  return bad;
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Writes 8 consecutive k-values of row m of M as bf16 hi and lo chunks of the
+// K-major, 128-byte-swizzled MMA operand image (two 64-column halves of 16 KB).
+__device__ __forceinline__ void store_split_chunk(uint8_t* hi, uint8_t* lo, int m, int kchunk, const float (&v)[8]) {
+  float h[8], l[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+    l[i] = v[i] - h[i];
+  }
+  const uint32_t off = (kchunk / 8) * 16384u + sm100::sw128(m, kchunk % 8);
+  *reinterpret_cast<uint4*>(hi + off) = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
+  *reinterpret_cast<uint4*>(lo + off) = make_uint4(pack2(l[0], l[1]), pack2(l[2], l[3]), pack2(l[4], l[5]), pack2(l[6], l[7]));
+}
+
+// Writes this thread's block of the symmetric result and its transpose as
+// bf16 hi (bytes [0, 32K)) and lo ([32K, 64K)) halves of the K-major,
+// 128-byte-swizzled MMA operand image of a 128 x 128 matrix.
+__device__ __forceinline__ void store_split(const float (&a)[8][8], int R, int C, uint8_t* img) {
+  uint8_t* hi = img;
+  uint8_t* lo = img + 32768;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    float v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) v[c] = a[r][c];
+    store_split_chunk(hi, lo, 8 * R + r, C, v);
+  }
+  if (R != C) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) v[r] = a[r][c];
+      store_split_chunk(hi, lo, 8 * C + c, R, v);
+    }
+  }
+}
+
+// Writes this thread's block and its transpose into a row-major D x D matrix.
+template <int D>
+__device__ __forceinline__ void store_f32(const float (&a)[8][8], int R, int C, float* A) {
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    float* row = A + (size_t)(8 * R + r) * D + 8 * C;
+    *reinterpret_cast<float4*>(row) = make_float4(a[r][0], a[r][1], a[r][2], a[r][3]);
+    *reinterpret_cast<float4*>(row + 4) = make_float4(a[r][4], a[r][5], a[r][6], a[r][7]);
+  }
+  if (R != C) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float* row = A + (size_t)(8 * C + c) * D + 8 * R;
+      *reinterpret_cast<float4*>(row) = make_float4(a[0][c], a[1][c], a[2][c], a[3][c]);
+      *reinterpret_cast<float4*>(row + 4) = make_float4(a[4][c], a[5][c], a[6][c], a[7][c]);
+    }
+  }
+}
+
+}  // namespace sweep
+}  // namespace vda
