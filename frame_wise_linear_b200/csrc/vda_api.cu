@@ -114,15 +114,14 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
   const TIn* vt = static_cast<const TIn*>(Vt);
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
   if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "event record");
-  if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-    if ((e = vda::launch_gram_tc(p, k, v, kt, vt, M, C, err, st)) != cudaSuccess)
-      return cuda_fail(e, "gram launch");
+  constexpr bool kBf16 = std::is_same<TIn, __nv_bfloat16>::value;
+  if constexpr (kBf16) {
+    if ((e = vda::launch_gram_tc(p, k, v, kt, vt, M, C, err, st)) != cudaSuccess) return cuda_fail(e, "gram launch");
   } else {
     if ((e = vda::launch_gram_simt<TIn>(p, k, v, kt, vt, M, C, st)) != cudaSuccess)
       return cuda_fail(e, "gram launch");
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
-  constexpr bool kBf16 = std::is_same<TIn, __nv_bfloat16>::value;
   if ((e = vda::launch_factor(p, M, err, kBf16, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
   if constexpr (kBf16) {

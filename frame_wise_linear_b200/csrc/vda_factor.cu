@@ -32,6 +32,7 @@ __global__ void __launch_bounds__(kThreads, 3) factor_sweep_kernel(float* __rest
                                                                    unsigned* __restrict__ err) {
   // xs[b][0] = column k, xs[b][1] = column k + 1, both before the pair of pivots.
   __shared__ __align__(16) float xs[2][2][D];
+  __shared__ __align__(16) float sc[2][4];
 
   int R, C;
   const bool active = sweep::block_of<D>(threadIdx.x, R, C);
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(kThreads, 3) factor_sweep_kernel(float* __rest
       a[r][4] = v1.x; a[r][5] = v1.y; a[r][6] = v1.z; a[r][7] = v1.w;
     }
   }
-  const bool bad = sweep::invert<D>(a, R, C, active, xs, [] { __syncthreads(); });
+  const bool bad = sweep::invert<D>(a, R, C, active, xs, sc, [] { __syncthreads(); });
   if (bad) atomicOr(err, kDevErrNotSpd);
   if (!active) return;
 

@@ -9,14 +9,15 @@
 //
 // Design (persistent, one CTA per SM, 6 warps):
 //   warp 0      TMA producer: 64-token chunks of K_t and V_t, each as two
-//               64-feature boxes with the 128-byte swizzle, into a 6-stage ring
+//               64-feature boxes with the 128-byte swizzle, into a 5-stage ring
 //               (32 KB per stage).  Rows past the frame's end read as zeros.
 //   warp 1      allocates TMEM (2 x 256 columns) and issues the MMAs from one
 //               thread: both operands are MN-major in shared memory (features
 //               contiguous), 4 MMAs (16 tokens each) per chunk.
-//   warps 2..5  epilogue: TMEM -> registers -> A (+ lambda on the diagonal)
-//               and B rows in global memory, while the MMAs of the next slot
-//               run into the other TMEM buffer.
+//   warps 2..5  epilogue: TMEM -> registers -> 32-column chunks of A (+ lambda
+//               on the diagonal) and B, staged swizzled in shared memory and
+//               written by TMA stores, while the MMAs of the next slot run into
+//               the other TMEM buffer.
 // Every wait is bounded; a wait that runs out sets the timeout bit of the
 // error word and the CTA winds down (waiting, bounded, for its own copies).
 #include "sm100.cuh"
@@ -27,16 +28,19 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 6;
+constexpr int kStages = 5;
 constexpr int kChunk = 64;                    // tokens per stage
 constexpr int kBox = 64 * 64 * 2;             // one 64 x 64 bf16 box: 8 KB
 constexpr int kStageBytes = 4 * kBox;         // K lo/hi features, V lo/hi features
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;           // two 256-column accumulators
+constexpr int kOutChunk = 128 * 32 * 4;       // epilogue staging: 32 float32 columns x 128 rows
+constexpr int kEpiBar = 1;                    // named barrier of the 4 epilogue warps
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, /*a MN*/ true, /*b MN*/ true);
 
 struct GramTcParams {
   CUtensorMap mK, mV, mKt, mVt;
+  CUtensorMap mA, mB;   // [slots * 128][128] float32, 32 x 128 boxes
   float* A;
   float* Bm;
   unsigned* err;
@@ -72,7 +76,8 @@ __global__ void __launch_bounds__(kThreads, 1) gram_tc_kernel(const __grid_const
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
-  Shared& sh = *reinterpret_cast<Shared*>(base + kStages * kStageBytes);
+  uint8_t* ostage = base + kStages * kStageBytes;   // 2 x output staging chunk
+  Shared& sh = *reinterpret_cast<Shared*>(ostage + 2 * kOutChunk);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -201,54 +206,66 @@ __global__ void __launch_bounds__(kThreads, 1) gram_tc_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // D row by row (lane = feature i) into swizzled 32-column staging chunks,
+    // each stored by one TMA store: chunks 0..3 are A (+ lambda on the
+    // diagonal), 4..7 are B.
     const int quarter = warp % 4;            // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;     // feature index i of D
-    int tb = 0;
+    const bool leader = (warp == 2 && lane == 0);
+    int tb = 0, nst = 0;
     uint32_t tphase = 0;
     for (int s = blockIdx.x; s < slots; s += gridDim.x) {
       int rows, z;
       bool text;
       slot_info(p, s, rows, z, text);
-      float* Ar = p.A + (size_t)s * 128 * 128 + (size_t)row * 128;
-      float* Br = p.Bm + (size_t)s * 128 * 128 + (size_t)row * 128;
-      if (rows == 0) {  // no tokens: A = lambda I, B = 0
-        for (int c = 0; c < 128; c += 4) {
-          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (row >= c && row < c + 4) (&a.x)[row - c] = p.lam;
-          *reinterpret_cast<float4*>(Ar + c) = a;
-          *reinterpret_cast<float4*>(Br + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        continue;
-      }
-      // Keep the warp converged: tcgen05.ld below is a warp-wide instruction.
       if (__any_sync(0xffffffffu, aborted(sh))) break;
-      const bool ok = mbar_wait(&sh.tfull[tb], tphase);
-      if (!__all_sync(0xffffffffu, ok)) {
-        set_abort(sh, p.err);
-        break;
+      if (rows > 0) {
+        const bool ok = mbar_wait(&sh.tfull[tb], tphase);
+        if (!__all_sync(0xffffffffu, ok)) {
+          set_abort(sh, p.err);
+          break;
+        }
+        tc_fence_after();
       }
-      tc_fence_after();
       const uint32_t taddr = tmem + tb * 256 + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int chunk = 0; chunk < 8; ++chunk) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + chunk * 32, r);
-        tmem_ld_wait();
-        float* dst = chunk < 4 ? Ar + chunk * 32 : Br + (chunk - 4) * 32;
-        const int col0 = chunk * 32;
+        if (rows > 0) {
+          tmem_ld_32x32b_x32(taddr + chunk * 32, r);
+          tmem_ld_wait();
+        } else {  // no tokens: A = lambda I, B = 0
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          float4 v = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                 __uint_as_float(r[j + 3]));
-          if (chunk < 4 && row >= col0 + j && row < col0 + j + 4) (&v.x)[row - col0 - j] += p.lam;
-          *reinterpret_cast<float4*>(dst + j) = v;
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
         }
+        if (chunk < 4) {
+          const int j = row - chunk * 32;   // the diagonal entry, if in this chunk
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (jj == j) r[jj] = __float_as_uint(__uint_as_float(r[jj]) + p.lam);
+        }
+        uint8_t* stg = ostage + (nst & 1) * kOutChunk;
+        if (leader) bulk_wait_read<1>();      // the store two chunks back has read this buffer
+        named_bar_sync(kEpiBar, 128);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(stg + sw128(row, q)) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(kEpiBar, 128);
+        if (leader) {
+          tma_store_2d(chunk < 4 ? &p.mA : &p.mB, stg, (chunk % 4) * 32, s * 128);
+          bulk_commit();
+        }
+        ++nst;
       }
-      tc_fence_before();
-      mbar_arrive(&sh.tempty[tb]);
-      tb ^= 1;
-      if (tb == 0) tphase ^= 1;
+      if (rows > 0) {
+        tc_fence_before();
+        mbar_arrive(&sh.tempty[tb]);
+        tb ^= 1;
+        if (tb == 0) tphase ^= 1;
+      }
     }
+    if (leader) bulk_wait<0>();               // A and B stores complete before exit
   }
 
   tc_fence_before();
@@ -269,6 +286,9 @@ cudaError_t launch_gram_tc(const vda_problem& p, const __nv_bfloat16* K, const _
     return cudaErrorInvalidValue;
   if (p.n_txt > 0 && (!make_bf16_rows_map(&prm.mKt, Kt, p.n_txt, BH, 64) || !make_bf16_rows_map(&prm.mVt, Vt, p.n_txt, BH, 64)))
     return cudaErrorInvalidValue;
+  const long long rows = (long long)BH * (p.T + 1) * 128;
+  if (!make_f32_rows_map(&prm.mA, A, rows, 128) || !make_f32_rows_map(&prm.mB, Bm, rows, 128))
+    return cudaErrorInvalidValue;
   prm.A = A;
   prm.Bm = Bm;
   prm.err = err;
@@ -277,7 +297,7 @@ cudaError_t launch_gram_tc(const vda_problem& p, const __nv_bfloat16* K, const _
   prm.n = p.n;
   prm.n_txt = p.n_txt;
   prm.lam = p.lambda;
-  const size_t smem = 1024 + kStages * kStageBytes + sizeof(Shared);
+  const size_t smem = 1024 + kStages * kStageBytes + 2 * kOutChunk + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;

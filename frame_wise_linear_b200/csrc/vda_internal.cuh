@@ -65,12 +65,6 @@ cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool sp
 cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
                            unsigned* err, cudaStream_t st);
 
-// Gram and factor fused (vda_gram_factor_tc.cu): bf16, d_k = d_v = 128.
-// Writes M_t (split layout, as launch_factor with split_bf16) and B_t.
-cudaError_t launch_gram_factor_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                                  const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* M, float* Bm,
-                                  unsigned* err, cudaStream_t st);
-
 // Tensor-core Gram (vda_gram_tc.cu): bf16 inputs, d_k = d_v = 128.  Writes
 // the same A and B slots as launch_gram_simt.
 cudaError_t launch_gram_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
@@ -85,6 +79,9 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
 // TMA descriptor of a [items][rows][128] bf16 tensor, boxes of 64 features x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
 bool make_bf16_rows_map(CUtensorMap* m, const void* ptr, int rows, int items, int box_rows);
+// TMA descriptor of a [rows][128] float32 matrix, boxes of 32 columns x
+// box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
+bool make_f32_rows_map(CUtensorMap* m, const void* ptr, long long rows, int box_rows);
 
 // Replaces the thread-local message vda_last_error() returns (vda_api.cu).
 void set_error_message(const char* msg);

@@ -17,7 +17,8 @@
 // The recurrence is independent per column of S, so each chain is split over
 // kSplit CTAs of N = 128 / kSplit columns.  CTA layout (160 threads):
 //   warps 0..3  own TMEM lanes = rows of S: build X (row m) in shared memory,
-//               then read S_t back from TMEM and store it;
+//               then read S_t back from TMEM and stage it (double-buffered,
+//               swizzled) for a TMA store;
 //   warp 4      one thread: bulk-copies M_t (64 KB) into a 2-stage ring ahead
 //               of time and issues the 24 MMAs of each step.
 // Every wait is bounded; a timeout sets the error bit and the CTA winds down.
@@ -34,9 +35,12 @@ constexpr int N = 128 / kSplit;              // columns of S per CTA
 constexpr int kThreads = 160;
 constexpr int kMBytes = 65536;               // M_t hi | lo
 constexpr int kXHalf = (N / 64) * 16384;     // X hi (or lo): N/64 blocks of 128 rows x 128 B
+constexpr int kSStage = N * 128 * 4;         // S_t staging: N/32 boxes of 128 rows x 128 B
+constexpr int kEpiBar = 1;                   // named barrier of the 4 row warps
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, N, /*a MN*/ false, /*b MN*/ true);
 
 struct ScanTcParams {
+  CUtensorMap mSF, mSB; // [frames * 128][128] float32, 32 x 128 boxes
   const uint8_t* M;     // per slot 64 KB: M hi (32 KB) | M lo (32 KB)
   const float* Bm;      // per slot 128 x 128 float
   float* SF;
@@ -77,7 +81,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* mring = base;                     // 2 x 64 KB
   uint8_t* xbuf = base + 2 * kMBytes;        // X hi | X lo
-  Shared& sh = *reinterpret_cast<Shared*>(xbuf + 2 * kXHalf);
+  uint8_t* sstage = xbuf + 2 * kXHalf;       // 2 x S_t staging (double-buffered)
+  Shared& sh = *reinterpret_cast<Shared*>(sstage + 2 * kSStage);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -223,13 +228,27 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         for (int j = 0; j < 32; ++j) srow[c * 32 + j] = __uint_as_float(r[j]);
       }
       if (s > 0) {
+        // S_t row m -> swizzled staging (32-column boxes) -> TMA store.
         const int t = dir == 0 ? s : T + 1 - s;
-        float* out = (dir == 0 ? p.SF : p.SB) + (((size_t)bh * T + (t - 1)) * 128 + m) * 128 + c0;
+        uint8_t* stg = sstage + (s & 1) * kSStage;
+        if (warp == 0 && lane == 0) bulk_wait_read<1>();   // the store two steps back has read this buffer
+        named_bar_sync(kEpiBar, 128);
 #pragma unroll
-        for (int j = 0; j < N; j += 4)
-          *reinterpret_cast<float4*>(out + j) = make_float4(srow[j], srow[j + 1], srow[j + 2], srow[j + 3]);
+        for (int q = 0; q < N / 4; ++q)
+          *reinterpret_cast<float4*>(stg + (q / 8) * 16384 + sw128(m, q % 8)) =
+              make_float4(srow[4 * q], srow[4 * q + 1], srow[4 * q + 2], srow[4 * q + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(kEpiBar, 128);
+        if (warp == 0 && lane == 0) {
+          const CUtensorMap* map = dir == 0 ? &p.mSF : &p.mSB;
+          const int y = ((bh * T) + (t - 1)) * 128;
+#pragma unroll
+          for (int b = 0; b < N / 32; ++b) tma_store_2d(map, stg + b * 16384, c0 + 32 * b, y);
+          bulk_commit();
+        }
       }
     }
+    if (warp == 0 && lane == 0) bulk_wait<0>();   // S stores complete before exit
   }
 
   tc_fence_before();
@@ -243,6 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
 cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
                            unsigned* err, cudaStream_t st) {
   ScanTcParams prm;
+  memset(&prm, 0, sizeof(prm));
+  const long long rows = (long long)p.B * p.H * p.T * 128;
+  if (!make_f32_rows_map(&prm.mSF, SF, rows, 128) || !make_f32_rows_map(&prm.mSB, SB, rows, 128))
+    return cudaErrorInvalidValue;
   prm.M = reinterpret_cast<const uint8_t*>(M);
   prm.Bm = Bm;
   prm.SF = SF;
@@ -250,7 +273,7 @@ cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm
   prm.err = err;
   prm.T = p.T;
   prm.lam = p.lambda;
-  const size_t smem = 1024 + 2 * kMBytes + 2 * kXHalf + sizeof(Shared);
+  const size_t smem = 1024 + 2 * kMBytes + 2 * kXHalf + 2 * kSStage + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(kSplit, 2, p.B * p.H);

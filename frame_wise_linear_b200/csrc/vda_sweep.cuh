@@ -7,8 +7,9 @@
 // which are the positive LDL^T pivots of an SPD matrix); after all pivots the
 // matrix is -A^{-1}.  Each pivot is one symmetric rank-1 update: with
 // x = column k (x_k := -1), p = 1/a_kk and row/column k zeroed, a -= x (p x)^T.
-// Pivots go in pairs: the owners publish columns k and k + 1, one barrier per
-// pair, and every thread derives the second pivot's column from the two.
+// Pivots go in pairs: the owners publish columns k and k + 1 and the pair's
+// scalars, one barrier per pair, and every thread derives the second pivot's
+// column from the two.
 #pragma once
 
 #include "sm100.cuh"
@@ -32,15 +33,25 @@ __device__ __forceinline__ bool block_of(int tid, int& R, int& C) {
 }
 
 // Runs all D pivots on `a` (this thread's block).  `xs` is shared scratch of
-// [2][2][D] floats (16-byte aligned); `sync` is a barrier over all threads
-// taking part (inactive ones included).  Returns true if a pivot was not
-// positive and finite.  On return a holds this block of -A^{-1}.
+// [2][2][D] floats and `sc` of [2][4] floats (16-byte aligned); `sync` is a
+// barrier over all threads taking part (inactive ones included).  Returns
+// true if a pivot was not positive and finite.  On return a holds this block
+// of -A^{-1}.
+//
+// Each pivot is applied without zeroing its row and column: with
+// x = column k except x_k = a_kk - 1 and p = 1/a_kk, the update
+// a -= x (p x)^T leaves exactly the swept row and column k, and the swept
+// diagonal entry after subtracting a further 2.  For the second pivot of a
+// pair, column k + 1 after the first is v - x g with g = p u_{k+1}.
 template <int D, typename Sync>
-__device__ __forceinline__ bool invert(float (&a)[8][8], int R, int C, bool active, float (*xs)[2][D], Sync sync) {
+__device__ __forceinline__ bool invert(float (&a)[8][8], int R, int C, bool active, float (*xs)[2][D],
+                                       float (*sc)[4], Sync sync) {
   constexpr int NB = D / 8;
   bool bad = false;
 
-  // Publishes columns k and k + 1 = 8K + kk, 8K + kk + 1 (current values) into buffer b.
+  // Publishes columns k and k + 1 = 8K + kk, 8K + kk + 1 (current values) into
+  // buffer b; the owner of the diagonal block also publishes the pair's
+  // scalars p1 = 1/a_kk, g = p1 a_{k+1,k} and p2 = 1/(a_{k+1,k+1} - a_{k+1,k} g).
   auto publish = [&](int K, auto kk_c, int b) {
     constexpr int kk = decltype(kk_c)::value;
     if (!active) return;
@@ -58,6 +69,16 @@ __device__ __forceinline__ bool invert(float (&a)[8][8], int R, int C, bool acti
         xs[b][1][8 * C + c] = a[kk + 1][c];
       }
     }
+    if (R == K && C == K) {
+      const float uk = a[kk][kk], uk1 = a[kk + 1][kk], vk1 = a[kk + 1][kk + 1];
+      const float p1 = 1.f / uk;
+      const float g = p1 * uk1;
+      const float piv2 = vk1 - uk1 * g;
+      if (!(uk > 0.f) || !isfinite(uk) || !(piv2 > 0.f) || !isfinite(piv2)) bad = true;
+      sc[b][0] = p1;
+      sc[b][1] = g;
+      sc[b][2] = 1.f / piv2;
+    }
   };
   auto load8 = [&](const float* src, float (&v)[8]) {
     const float4 lo = *reinterpret_cast<const float4*>(src);
@@ -70,83 +91,44 @@ __device__ __forceinline__ bool invert(float (&a)[8][8], int R, int C, bool acti
   int buf = 0;
 #pragma unroll 1
   for (int K = 0; K < NB; ++K) {
-    // Two pivots k = 8K + kk and k + 1 per barrier.  With u, v the columns
-    // before both: pivot k uses x = u (x_k = -1), p1 = 1/u_k; column k + 1
-    // after it is v' = v - u p1 u_{k+1} (v'_k = p1 u_{k+1}); pivot k + 1 uses
-    // y = v' (y_{k+1} = -1), p2 = 1/v'_{k+1}.
     auto pair = [&](auto kk_c) {
       constexpr int kk = decltype(kk_c)::value;
       sync();
-      const float uk = xs[buf][0][8 * K + kk];
-      const float uk1 = xs[buf][0][8 * K + kk + 1];
-      const float vk1 = xs[buf][1][8 * K + kk + 1];
-      const float p1 = 1.f / uk;
-      const float g = p1 * uk1;                 // v' = v - u g
-      const float piv2 = vk1 - uk1 * g;
-      const float p2 = 1.f / piv2;
       if (active) {
-        if (R == K && C == K && (!(uk > 0.f) || !isfinite(uk) || !(piv2 > 0.f) || !isfinite(piv2))) bad = true;
-        float ur[8], uc[8];
-        load8(&xs[buf][0][8 * R], ur);
-        load8(&xs[buf][0][8 * C], uc);
+        const float4 s4 = *reinterpret_cast<const float4*>(sc[buf]);
+        const float p1 = s4.x, g = s4.y, p2 = s4.z;
+        const bool rk = (R == K), ck = (C == K);
+        float xr[8], xc[8], yc[8];
+        load8(&xs[buf][0][8 * R], xr);
+        load8(&xs[buf][0][8 * C], xc);
+        if (rk) xr[kk] -= 1.f;
+        if (ck) xc[kk] -= 1.f;
         // ---- pivot k
-        {
-          float xr[8], yc[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            xr[i] = ur[i];
-            yc[i] = uc[i];
-          }
-          if (R == K) xr[kk] = -1.f;
-          if (C == K) yc[kk] = -1.f;
+        for (int i = 0; i < 8; ++i) yc[i] = p1 * xc[i];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) yc[i] *= p1;
-          if (R == K) {
+        for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) a[kk][c] = 0.f;
-          }
-          if (C == K) {
+          for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-xr[r], yc[c], a[r][c]);
+        if (rk && ck) a[kk][kk] -= 2.f;
+        // ---- pivot k + 1: x' = v - x g, x'_{k+1} -= 1
+        float vr[8], vc[8];
+        load8(&xs[buf][1][8 * R], vr);
+        load8(&xs[buf][1][8 * C], vc);
 #pragma unroll
-            for (int r = 0; r < 8; ++r) a[r][kk] = 0.f;
-          }
-#pragma unroll
-          for (int r = 0; r < 8; ++r)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-xr[r], yc[c], a[r][c]);
+        for (int i = 0; i < 8; ++i) {
+          vr[i] = fmaf(-xr[i], g, vr[i]);
+          vc[i] = fmaf(-xc[i], g, vc[i]);
         }
-        // ---- pivot k + 1
-        {
-          float vr[8], vc[8];
-          load8(&xs[buf][1][8 * R], vr);
-          load8(&xs[buf][1][8 * C], vc);
+        if (rk) vr[kk + 1] -= 1.f;
+        if (ck) vc[kk + 1] -= 1.f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            vr[i] = fmaf(-ur[i], g, vr[i]);
-            vc[i] = fmaf(-uc[i], g, vc[i]);
-          }
-          if (R == K) {
-            vr[kk] = g;
-            vr[kk + 1] = -1.f;
-          }
-          if (C == K) {
-            vc[kk] = g;
-            vc[kk + 1] = -1.f;
-          }
+        for (int i = 0; i < 8; ++i) yc[i] = p2 * vc[i];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) vc[i] *= p2;
-          if (R == K) {
+        for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) a[kk + 1][c] = 0.f;
-          }
-          if (C == K) {
-#pragma unroll
-            for (int r = 0; r < 8; ++r) a[r][kk + 1] = 0.f;
-          }
-#pragma unroll
-          for (int r = 0; r < 8; ++r)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-vr[r], vc[c], a[r][c]);
-        }
+          for (int c = 0; c < 8; ++c) a[r][c] = fmaf(-vr[r], yc[c], a[r][c]);
+        if (rk && ck) a[kk + 1][kk + 1] -= 2.f;
       }
       buf ^= 1;
       if constexpr (kk + 2 < 8) {
