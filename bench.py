@@ -42,7 +42,7 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # Kernel of each stage and the source file that defines it (for ncu traffic lookups).
 STAGE_SOURCES = {
     "gram": "frame_wise_linear_b200/csrc/vda_gram_tc.cu",
-    "factor": "frame_wise_linear_b200/csrc/vda_factor.cu",
+    "factor": "frame_wise_linear_b200/csrc/vda_factor_tc.cu",
     "scan": "frame_wise_linear_b200/csrc/vda_scan_tc.cu",
     "readout": "frame_wise_linear_b200/csrc/vda_readout_tc.cu",
 }

@@ -122,7 +122,11 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
       return cuda_fail(e, "gram launch");
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
-  if ((e = vda::launch_factor(p, M, err, kBf16, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
+  if constexpr (kBf16) {
+    if ((e = vda::launch_factor_tc(p, M, err, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
+  } else {
+    if ((e = vda::launch_factor(p, M, err, false, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
+  }
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
   if constexpr (kBf16) {
     if ((e = vda::launch_scan_tc(p, M, C, SF, SB, err, st)) != cudaSuccess) return cuda_fail(e, "scan launch");

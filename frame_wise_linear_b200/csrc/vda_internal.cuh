@@ -60,6 +60,10 @@ cudaError_t launch_readout_simt(const vda_problem& p, const TIn* Q, const TIn* G
 // (32 KB each, same 64 KB per slot).
 cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool split_bf16, cudaStream_t st);
 
+// Tensor-core factor step (vda_factor_tc.cu): bf16 path, d_k = 128; same
+// output as launch_factor with split_bf16.
+cudaError_t launch_factor_tc(const vda_problem& p, float* M, unsigned* err, cudaStream_t st);
+
 // Tensor-core scan (vda_scan_tc.cu): bf16 path, d_k = d_v = 128; M in the
 // split layout above, B_t float32 in the C region.
 cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,

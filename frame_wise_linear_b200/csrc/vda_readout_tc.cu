@@ -13,12 +13,13 @@
 //   warp 0      TMA producer: Q tiles (3-stage ring) and G tiles (2-stage ring),
 //               each tile as two 64-feature boxes with the 128-byte swizzle.
 //   warp 1      TMEM (2 x 128 columns) and the MMAs (one thread).
-//   warps 2..9  at each new frame: S = S^f + S^b split into bf16 hi/lo in
-//               shared memory (the MMA B operand); per tile: TMEM -> registers,
-//               gate from the G tile, O written over the G tile in shared
-//               memory, then a TMA store per 64-column half.  Warps 2..5 take
-//               columns 0..63 and warps 6..9 columns 64..127 (two warps per
-//               TMEM lane quarter).
+//   warps 2..9  per tile: TMEM -> registers, gate from the G tile, O written
+//               over the G tile in shared memory, then a TMA store per
+//               64-column half.  Warps 2..5 take columns 0..63 and warps 6..9
+//               columns 64..127 (two warps per TMEM lane quarter).
+//   warps 10..17 S = S^f + S^b of the next frame, loaded into registers a
+//               whole frame ahead, then split into bf16 hi/lo in shared memory
+//               (the MMA B operand) as soon as the MMAs release the buffer.
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
@@ -35,7 +36,7 @@ constexpr int kRows = 128;                   // tokens per tile
 constexpr int kBox = kRows * 64 * 2;         // 128 rows x 64 features bf16: 16 KB
 constexpr int kTile = 2 * kBox;              // 32 KB
 constexpr int kSig = 2 * kTile;              // S_hi and S_lo, 32 KB each
-constexpr int kThreads = 320;              // 2 control warps + 8 epilogue warps
+constexpr int kThreads = 576;              // 2 control warps + 8 epilogue warps + 8 prep warps
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
 
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       mbar_init(&sh.t_full[i], 1);
       mbar_init(&sh.t_empty[i], 256);
     }
-    mbar_init(&sh.sig_full, 256);
+    mbar_init(&sh.sig_full, 256);   // the 8 prep warps
     mbar_init(&sh.sig_empty, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -195,58 +196,18 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       mma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
     }
-  } else {
-    // ------------------------------------------------------------ S prep + epilogue
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;          // 0..255
     const int quarter = warp % 4;             // TMEM lanes this warp may access
     const int half = (warp - 2) / 4;          // column half 0..63 or 64..127
     const int row = quarter * 32 + lane;      // tile row this thread owns in TMEM
-    const int srow_i = et % 128;              // row of S this thread prepares
-    const int shalf = et / 128;               // and which 64 of its columns
-    int gs = 0, tb = 0, cur_u = -1;
-    uint32_t gph = 0, tph = 0, seph = 0;
+    int gs = 0, tb = 0;
+    uint32_t gph = 0, tph = 0;
     for (int tile = t_begin; tile < t_end; ++tile) {
       const int u = tile / p.tiles_per_unit;
       const int y = (tile % p.tiles_per_unit) * kRows;
       if (__any_sync(0xffffffffu, aborted(sh))) break;
-      if (u != cur_u) {
-        const bool ok = mbar_wait(&sh.sig_empty, seph ^ 1);
-        if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
-        seph ^= 1;
-        // S = S^f + S^b, row srow_i, columns 64*shalf .. +63: split into hi/lo
-        // bf16, MN-major swizzled (the MMA B operand).
-        const float4* f = reinterpret_cast<const float4*>(p.SF + ((size_t)u * 128 + srow_i) * 128 + 64 * shalf);
-        const float4* b = reinterpret_cast<const float4*>(p.SB + ((size_t)u * 128 + srow_i) * 128 + 64 * shalf);
-        float4 fv[16], bv[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          fv[c] = __ldg(f + c);
-          bv[c] = __ldg(b + c);
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {   // 8 columns per chunk
-          const float4 f0 = fv[2 * c], f1 = fv[2 * c + 1];
-          const float4 b0 = bv[2 * c], b1 = bv[2 * c + 1];
-          const float x[8] = {f0.x + b0.x, f0.y + b0.y, f0.z + b0.z, f0.w + b0.w,
-                              f1.x + b1.x, f1.y + b1.y, f1.z + b1.z, f1.w + b1.w};
-          float hi[8], lo[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
-            lo[i] = x[i] - hi[i];
-          }
-          const uint32_t off = shalf * kBox + sw128(srow_i, c);
-          *reinterpret_cast<uint4*>(sig + off) =
-              make_uint4(pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]),
-                         pack_bf16(hi[6], hi[7]));
-          *reinterpret_cast<uint4*>(sig + kTile + off) =
-              make_uint4(pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]),
-                         pack_bf16(lo[6], lo[7]));
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&sh.sig_full);
-        cur_u = u;
-      }
       bool ok = mbar_wait(&sh.t_full[tb], tph);
       ok = ok && mbar_wait(&sh.g_full[gs], gph);
       if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
@@ -290,6 +251,54 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       if (tb == 0) tph ^= 1;
     }
     if (et % 128 == 0) bulk_wait<0>();         // O stores complete before exit
+  } else {
+    // ------------------------------------------------------------ S prep
+    // Row srow of S = S^f + S^b, columns 64*shalf .. +63, for each frame of this
+    // CTA's range in order: loaded into registers as soon as the previous
+    // frame's S is in shared memory, written (split) once the MMAs release it.
+    const int pt = threadIdx.x - 320;         // 0..255
+    const int srow = pt % 128;
+    const int shalf = pt / 128;
+    const int u_first = t_begin / p.tiles_per_unit;
+    const int u_last = t_end > t_begin ? (t_end - 1) / p.tiles_per_unit : u_first - 1;
+    uint32_t seph = 0;
+    float x[64];
+    auto load = [&](int u) {
+      const float4* f = reinterpret_cast<const float4*>(p.SF + ((size_t)u * 128 + srow) * 128 + 64 * shalf);
+      const float4* b = reinterpret_cast<const float4*>(p.SB + ((size_t)u * 128 + srow) * 128 + 64 * shalf);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float4 fv = __ldg(f + c), bv = __ldg(b + c);
+        x[4 * c] = fv.x + bv.x;
+        x[4 * c + 1] = fv.y + bv.y;
+        x[4 * c + 2] = fv.z + bv.z;
+        x[4 * c + 3] = fv.w + bv.w;
+      }
+    };
+    if (u_first <= u_last) load(u_first);
+    for (int u = u_first; u <= u_last; ++u) {
+      const bool ok = mbar_wait(&sh.sig_empty, seph ^ 1);
+      if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
+      seph ^= 1;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {   // 8 columns per 16-byte chunk
+        float hi[8], lo[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          hi[i] = __bfloat162float(__float2bfloat16_rn(x[8 * c + i]));
+          lo[i] = x[8 * c + i] - hi[i];
+        }
+        const uint32_t off = shalf * kBox + sw128(srow, c);
+        *reinterpret_cast<uint4*>(sig + off) =
+            make_uint4(pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]), pack_bf16(hi[6], hi[7]));
+        *reinterpret_cast<uint4*>(sig + kTile + off) =
+            make_uint4(pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]), pack_bf16(lo[6], lo[7]));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sh.sig_full);
+      if (u + 1 <= u_last) load(u + 1);
+      if (__any_sync(0xffffffffu, aborted(sh))) break;
+    }
   }
 
   tc_fence_before();
