@@ -16,11 +16,13 @@
 //
 // Layout: one CTA of 4 warps per slot; A lives in TMEM as a 128 x 128 float32
 // accumulator (lane i = row i).  Per block: each thread reads its row's 8
-// pivot columns from TMEM; the 8 lanes holding P factor it (8 x 8 Cholesky
-// over warp shuffles); each thread solves for its row of Y; Y goes to shared
-// memory as tf32 hi + lo (both rounded to nearest, about 2^-24 together); one
-// thread issues the symmetric rank-8 update as four kind::tf32 MMAs (all
-// hi/lo products of Y Y^T, A negated), float32-level accuracy.  Up to 4 CTAs
+// pivot columns from TMEM; the 8 rows of P publish them in shared memory and
+// every thread factors P in registers (rsqrt, no divides: a short dependency
+// chain instead of a one-warp Cholesky that the other warps would wait for);
+// each thread solves for its row of Y; Y goes to shared
+// memory as tf32 hi + lo (both rounded to nearest, about 2^-22 together); one
+// thread issues the symmetric rank-8 update as three kind::tf32 MMAs (the
+// hi/lo products of Y Y^T above float32 rounding, A negated).  Up to 4 CTAs
 // share an SM (128 TMEM columns each).  M is written as bf16 hi/lo in the
 // scan's MMA operand layout.  A non-positive or non-finite pivot sets the
 // NOT_SPD bit; every wait is bounded.
@@ -38,7 +40,8 @@ constexpr int kOp = 128 * 8 * 4;              // one operand: 128 rows x 8 tf32 
 constexpr uint32_t kIdesc = idesc_tf32_f32(128, 128, /*negate A*/ true);
 
 struct Shared {
-  uint64_t mma_done;
+  uint64_t mma_done;     // one phase per step: the step's update has completed
+  uint64_t final_done;   // every MMA of the CTA has completed
   uint32_t tmem_base;
   int bad;
   int abort;
@@ -59,8 +62,7 @@ __device__ __forceinline__ void store_op(uint8_t* op, int i, const float (&v)[8]
 __global__ void __launch_bounds__(kThreads) factor_tc_kernel(float* __restrict__ Mreg, float lam,
                                                              unsigned* __restrict__ err) {
   __shared__ __align__(1024) uint8_t ops[2 * kOp];   // Y hi | Y lo
-  __shared__ __align__(16) float lsm[8][8];           // L of the pivot block (lower)
-  __shared__ __align__(16) float dinv[8];             // 1 / L_jj
+  __shared__ __align__(16) float psm[8][8];           // the pivot block P of this step
   __shared__ Shared sh;
 
   const int i = threadIdx.x;            // row of A = TMEM lane
@@ -69,6 +71,7 @@ __global__ void __launch_bounds__(kThreads) factor_tc_kernel(float* __restrict__
 
   if (i == 0) {
     mbar_init(&sh.mma_done, 1);
+    mbar_init(&sh.final_done, 1);
     sh.bad = 0;
     sh.abort = 0;
     fence_barrier_init();
@@ -105,8 +108,6 @@ __global__ void __launch_bounds__(kThreads) factor_tc_kernel(float* __restrict__
   __syncthreads();
   tc_fence_after();
 
-  const uint32_t opaddr = smem_u32(ops);
-  bool bad = false;
   int steps_issued = 0;
 #pragma unroll 1
   for (int K = 0; K < 16; ++K) {
@@ -124,42 +125,51 @@ __global__ void __launch_bounds__(kThreads) factor_tc_kernel(float* __restrict__
 #pragma unroll
       for (int j = 0; j < 8; ++j) x[j] = __uint_as_float(r[j]);
     }
-    // ---- P = L L^T: rows 8K..8K+7 are lanes l0..l0+7 of warp K/4.
-    if (warp == K / 4) {
-      const int l0 = 8 * (K % 4);
-      const int r = lane - l0;
-      const bool mine = (r >= 0 && r < 8);
-      float a[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) a[j] = x[j];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float piv = __shfl_sync(0xffffffffu, a[j], l0 + j);   // current a_jj
-        if (mine && r == j && (!(piv > 0.f) || !isfinite(piv))) bad = true;
-        const float d = sqrtf(piv);
-        const float lj = (r == j) ? d : a[j] / d;                    // L_rj (rows r >= j)
-        a[j] = lj;
-#pragma unroll
-        for (int m = j + 1; m < 8; ++m) {
-          const float lmj = __shfl_sync(0xffffffffu, lj, l0 + m);    // L_mj
-          if (m <= r) a[m] = fmaf(-lj, lmj, a[m]);
-        }
-      }
-      if (mine) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) lsm[r][j] = (j <= r) ? a[j] : 0.f;
-        dinv[r] = 1.f / a[r];
-      }
+    // ---- P = L L^T.  The 8 rows of the pivot block publish their pivot
+    // columns; every thread then factors P itself, in registers (rsqrt, no
+    // divides; the same operations in the same order, so every copy is
+    // identical).  A short dependency chain, and no warp waits for another.
+    if ((i >> 3) == K) {
+      *reinterpret_cast<float4*>(&psm[i & 7][0]) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(&psm[i & 7][4]) = make_float4(x[4], x[5], x[6], x[7]);
     }
     __syncthreads();
+    float l[8][8];     // lower triangle: P, then L
+    float dinv[8];     // 1 / L_jj
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+#pragma unroll
+      for (int c = 0; c <= r; ++c) l[r][c] = psm[r][c];
+    }
+    {
+      bool badp = false;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float piv = l[j][j];
+        badp |= !(piv > 0.f) || !isfinite(piv);
+        const float rs = rsqrtf(piv);
+        dinv[j] = rs;
+#pragma unroll
+        for (int r = j + 1; r < 8; ++r) l[r][j] *= rs;
+#pragma unroll
+        for (int r = j + 1; r < 8; ++r) {
+#pragma unroll
+          for (int c = j + 1; c <= r; ++c) l[r][c] = fmaf(-l[r][j], l[c][j], l[r][c]);
+        }
+      }
+      if (i == 0 && badp) sh.bad = 1;
+    }
     // ---- X~ (row i) and Y = X~ L^{-T}: forward substitution L y = x~.
-    if ((i >> 3) == K) x[i & 7] -= 1.f;
+    if ((i >> 3) == K) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] -= (j == (i & 7)) ? 1.f : 0.f;   // static indices only
+    }
     float y[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float acc = x[j];
 #pragma unroll
-      for (int m = 0; m < j; ++m) acc = fmaf(-lsm[j][m], y[m], acc);
+      for (int m = 0; m < j; ++m) acc = fmaf(-l[j][m], y[m], acc);
       y[j] = acc * dinv[j];
     }
     // ---- tf32 hi + lo operand (row i)
@@ -178,22 +188,24 @@ __global__ void __launch_bounds__(kThreads) factor_tc_kernel(float* __restrict__
     __syncthreads();
     if (i == 0) {
       tc_fence_after();
-      // Y is both operands: A = Y (M x K), B = Y^T (K x N) read K-major from the same rows.
+      // A -= Y Y^T: Y is the A operand (M x K) and, read K-major from the same
+      // rows, the B operand (K x N).  Three tf32 passes: hi hi, hi lo, lo hi;
+      // the lo lo product is below float32 rounding of the update.
+      const uint32_t opaddr = smem_u32(ops);
       const uint64_t yhi = smem_desc(opaddr + 0 * kOp, 2048, 128, kSwizzleNone);
       const uint64_t ylo = smem_desc(opaddr + 1 * kOp, 2048, 128, kSwizzleNone);
-      mma_tf32_ss(tmem, yhi, yhi, kIdesc, 1u);   // A -= Y Y^T in four tf32 passes
+      mma_tf32_ss(tmem, yhi, yhi, kIdesc, 1u);
       mma_tf32_ss(tmem, yhi, ylo, kIdesc, 1u);
       mma_tf32_ss(tmem, ylo, yhi, kIdesc, 1u);
-      mma_tf32_ss(tmem, ylo, ylo, kIdesc, 1u);
       mma_commit(&sh.mma_done);
     }
     ++steps_issued;
   }
-  if (bad) atomicOr(&sh.bad, 1);
 
-  // Wait (bounded) for the last update issued, also on the error path, so no
-  // MMA still runs when TMEM is released.
-  bool ok = steps_issued > 0 && mbar_wait(&sh.mma_done, (steps_issued - 1) & 1);
+  // One more commit covers every MMA issued; wait for it (bounded), also on
+  // the error path, so no MMA still runs when TMEM is read or released.
+  if (i == 0) mma_commit(&sh.final_done);
+  bool ok = steps_issued > 0 && mbar_wait(&sh.final_done, 0);
   if (!ok) *reinterpret_cast<volatile int*>(&sh.abort) = 1;
   tc_fence_after();
   __syncthreads();
@@ -240,7 +252,9 @@ cudaError_t launch_factor_tc(const vda_problem& p, float* M, unsigned* err, cuda
   if (p.d_k != 128) return cudaErrorInvalidValue;
   const unsigned slots = (unsigned)(p.B * p.H * (p.T + 1));
   // Unused dynamic shared memory that caps residency at 4 CTAs per SM, the
-  // number whose 128-column TMEM allocations fit (a fifth would wait in alloc).
+  // number whose 128-column TMEM allocations fit (a fifth would wait in
+  // alloc): with 8.5 KB static and 1 KB reserved per CTA, 4 x 53.5 KB fit in
+  // the SM's 228 KB and 5 do not.
   const int pad = 44 * 1024;
   cudaError_t e = cudaFuncSetAttribute(factor_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pad);
   if (e != cudaSuccess) return e;
