@@ -10,16 +10,18 @@
 //
 // Design (persistent, one CTA per SM, 6 warps), work = 128-row tiles of every
 // frame, a contiguous range of tiles per CTA:
-//   warp 0      TMA producer: Q tiles (3-stage ring) and G tiles (2-stage ring),
-//               each tile as two 64-feature boxes with the 128-byte swizzle.
+//   warp 0      TMA producer: Q tiles and G tiles (2-stage rings), each tile
+//               as two 64-feature boxes with the 128-byte swizzle.
 //   warp 1      TMEM (2 x 128 columns) and the MMAs (one thread).
-//   warps 2..9  per tile: TMEM -> registers, gate from the G tile, O written
+//   warps 2..9  per tile: TMEM -> registers, gate from the G tile (sigmoid
+//               as (1 + tanh(g/2)) / 2, one special-function op), O written
 //               over the G tile in shared memory, then a TMA store per
 //               64-column half.  Warps 2..5 take columns 0..63 and warps 6..9
 //               columns 64..127 (two warps per TMEM lane quarter).
-//   warps 10..17 S = S^f + S^b of the next frame, loaded into registers a
-//               whole frame ahead, then split into bf16 hi/lo in shared memory
-//               (the MMA B operand) as soon as the MMAs release the buffer.
+//   warps 10..17 S = S^f + S^b of the next frame, streamed by bulk copies
+//               through a 2-slot shared-memory ring into registers a frame
+//               ahead, then split into bf16 hi/lo in shared memory (the MMA B
+//               operand) as soon as the MMAs release the buffer.
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
@@ -30,12 +32,16 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kQStages = 3;
+constexpr int kQStages = 2;
 constexpr int kGStages = 2;
 constexpr int kRows = 128;                   // tokens per tile
 constexpr int kBox = kRows * 64 * 2;         // 128 rows x 64 features bf16: 16 KB
 constexpr int kTile = 2 * kBox;              // 32 KB
 constexpr int kSig = 2 * kTile;              // S_hi and S_lo, 32 KB each
+constexpr int kPieceRows = 16;               // S^f, S^b streamed in 16-row pieces
+constexpr int kPieces = 128 / kPieceRows;    // 8 pieces per frame
+constexpr int kPieceHalf = kPieceRows * 128 * 4;   // 8 KB of S^f (or S^b) per piece
+constexpr int kPiece = 2 * kPieceHalf;       // one staging slot: S^f piece | S^b piece
 constexpr int kThreads = 576;              // 2 control warps + 8 epilogue warps + 8 prep warps
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
@@ -54,6 +60,7 @@ struct Shared {
   uint64_t g_full[kGStages], g_empty[kGStages];
   uint64_t t_full[2], t_empty[2];
   uint64_t sig_full, sig_empty;
+  uint64_t p_full[2];   // S staging slots
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -76,7 +83,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
   uint8_t* sig = base;                              // S_hi | S_lo
   uint8_t* qbuf = base + kSig;                      // kQStages tiles
   uint8_t* gbuf = qbuf + kQStages * kTile;          // kGStages tiles (G in, O out)
-  Shared& sh = *reinterpret_cast<Shared*>(gbuf + kGStages * kTile);
+  uint8_t* sstage = gbuf + kGStages * kTile;        // 2 S staging slots
+  Shared& sh = *reinterpret_cast<Shared*>(sstage + 2 * kPiece);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -99,6 +107,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     }
     mbar_init(&sh.sig_full, 256);   // the 8 prep warps
     mbar_init(&sh.sig_empty, 1);
+    mbar_init(&sh.p_full[0], 1);
+    mbar_init(&sh.p_full[1], 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     fence_barrier_init();
@@ -230,8 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
           for (int e = 0; e < 4; ++e) {
             const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(&gw[e]);
             const float g0 = __low2float(g2), g1 = __high2float(g2);
-            const float d0 = __uint_as_float(r[q * 8 + 2 * e]), d1 = __uint_as_float(r[q * 8 + 2 * e + 1]);
-            ow[e] = pack_bf16(__fdividef(d0, 1.f + __expf(-g0)), __fdividef(d1, 1.f + __expf(-g1)));
+            // sigmoid(g) d = (1 + tanh(g / 2)) d / 2: one special-function op.
+            const float h0 = 0.5f * __uint_as_float(r[q * 8 + 2 * e]);
+            const float h1 = 0.5f * __uint_as_float(r[q * 8 + 2 * e + 1]);
+            ow[e] = pack_bf16(fmaf(h0, tanh_approx(0.5f * g0), h0), fmaf(h1, tanh_approx(0.5f * g1), h1));
           }
           *reinterpret_cast<uint4*>(rowp + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
@@ -253,42 +265,74 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     if (et % 128 == 0) bulk_wait<0>();         // O stores complete before exit
   } else {
     // ------------------------------------------------------------ S prep
-    // Row srow of S = S^f + S^b, columns 64*shalf .. +63, for each frame of this
-    // CTA's range in order: loaded into registers as soon as the previous
-    // frame's S is in shared memory, written (split) once the MMAs release it.
+    // S = S^f + S^b of each frame of this CTA's range, in order.  The frame's
+    // 8 pieces (16 rows of S^f and of S^b, 8 KB each, contiguous) arrive by
+    // bulk copy in a 2-slot ring, issued by the first prep thread as slots
+    // free up, so no global load goes through the load/store unit (a burst
+    // of them there stalls the epilogue's shared-memory traffic).  Thread pt
+    // keeps row 16 j + pt / 16, columns 8 (pt % 16) .. + 7 of every piece j
+    // in registers; once the MMAs release the operand buffer it writes them
+    // split into bf16 hi/lo and the next frame's pieces start.
     const int pt = threadIdx.x - 320;         // 0..255
-    const int srow = pt % 128;
-    const int shalf = pt / 128;
+    const int prow = pt / 16;                 // row inside a piece
+    const int pchunk = pt % 16;               // 8-column chunk
     const int u_first = t_begin / p.tiles_per_unit;
     const int u_last = t_end > t_begin ? (t_end - 1) / p.tiles_per_unit : u_first - 1;
-    uint32_t seph = 0;
-    float x[64];
-    auto load = [&](int u) {
-      const float4* f = reinterpret_cast<const float4*>(p.SF + ((size_t)u * 128 + srow) * 128 + 64 * shalf);
-      const float4* b = reinterpret_cast<const float4*>(p.SB + ((size_t)u * 128 + srow) * 128 + 64 * shalf);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 fv = __ldg(f + c), bv = __ldg(b + c);
-        x[4 * c] = fv.x + bv.x;
-        x[4 * c + 1] = fv.y + bv.y;
-        x[4 * c + 2] = fv.z + bv.z;
-        x[4 * c + 3] = fv.w + bv.w;
-      }
+    const int n_pieces = (u_last - u_first + 1) * kPieces;
+    auto issue = [&](int g) {                 // piece g of the sequence into slot g % 2
+      const int u = u_first + g / kPieces, j = g % kPieces;
+      const size_t off = ((size_t)u * 128 + (size_t)j * kPieceRows) * 128;
+      uint8_t* dst = sstage + (g & 1) * kPiece;
+      mbar_expect_tx(&sh.p_full[g & 1], kPiece);
+      bulk_load(dst, p.SF + off, kPieceHalf, &sh.p_full[g & 1]);
+      bulk_load(dst + kPieceHalf, p.SB + off, kPieceHalf, &sh.p_full[g & 1]);
     };
-    if (u_first <= u_last) load(u_first);
+    int issued = 0;
+    if (pt == 0) {
+      for (; issued < 2 && issued < n_pieces; ++issued) issue(issued);
+    }
+    uint32_t seph = 0;
+    int g = 0;                                 // pieces consumed
     for (int u = u_first; u <= u_last; ++u) {
-      const bool ok = mbar_wait(&sh.sig_empty, seph ^ 1);
-      if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
+      if (pt == 0 && u + 1 <= u_last) {
+        // Read about a frame from now: bring into L2 first.
+        bulk_prefetch_l2(p.SF + (size_t)(u + 1) * 128 * 128, 128 * 128 * 4);
+        bulk_prefetch_l2(p.SB + (size_t)(u + 1) * 128 * 128, 128 * 128 * 4);
+      }
+      float x[64];
+      bool ok = true;
+#pragma unroll
+      for (int j = 0; j < kPieces; ++j, ++g) {
+        ok = ok && mbar_wait(&sh.p_full[g & 1], (g >> 1) & 1);
+        const float* f = reinterpret_cast<const float*>(sstage + (g & 1) * kPiece) + prow * 128 + pchunk * 8;
+        const float* b = f + kPieceHalf / 4;
+        const float4 f0 = *reinterpret_cast<const float4*>(f), f1 = *reinterpret_cast<const float4*>(f + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(b), b1 = *reinterpret_cast<const float4*>(b + 4);
+        x[8 * j + 0] = f0.x + b0.x;
+        x[8 * j + 1] = f0.y + b0.y;
+        x[8 * j + 2] = f0.z + b0.z;
+        x[8 * j + 3] = f0.w + b0.w;
+        x[8 * j + 4] = f1.x + b1.x;
+        x[8 * j + 5] = f1.y + b1.y;
+        x[8 * j + 6] = f1.z + b1.z;
+        x[8 * j + 7] = f1.w + b1.w;
+        named_bar_sync(3, 256);                // every prep thread is done with the slot
+        if (pt == 0 && ok && issued < n_pieces) issue(issued++);
+      }
+      if (!ok) set_abort(sh, p.err);
+      ok = ok && !aborted(sh) && mbar_wait(&sh.sig_empty, seph ^ 1);
+      if (!ok) set_abort(sh, p.err);
+      if (named_bar_or(3, 256, !ok)) break;    // one decision for all prep threads
       seph ^= 1;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {   // 8 columns per 16-byte chunk
+      for (int j = 0; j < kPieces; ++j) {
         float hi[8], lo[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          hi[i] = __bfloat162float(__float2bfloat16_rn(x[8 * c + i]));
-          lo[i] = x[8 * c + i] - hi[i];
+        for (int e = 0; e < 8; ++e) {
+          hi[e] = __bfloat162float(__float2bfloat16_rn(x[8 * j + e]));
+          lo[e] = x[8 * j + e] - hi[e];
         }
-        const uint32_t off = shalf * kBox + sw128(srow, c);
+        const uint32_t off = (pchunk / 8) * kBox + sw128(j * kPieceRows + prow, pchunk % 8);
         *reinterpret_cast<uint4*>(sig + off) =
             make_uint4(pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]), pack_bf16(hi[6], hi[7]));
         *reinterpret_cast<uint4*>(sig + kTile + off) =
@@ -296,8 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       }
       fence_proxy_async_smem();
       mbar_arrive(&sh.sig_full);
-      if (u + 1 <= u_last) load(u + 1);
-      if (__any_sync(0xffffffffu, aborted(sh))) break;
+    }
+    if (pt == 0) {   // let the copies still in flight land before exit
+      for (int c = g; c < issued; ++c) mbar_wait(&sh.p_full[c & 1], (c >> 1) & 1);
     }
   }
 
@@ -323,7 +368,7 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
   prm.err = err;
   prm.units = units;
   prm.tiles_per_unit = (p.n + kRows - 1) / kRows;
-  const size_t smem = 1024 + kSig + (kQStages + kGStages) * kTile + sizeof(Shared);
+  const size_t smem = 1024 + kSig + (kQStages + kGStages) * kTile + 2 * kPiece + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
