@@ -17,8 +17,9 @@
 // The recurrence is independent per column of S, so each chain is split over
 // kSplit CTAs of N = 128 / kSplit columns.  CTA layout (160 threads):
 //   warps 0..3  own TMEM lanes = rows of S: build X (row m) in shared memory,
-//               then read S_t back from TMEM and stage it (double-buffered,
-//               swizzled) for a TMA store;
+//               stage the previous state (double-buffered, swizzled) for a
+//               TMA store while the step's MMAs run, then read S_t back from
+//               TMEM;
 //   warp 4      one thread: bulk-copies M_t (64 KB) into a 2-stage ring ahead
 //               of time and issues the 24 MMAs of each step.
 // Every wait is bounded; a timeout sets the error bit and the CTA winds down.
@@ -36,11 +37,14 @@ constexpr int kThreads = 160;
 constexpr int kMBytes = 65536;               // M_t hi | lo
 constexpr int kXHalf = (N / 64) * 16384;     // X hi (or lo): N/64 blocks of 128 rows x 128 B
 constexpr int kSStage = N * 128 * 4;         // S_t staging: N/32 boxes of 128 rows x 128 B
+constexpr int kBBuf = N * 128 * 4;           // B_t columns of this CTA, same layout
 constexpr int kEpiBar = 1;                   // named barrier of the 4 row warps
+constexpr int kAhead = 4;                    // steps of M_t and B_t prefetched into L2
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, N, /*a MN*/ false, /*b MN*/ true);
 
 struct ScanTcParams {
   CUtensorMap mSF, mSB; // [frames * 128][128] float32, 32 x 128 boxes
+  CUtensorMap mB;       // [slots * 128][128] float32, 32 x 128 boxes
   const uint8_t* M;     // per slot 64 KB: M hi (32 KB) | M lo (32 KB)
   const float* Bm;      // per slot 128 x 128 float
   float* SF;
@@ -52,7 +56,7 @@ struct ScanTcParams {
 
 struct Shared {
   uint64_t m_full[2], m_empty[2];
-  uint64_t x_full, d_full;
+  uint64_t x_full, d_full, b_full;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -74,8 +78,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* mring = base;                     // 2 x 64 KB
   uint8_t* xbuf = base + 2 * kMBytes;        // X hi | X lo
-  uint8_t* sstage = xbuf + 2 * kXHalf;       // 2 x S_t staging (double-buffered)
-  Shared& sh = *reinterpret_cast<Shared*>(sstage + 2 * kSStage);
+  uint8_t* sstage = xbuf + 2 * kXHalf;       // S_t staging
+  uint8_t* bbuf = sstage + kSStage;          // B_t (this CTA's columns)
+  Shared& sh = *reinterpret_cast<Shared*>(bbuf + kBBuf);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -93,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     }
     mbar_init(&sh.x_full, 128);
     mbar_init(&sh.d_full, 1);
+    mbar_init(&sh.b_full, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     fence_barrier_init();
@@ -109,6 +115,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   if (warp == 4) {
     if (lane == 0) {
       // ---------------------------------------------------- loads + MMAs
+      // B_s: one box per 32 columns, into the buffer the row warps build X from.
+      const uint64_t pol = policy_evict_first();
+      auto issue_b = [&](int s) {
+        mbar_expect_tx(&sh.b_full, kBBuf);
+#pragma unroll
+        for (int b = 0; b < N / 32; ++b)
+          tma_load_2d(bbuf + b * 16384, &p.mB, &sh.b_full, c0 + 32 * b, (int)(slot_of(s) * 128), pol);
+      };
       auto issue_load = [&](int s) {
         const int st = s & 1;
         const uint8_t* src = p.M + slot_of(s) * (size_t)kMBytes;
@@ -116,13 +130,22 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         bulk_load(mring + st * kMBytes, src, kMBytes / 2, &sh.m_full[st]);
         bulk_load(mring + st * kMBytes + kMBytes / 2, src + kMBytes / 2, kMBytes / 2, &sh.m_full[st]);
       };
+      // Steps further ahead are brought into L2 by the TMA engine, so that the
+      // row warps' B_t loads and the M_t copies hit L2 (one CTA of the pair).
+      auto prefetch = [&](int s) {
+        if (blockIdx.x != 0 || s > T) return;
+        bulk_prefetch_l2(p.M + slot_of(s) * (size_t)kMBytes, kMBytes);
+        bulk_prefetch_l2(p.Bm + slot_of(s) * 128 * 128, 128 * 128 * 4);
+      };
       int issued = 0;
+      issue_b(0);
       issue_load(0);
       ++issued;
       if (T >= 1) {
         issue_load(1);
         ++issued;
       }
+      for (int s = 1; s < kAhead; ++s) prefetch(s);
       const uint32_t maddr = smem_u32(mring);
       const uint32_t xaddr = smem_u32(xbuf);
       for (int s = 0; s <= T; ++s) {
@@ -132,6 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
           break;
         }
         tc_fence_after();
+        if (s + 1 <= T) issue_b(s + 1);        // X_s is built: the B buffer is free
+        prefetch(s + kAhead);
         const uint32_t ma = maddr + st * kMBytes;
 #pragma unroll
         for (int pass = 0; pass < 3; ++pass) {
@@ -166,31 +191,46 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     // ---------------------------------------------------- rows of S (warps 0..3)
     const int m = warp * 32 + lane;          // row of S = TMEM lane
     const float inv_lam = 1.f / p.lam;
-    float srow[N], brow[N];
+    float srow[N];
 #pragma unroll
     for (int j = 0; j < N; ++j) srow[j] = 0.f;
-    // B_t row m of the first step; each later row is fetched while the
-    // previous step's MMAs run.
-    auto fetch_b = [&](int s) {
-      const float4* src = reinterpret_cast<const float4*>(p.Bm + (slot_of(s) * 128 + m) * 128 + c0);
+    // S_t row m -> swizzled staging (32-column boxes, double-buffered) -> TMA
+    // store.  Runs while the next step's MMAs do: S_{t+1} needs only srow.
+    auto store_state = [&](int s) {
+      const int t = dir == 0 ? s : T + 1 - s;
+      uint8_t* stg = sstage;
+      if (warp == 0 && lane == 0) bulk_wait_read<0>();   // the previous store has read the buffer
+      named_bar_sync(kEpiBar, 128);
 #pragma unroll
-      for (int q = 0; q < N / 4; ++q) {
-        const float4 v = __ldg(src + q);
-        brow[4 * q] = v.x;
-        brow[4 * q + 1] = v.y;
-        brow[4 * q + 2] = v.z;
-        brow[4 * q + 3] = v.w;
+      for (int q = 0; q < N / 4; ++q)
+        *reinterpret_cast<float4*>(stg + (q / 8) * 16384 + sw128(m, q % 8)) =
+            make_float4(srow[4 * q], srow[4 * q + 1], srow[4 * q + 2], srow[4 * q + 3]);
+      fence_proxy_async_smem();
+      named_bar_sync(kEpiBar, 128);
+      if (warp == 0 && lane == 0) {
+        const CUtensorMap* map = dir == 0 ? &p.mSF : &p.mSB;
+        const int y = ((bh * T) + (t - 1)) * 128;
+#pragma unroll
+        for (int b = 0; b < N / 32; ++b) tma_store_2d(map, stg + b * 16384, c0 + 32 * b, y);
+        bulk_commit();
       }
     };
-    fetch_b(0);
+    // The loop never breaks: after a timeout the waits are skipped, so the
+    // four warps always meet at the named barriers the same number of times.
     for (int s = 0; s <= T; ++s) {
-      // X row m = S row m + B_t row m / lambda, split into hi / lo, MN-major swizzled.
+      // X row m = S_{s-1} row m + B_s row m / lambda, split into hi / lo, MN-major swizzled.
+      const bool okb = !aborted(sh) && mbar_wait(&sh.b_full, s & 1);
+      if (!okb && !aborted(sh)) set_abort(sh, p.err);
 #pragma unroll
       for (int q = 0; q < N / 8; ++q) {
         float h[8], l[8];
+        const uint32_t boff = (q / 4) * 16384u + sw128(m, (2 * q) % 8);
+        const float4 b0 = *reinterpret_cast<const float4*>(bbuf + boff);
+        const float4 b1 = *reinterpret_cast<const float4*>(bbuf + (q / 4) * 16384u + sw128(m, (2 * q + 1) % 8));
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float x = fmaf(brow[8 * q + i], inv_lam, srow[8 * q + i]);
+          const float x = fmaf(bv[i], inv_lam, srow[8 * q + i]);
           h[i] = __bfloat162float(__float2bfloat16_rn(x));
           l[i] = x - h[i];
         }
@@ -203,13 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sh.x_full);
-      if (s + 1 <= T) fetch_b(s + 1);
-      if (__any_sync(0xffffffffu, aborted(sh))) break;
-      const bool ok = mbar_wait(&sh.d_full, s & 1);
-      if (!__all_sync(0xffffffffu, ok)) {
-        set_abort(sh, p.err);
-        break;
-      }
+      if (s >= 2) store_state(s - 1);          // S_{s-1}, still in srow
+      const bool ok = !aborted(sh) && mbar_wait(&sh.d_full, s & 1);
+      if (!ok && !aborted(sh)) set_abort(sh, p.err);
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
 #pragma unroll
@@ -220,27 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
 #pragma unroll
         for (int j = 0; j < 32; ++j) srow[c * 32 + j] = __uint_as_float(r[j]);
       }
-      if (s > 0) {
-        // S_t row m -> swizzled staging (32-column boxes) -> TMA store.
-        const int t = dir == 0 ? s : T + 1 - s;
-        uint8_t* stg = sstage + (s & 1) * kSStage;
-        if (warp == 0 && lane == 0) bulk_wait_read<1>();   // the store two steps back has read this buffer
-        named_bar_sync(kEpiBar, 128);
-#pragma unroll
-        for (int q = 0; q < N / 4; ++q)
-          *reinterpret_cast<float4*>(stg + (q / 8) * 16384 + sw128(m, q % 8)) =
-              make_float4(srow[4 * q], srow[4 * q + 1], srow[4 * q + 2], srow[4 * q + 3]);
-        fence_proxy_async_smem();
-        named_bar_sync(kEpiBar, 128);
-        if (warp == 0 && lane == 0) {
-          const CUtensorMap* map = dir == 0 ? &p.mSF : &p.mSB;
-          const int y = ((bh * T) + (t - 1)) * 128;
-#pragma unroll
-          for (int b = 0; b < N / 32; ++b) tma_store_2d(map, stg + b * 16384, c0 + 32 * b, y);
-          bulk_commit();
-        }
-      }
     }
+    if (T >= 1) store_state(T);
     if (warp == 0 && lane == 0) bulk_wait<0>();   // S stores complete before exit
   }
 
@@ -257,7 +274,9 @@ cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm
   ScanTcParams prm;
   memset(&prm, 0, sizeof(prm));
   const long long rows = (long long)p.B * p.H * p.T * 128;
-  if (!make_f32_rows_map(&prm.mSF, SF, rows, 128) || !make_f32_rows_map(&prm.mSB, SB, rows, 128))
+  const long long brows = (long long)p.B * p.H * (p.T + 1) * 128;
+  if (!make_f32_rows_map(&prm.mSF, SF, rows, 128) || !make_f32_rows_map(&prm.mSB, SB, rows, 128) ||
+      !make_f32_rows_map(&prm.mB, Bm, brows, 128))
     return cudaErrorInvalidValue;
   prm.M = reinterpret_cast<const uint8_t*>(M);
   prm.Bm = Bm;
@@ -266,7 +285,7 @@ cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm
   prm.err = err;
   prm.T = p.T;
   prm.lam = p.lambda;
-  const size_t smem = 1024 + 2 * kMBytes + 2 * kXHalf + 2 * kSStage + sizeof(Shared);
+  const size_t smem = 1024 + 2 * kMBytes + 2 * kXHalf + kSStage + kBBuf + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(kSplit, 2, p.B * p.H);
