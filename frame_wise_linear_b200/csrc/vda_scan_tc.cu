@@ -15,13 +15,14 @@
 // per-step error does not grow along the chain.
 //
 // The recurrence is independent per column of S, so each chain is split over
-// kSplit CTAs of N = 128 / kSplit columns.  CTA layout (160 threads):
-//   warps 0..3  own TMEM lanes = rows of S: build X (row m) in shared memory,
-//               stage the previous state (double-buffered, swizzled) for a
-//               TMA store while the step's MMAs run, then read S_t back from
-//               TMEM;
-//   warp 4      one thread: bulk-copies M_t (64 KB) into a 2-stage ring ahead
-//               of time and issues the 24 MMAs of each step.
+// kSplit CTAs of N = 128 / kSplit columns.  CTA layout (288 threads):
+//   warps 0..7  own TMEM lanes = rows of S (two warps per lane quarter, 32
+//               columns each): build X (row m) in shared memory from S_{t-1}
+//               and B_t, stage the previous state (swizzled) for a TMA store
+//               while the step's MMAs run, then read S_t back from TMEM;
+//   warp 8      one thread: bulk-copies M_t (64 KB) into a 2-stage ring and
+//               B_t (this CTA's columns) by TMA, ahead of time, and issues
+//               the 24 MMAs of each step.
 // Every wait is bounded; a timeout sets the error bit and the CTA winds down.
 #include "sm100.cuh"
 #include "vda_internal.cuh"
@@ -33,12 +34,16 @@ using namespace sm100;
 
 constexpr int kSplit = 2;
 constexpr int N = 128 / kSplit;              // columns of S per CTA
-constexpr int kThreads = 160;
+constexpr int kRowWarps = 8;                 // two per TMEM lane quarter
+constexpr int kMmaWarp = kRowWarps;
+constexpr int kCols = N / 2;                 // columns of S per row thread
+constexpr int kThreads = 32 * (kRowWarps + 1);
+static_assert(N == 64 && kCols == 32, "row warps hold one 32-column TMEM load and one 128-byte X row");
 constexpr int kMBytes = 65536;               // M_t hi | lo
 constexpr int kXHalf = (N / 64) * 16384;     // X hi (or lo): N/64 blocks of 128 rows x 128 B
 constexpr int kSStage = N * 128 * 4;         // S_t staging: N/32 boxes of 128 rows x 128 B
 constexpr int kBBuf = N * 128 * 4;           // B_t columns of this CTA, same layout
-constexpr int kEpiBar = 1;                   // named barrier of the 4 row warps
+constexpr int kEpiBar = 1;                   // named barrier of the row warps
 constexpr int kAhead = 4;                    // steps of M_t and B_t prefetched into L2
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, N, /*a MN*/ false, /*b MN*/ true);
 
@@ -96,14 +101,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       mbar_init(&sh.m_full[i], 1);
       mbar_init(&sh.m_empty[i], 1);
     }
-    mbar_init(&sh.x_full, 128);
+    mbar_init(&sh.x_full, 32 * kRowWarps);
     mbar_init(&sh.d_full, 1);
     mbar_init(&sh.b_full, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&sh.tmem_base, N);
     tmem_relinquish();
   }
@@ -112,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     if (lane == 0) {
       // ---------------------------------------------------- loads + MMAs
       // B_s: one box per 32 columns, into the buffer the row warps build X from.
@@ -188,45 +193,45 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       mbar_wait(&sh.drain, 0);
     }
   } else {
-    // ---------------------------------------------------- rows of S (warps 0..3)
-    const int m = warp * 32 + lane;          // row of S = TMEM lane
+    // ---------------------------------------------------- rows of S (warps 0..7)
+    const int m = (warp % 4) * 32 + lane;    // row of S = TMEM lane (warp % 4 = lane quarter)
+    const int hc = warp / 4;                 // columns kCols * hc .. + kCols - 1 of this CTA's N
     const float inv_lam = 1.f / p.lam;
-    float srow[N];
+    float srow[kCols];
 #pragma unroll
-    for (int j = 0; j < N; ++j) srow[j] = 0.f;
-    // S_t row m -> swizzled staging (32-column boxes, double-buffered) -> TMA
-    // store.  Runs while the next step's MMAs do: S_{t+1} needs only srow.
+    for (int j = 0; j < kCols; ++j) srow[j] = 0.f;
+    // S_t row m -> swizzled staging (32-column boxes) -> TMA store.  Runs
+    // while the next step's MMAs do: S_{t+1} needs only srow.
     auto store_state = [&](int s) {
       const int t = dir == 0 ? s : T + 1 - s;
-      uint8_t* stg = sstage;
       if (warp == 0 && lane == 0) bulk_wait_read<0>();   // the previous store has read the buffer
-      named_bar_sync(kEpiBar, 128);
+      named_bar_sync(kEpiBar, 32 * kRowWarps);
 #pragma unroll
-      for (int q = 0; q < N / 4; ++q)
-        *reinterpret_cast<float4*>(stg + (q / 8) * 16384 + sw128(m, q % 8)) =
+      for (int q = 0; q < kCols / 4; ++q)
+        *reinterpret_cast<float4*>(sstage + hc * 16384 + sw128(m, q)) =
             make_float4(srow[4 * q], srow[4 * q + 1], srow[4 * q + 2], srow[4 * q + 3]);
       fence_proxy_async_smem();
-      named_bar_sync(kEpiBar, 128);
+      named_bar_sync(kEpiBar, 32 * kRowWarps);
       if (warp == 0 && lane == 0) {
         const CUtensorMap* map = dir == 0 ? &p.mSF : &p.mSB;
         const int y = ((bh * T) + (t - 1)) * 128;
 #pragma unroll
-        for (int b = 0; b < N / 32; ++b) tma_store_2d(map, stg + b * 16384, c0 + 32 * b, y);
+        for (int b = 0; b < N / 32; ++b) tma_store_2d(map, sstage + b * 16384, c0 + 32 * b, y);
         bulk_commit();
       }
     };
     // The loop never breaks: after a timeout the waits are skipped, so the
-    // four warps always meet at the named barriers the same number of times.
+    // row warps always meet at the named barrier the same number of times.
     for (int s = 0; s <= T; ++s) {
       // X row m = S_{s-1} row m + B_s row m / lambda, split into hi / lo, MN-major swizzled.
       const bool okb = !aborted(sh) && mbar_wait(&sh.b_full, s & 1);
       if (!okb && !aborted(sh)) set_abort(sh, p.err);
 #pragma unroll
-      for (int q = 0; q < N / 8; ++q) {
+      for (int q = 0; q < kCols / 8; ++q) {
         float h[8], l[8];
-        const uint32_t boff = (q / 4) * 16384u + sw128(m, (2 * q) % 8);
-        const float4 b0 = *reinterpret_cast<const float4*>(bbuf + boff);
-        const float4 b1 = *reinterpret_cast<const float4*>(bbuf + (q / 4) * 16384u + sw128(m, (2 * q + 1) % 8));
+        // B box hc (32 columns); this chunk of 8 columns is 16-byte chunks 2q, 2q + 1.
+        const float4 b0 = *reinterpret_cast<const float4*>(bbuf + hc * 16384 + sw128(m, 2 * q));
+        const float4 b1 = *reinterpret_cast<const float4*>(bbuf + hc * 16384 + sw128(m, 2 * q + 1));
         const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -234,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
           h[i] = __bfloat162float(__float2bfloat16_rn(x));
           l[i] = x - h[i];
         }
-        const uint32_t off = (q / 8) * 16384u + sw128(m, q % 8);
+        const uint32_t off = sw128(m, (kCols / 8) * hc + q);   // N = 64: one 128-byte row per k
         *reinterpret_cast<uint4*>(xbuf + off) =
             make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(h[4], h[5]), pack_bf16(h[6], h[7]));
         *reinterpret_cast<uint4*>(xbuf + kXHalf + off) =
@@ -247,14 +252,12 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       const bool ok = !aborted(sh) && mbar_wait(&sh.d_full, s & 1);
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-      for (int c = 0; c < N / 32; ++c) {
+      {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)((warp % 4) * 32) << 16) + kCols * hc, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) srow[c * 32 + j] = __uint_as_float(r[j]);
+        for (int j = 0; j < kCols; ++j) srow[j] = __uint_as_float(r[j]);
       }
     }
     if (T >= 1) store_state(T);
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, N);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, N);
 }
 
 }  // namespace
