@@ -39,12 +39,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # FP32 SIMT peak from unit counts and clock: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz.
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
-# Kernel of each stage and the source file that defines it (for ncu traffic lookups).
+# Kernel of each reported stage and the source file that defines it (for ncu
+# traffic lookups), by input dtype.  With bf16 inputs the Gram and the factor
+# are one kernel.
 STAGE_SOURCES = {
-    "gram": "frame_wise_linear_b200/csrc/vda_gram_tc.cu",
-    "factor": "frame_wise_linear_b200/csrc/vda_factor_tc.cu",
-    "scan": "frame_wise_linear_b200/csrc/vda_scan_tc.cu",
-    "readout": "frame_wise_linear_b200/csrc/vda_readout_tc.cu",
+    1: {"gram+factor": "frame_wise_linear_b200/csrc/vda_gramfactor_tc.cu",
+        "scan": "frame_wise_linear_b200/csrc/vda_scan_tc.cu",
+        "readout": "frame_wise_linear_b200/csrc/vda_readout_tc.cu"},
+    0: {"gram": "frame_wise_linear_b200/csrc/vda_simt.cu",
+        "factor": "frame_wise_linear_b200/csrc/vda_factor.cu",
+        "scan": "frame_wise_linear_b200/csrc/vda_simt.cu",
+        "readout": "frame_wise_linear_b200/csrc/vda_simt.cu"},
 }
 
 
@@ -80,10 +85,13 @@ def stage_work(w):
     frames = bh * w.T
     slots = bh * (w.T + 1)
     d_k, d_v = w.d_k, w.d_v
+    gram = dict(bound="hbm", bytes=(frames * w.n + bh * w.n_txt) * (d_k + d_v) * es,
+                flops=2.0 * (frames * w.n + bh * w.n_txt) * d_k * (d_k + d_v))
     return {
         # reads K_t, V_t of every frame and the text once
-        "gram": dict(bound="hbm", bytes=(frames * w.n + bh * w.n_txt) * (d_k + d_v) * es,
-                     flops=2.0 * (frames * w.n + bh * w.n_txt) * d_k * (d_k + d_v)),
+        "gram": gram,
+        # the same, with the factor in the same kernel (no algorithmic bytes of its own)
+        "gram+factor": dict(bound="hbm", bytes=gram["bytes"], flops=gram["flops"] + slots * float(d_k) ** 3),
         # lambda A^{-1} by the symmetric sweep: d^3/2 FMA = d^3 flops per slot
         "factor": dict(bound="alu", bytes=0, flops=slots * float(d_k) ** 3),
         # two directions, one d_k x d_k by d_k x d_v product per frame
@@ -107,12 +115,12 @@ def path_roofline(w, peaks):
                 bound="hbm" if t_hbm >= t_tc else "tensor")
 
 
-def traffic_lookup(stage):
+def traffic_lookup(stage, dtype=1):
     """DRAM bytes per launch from a committed ncu summary, if the kernel's source is unchanged."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or stage not in STAGE_SOURCES[dtype]:
         return None
-    src = os.path.join(ROOT, STAGE_SOURCES[stage])
+    src = os.path.join(ROOT, STAGE_SOURCES[dtype][stage])
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     with open(path) as fh:
         for line in fh:
@@ -347,6 +355,9 @@ def run_b200(args, w):
     vda.vda_sync_status(wsp, stream=stream)
     ms = start.elapsed_time(end)
     stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i, s in enumerate(vda.STAGES)}
+    if w.dtype == 1:   # one kernel for the Gram and the factor: report them as one stage
+        stage_ms = {"gram+factor": stage_ms["gram"] + stage_ms["factor"], "scan": stage_ms["scan"],
+                    "readout": stage_ms["readout"]}
     if pg:
         t = torch.tensor([ms], device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
@@ -366,7 +377,7 @@ def run_b200(args, w):
         roof = {"kernel": dom, "bound": "alu", "achieved": wk["flops"] / t_s / 1e12, "peak": FP32_SIMT_TFLOPS,
                 "unit": "TFLOP/s", "peak_source": "derived: 148 SMs x 128 FP32 FMA/clk x 2 x 1.965 GHz"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    tr = traffic_lookup(dom)
+    tr = traffic_lookup(dom, w.dtype)
     roof["traffic"] = tr
     pr = path_roofline(w, peaks)
     path = {"t_roof_us": pr["t_roof_s"] * 1e6, "bound": pr["bound"], "bytes": pr["bytes"],
@@ -413,7 +424,7 @@ def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == 1 else "f32", "data": "synthetic",
         "config": config_of(w, ws_n), "roofline": roof, "roofline_path": path, "e2e": e2e,
-        "clocks": clocks, "gpu_launches": len(vda.STAGES) * args.steps,
+        "clocks": clocks, "gpu_launches": vda.LAUNCHES_PER_FORWARD[w.dtype] * args.steps,
     }
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         v, units, desc = cpu_oracle_sample(w, args.cpu_seconds)

@@ -116,15 +116,16 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
   if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "event record");
   constexpr bool kBf16 = std::is_same<TIn, __nv_bfloat16>::value;
   if constexpr (kBf16) {
-    if ((e = vda::launch_gram_tc(p, k, v, kt, vt, M, C, err, st)) != cudaSuccess) return cuda_fail(e, "gram launch");
+    // Gram and factor in one kernel: M_t and B_t, A_t never leaves TMEM.  The
+    // factor interval between events 1 and 2 is empty on this path.
+    if ((e = vda::launch_gramfactor_tc(p, k, v, kt, vt, M, C, err, st)) != cudaSuccess)
+      return cuda_fail(e, "gram+factor launch");
   } else {
     if ((e = vda::launch_gram_simt<TIn>(p, k, v, kt, vt, M, C, st)) != cudaSuccess)
       return cuda_fail(e, "gram launch");
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
-  if constexpr (kBf16) {
-    if ((e = vda::launch_factor_tc(p, M, err, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
-  } else {
+  if constexpr (!kBf16) {
     if ((e = vda::launch_factor(p, M, err, false, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
   }
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");

@@ -1,0 +1,506 @@
+// Gram / cross products and the factor step in one kernel, on tcgen05 tensor
+// cores (bf16 inputs, d = 128).
+//
+// For every slot (b, h, t) -- t = 0 is the text, t = 1..T the frames -- this
+// computes, after "VDN-MiniMax-H3" (aiezz.com), section 03, Video Delta
+// Attention item (each frame's state comes from a joint solve of the normal
+// equations over all of its tokens):
+//     A_t = K_t^T K_t + lambda I,    B_t = K_t^T V_t          (float32)
+//     M_t = lambda A_t^{-1}                                   (written as bf16 hi + lo)
+// The scan then runs S_t = M_t (S_{t-1} + B_t / lambda).
+//
+// Gram: one MMA chain D = K_t^T [K_t | V_t] (M = 128 features of K, N = 256,
+// K-dim = tokens) into a 256-column TMEM buffer, double-buffered.
+// Factor: A_t stays where the chain left it, in TMEM (lane i = row i), and is
+// swept there: the sweep operator taken 8 pivots at a time in its Cholesky
+// form.  For a pivot block K with P = A_KK = L L^T and X = A[:, K],
+//     X~ = X with X~_K = P - I,   Y = X~ L^{-T},   A <- A - Y Y^T,
+// leaves the swept block row and column in place; the -2 on the swept
+// diagonal commutes with later blocks and is applied once at the end:
+// -A^{-1} = A_final - 2I, so M = lambda (2I - A_final).  Each thread forms its
+// row of Y; the rank-8 update is three kind::tf32 MMAs (Y hi/lo products above
+// float32 rounding, A negated).  A never goes through HBM.
+//
+// Design (persistent, one CTA per SM, 10 warps), slots round-robin over CTAs:
+//   warp 0      TMA producer: 64-token chunks of K_t and V_t, each as two
+//               64-feature boxes with the 128-byte swizzle, 5-stage ring.
+//   warp 1      allocates TMEM (2 x 256 columns) and issues the Gram MMAs
+//               from one thread (both operands MN-major in shared memory).
+//   warps 2..5  B epilogue: TMEM -> registers -> 32-column swizzled chunks ->
+//               TMA stores of B_t.
+//   warps 6..9  factor group (one thread per row of A): lambda on the
+//               diagonal, the 16 block steps (its first thread issues the
+//               update MMAs), then M_t as bf16 hi/lo in the scan's operand
+//               layout.  The next slot's Gram runs meanwhile into the other
+//               TMEM buffer.
+// A buffer is reused once both the B epilogue and the factor group release
+// it.  A non-positive or non-finite pivot sets the NOT_SPD bit; every wait is
+// bounded, and a wait that runs out sets the timeout bit and winds the CTA
+// down (waiting, bounded, for its own copies and MMAs).
+#include "sm100.cuh"
+#include "vda_internal.cuh"
+
+namespace vda {
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 5;
+constexpr int kChunk = 64;                    // tokens per stage
+constexpr int kBox = 64 * 64 * 2;             // one 64 x 64 bf16 box: 8 KB
+constexpr int kStageBytes = 4 * kBox;         // K lo/hi features, V lo/hi features
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;           // two 256-column [A | B] buffers
+constexpr int kOutChunk = 128 * 32 * 4;       // B staging: 32 float32 columns x 128 rows
+constexpr int kEpiBar = 1;                    // named barrier of the B epilogue warps
+constexpr int kFacBar = 2;                    // named barrier of the factor group
+constexpr int kOp = 128 * 8 * 4;              // factor operand: 128 rows x 8 tf32 (4 KB)
+constexpr uint32_t kIdescGram = idesc_bf16_f32(128, 256, /*a MN*/ true, /*b MN*/ true);
+constexpr uint32_t kIdescUpd = idesc_tf32_f32(128, 128, /*negate A*/ true);
+
+struct GramFactorParams {
+  CUtensorMap mK, mV, mKt, mVt;
+  CUtensorMap mB;       // [slots * 128][128] float32, 32 x 128 boxes
+  uint8_t* M;           // per slot 64 KB: M hi | M lo
+  unsigned* err;
+  int BH, T, n, n_txt;
+  float lam;
+};
+
+struct Shared {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t upd;         // factor: one phase per block step
+  uint64_t fdone;       // factor: one phase per slot, all its MMAs complete
+  uint64_t drain;
+  uint32_t tmem_base;
+  int bad;
+  int abort;
+};
+
+__device__ __forceinline__ bool aborted(Shared& sh) { return *reinterpret_cast<volatile int*>(&sh.abort) != 0; }
+__device__ __forceinline__ void set_abort(Shared& sh, unsigned* err) {
+  atomicOr(err, kDevErrTimeout);
+  *reinterpret_cast<volatile int*>(&sh.abort) = 1;
+}
+
+__device__ __forceinline__ void slot_info(const GramFactorParams& p, int s, int& rows, int& z, bool& text) {
+  const int bh = s / (p.T + 1);
+  const int t = s % (p.T + 1);
+  text = (t == 0);
+  rows = text ? p.n_txt : p.n;
+  z = text ? bh : bh * p.T + (t - 1);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Row i, K-chunk c (4 tf32 values) of a K-major, non-swizzled operand: 8-row
+// core matrices of 128 bytes (SBO = 128), the two K-chunks 2 KB apart (LBO).
+__device__ __forceinline__ void store_op(uint8_t* op, int i, const float (&v)[8]) {
+  *reinterpret_cast<float4*>(op + i * 16) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(op + 2048 + i * 16) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid_constant__ GramFactorParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = base;
+  uint8_t* ostage = base + kStages * kStageBytes;   // 2 x B staging chunk
+  uint8_t* ops = ostage + 2 * kOutChunk;            // factor: Y hi | Y lo
+  float (*psm)[8] = reinterpret_cast<float (*)[8]>(ops + 2 * kOp);   // factor: the pivot block
+  Shared& sh = *reinterpret_cast<Shared*>(ops + 2 * kOp + 8 * 8 * 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int slots = p.BH * (p.T + 1);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.tfull[i], 1);
+      mbar_init(&sh.tempty[i], 256);   // 128 B-epilogue threads + 128 factor threads
+    }
+    mbar_init(&sh.upd, 1);
+    mbar_init(&sh.fdone, 1);
+    mbar_init(&sh.drain, 1);
+    sh.bad = 0;
+    sh.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.mK);
+    tma_prefetch_desc(&p.mV);
+    tma_prefetch_desc(&p.mB);
+    if (p.n_txt > 0) {
+      tma_prefetch_desc(&p.mKt);
+      tma_prefetch_desc(&p.mVt);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int s = blockIdx.x; s < slots && !aborted(sh); s += gridDim.x) {
+        int rows, z;
+        bool text;
+        slot_info(p, s, rows, z, text);
+        const CUtensorMap* mk = text ? &p.mKt : &p.mK;
+        const CUtensorMap* mv = text ? &p.mVt : &p.mV;
+        for (int r0 = 0; r0 < rows; r0 += kChunk) {
+          if (!mbar_wait(&sh.empty[stage], phase ^ 1)) {
+            set_abort(sh, p.err);
+            break;
+          }
+          uint8_t* st = stages + stage * kStageBytes;
+          mbar_expect_tx(&sh.full[stage], kStageBytes);
+          tma_load_3d(st + 0 * kBox, mk, &sh.full[stage], 0, r0, z, pol);
+          tma_load_3d(st + 1 * kBox, mk, &sh.full[stage], 64, r0, z, pol);
+          tma_load_3d(st + 2 * kBox, mv, &sh.full[stage], 0, r0, z, pol);
+          tma_load_3d(st + 3 * kBox, mv, &sh.full[stage], 64, r0, z, pol);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (aborted(sh)) {
+        // Error path: the chunks that may still be in flight land first.
+        for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+          mbar_wait(&sh.full[c % kStages], (c / kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ Gram MMAs
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int tb = 0;
+      uint32_t tphase = 0;
+      const uint32_t sbase = smem_u32(stages);
+      for (int s = blockIdx.x; s < slots && !aborted(sh); s += gridDim.x) {
+        int rows, z;
+        bool text;
+        slot_info(p, s, rows, z, text);
+        if (!mbar_wait(&sh.tempty[tb], tphase ^ 1)) {
+          set_abort(sh, p.err);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + tb * 256;
+        bool first = true;
+        for (int r0 = 0; r0 < rows; r0 += kChunk) {
+          if (!mbar_wait(&sh.full[stage], phase)) {
+            set_abort(sh, p.err);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * kStageBytes;
+#pragma unroll
+          for (int k = 0; k < kChunk / 16; ++k) {
+            // 16 tokens = 16 rows of 128 bytes; MN blocks of 64 features 8 KB apart.
+            const uint64_t desc = smem_desc(sa + k * 16 * 128, kBox, 1024, kSwizzle128B);
+            mma_bf16_ss(d, desc, desc, kIdescGram, first ? 0u : 1u);
+            first = false;
+          }
+          mma_commit(&sh.empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (aborted(sh)) break;
+        mma_commit(&sh.tfull[tb]);   // with no tokens this only marks the buffer (A = lambda I, B = 0)
+        tb ^= 1;
+        if (tb == 0) tphase ^= 1;
+      }
+      // Make sure no MMA is still running before TMEM is released.
+      mma_commit(&sh.drain);
+      mbar_wait(&sh.drain, 0);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ B epilogue
+    // B row by row (lane = feature i) into swizzled 32-column staging chunks,
+    // each stored by one TMA store.
+    const int quarter = warp % 4;            // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;     // feature index i of D
+    const bool leader = (warp == 2 && lane == 0);
+    int tb = 0, nst = 0;
+    uint32_t tphase = 0;
+    for (int s = blockIdx.x; s < slots; s += gridDim.x) {
+      int rows, z;
+      bool text;
+      slot_info(p, s, rows, z, text);
+      const bool ok = !aborted(sh) && mbar_wait(&sh.tfull[tb], tphase);
+      if (!ok && !aborted(sh)) set_abort(sh, p.err);
+      if (named_bar_or(kEpiBar, 128, !ok)) break;   // one decision for the four warps
+      tc_fence_after();
+      const uint32_t taddr = tmem + tb * 256 + 128 + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int chunk = 0; chunk < 4; ++chunk) {
+        uint32_t r[32];
+        if (rows > 0) {
+          tmem_ld_32x32b_x32(taddr + chunk * 32, r);
+          tmem_ld_wait();
+        } else {  // no tokens: B = 0
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
+        }
+        uint8_t* stg = ostage + (nst & 1) * kOutChunk;
+        if (leader) bulk_wait_read<1>();      // the store two chunks back has read this buffer
+        named_bar_sync(kEpiBar, 128);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(stg + sw128(row, q)) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(kEpiBar, 128);
+        if (leader) {
+          tma_store_2d(&p.mB, stg, chunk * 32, s * 128);
+          bulk_commit();
+        }
+        ++nst;
+      }
+      tc_fence_before();
+      mbar_arrive(&sh.tempty[tb]);
+      tb ^= 1;
+      if (tb == 0) tphase ^= 1;
+    }
+    if (leader) bulk_wait<0>();               // B stores complete before exit
+  } else {
+    // ------------------------------------------------------------ factor group
+    const int i = (warp % 4) * 32 + lane;    // row of A = TMEM lane (warp % 4 = lane quarter)
+    const bool issuer = (warp == 6 && lane == 0);
+    const uint32_t opaddr = smem_u32(ops);
+    int tb = 0;
+    uint32_t tphase = 0;
+    int nslot = 0;                            // slots factored by this CTA
+    for (int s = blockIdx.x; s < slots; s += gridDim.x, ++nslot) {
+      int rows, z;
+      bool text;
+      slot_info(p, s, rows, z, text);
+      bool ok = !aborted(sh) && mbar_wait(&sh.tfull[tb], tphase);
+      if (!ok && !aborted(sh)) set_abort(sh, p.err);
+      if (named_bar_or(kFacBar, 128, !ok)) break;
+      tc_fence_after();
+      const uint32_t trow = tmem + tb * 256 + ((uint32_t)((warp % 4) * 32) << 16);
+      // lambda on the diagonal (A = lambda I when the slot has no tokens).
+      {
+        uint32_t r[32];
+        const int c0 = (i / 32) * 32;
+        if (rows > 0) {
+          tmem_ld_32x32b_x32(trow + c0, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
+          uint32_t zr[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) zr[j] = 0u;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (c * 32 != c0) tmem_st_32x32b_x32(trow + c * 32, zr);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j == i - c0) r[j] = __float_as_uint(__uint_as_float(r[j]) + p.lam);
+        tmem_st_32x32b_x32(trow + c0, r);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      named_bar_sync(kFacBar, 128);
+      tc_fence_after();
+
+      bool bad = false;
+      int steps_issued = 0;
+#pragma unroll 1
+      for (int K = 0; K < 16; ++K) {
+        if (K > 0) {
+          const bool okw = mbar_wait(&sh.upd, (K - 1) & 1);
+          if (!okw) set_abort(sh, p.err);
+          if (named_bar_or(kFacBar, 128, !okw)) break;   // the same for every thread
+          tc_fence_after();
+        }
+        float x[8];
+        {
+          uint32_t r[8];
+          tmem_ld_32x32b_x8(trow + 8 * K, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) x[j] = __uint_as_float(r[j]);
+        }
+        // ---- P = L L^T.  The 8 rows of the pivot block publish their pivot
+        // columns; every thread factors P itself, in registers (rsqrt, no
+        // divides; the same operations in the same order in every thread).
+        if ((i >> 3) == K) {
+          *reinterpret_cast<float4*>(&psm[i & 7][0]) = make_float4(x[0], x[1], x[2], x[3]);
+          *reinterpret_cast<float4*>(&psm[i & 7][4]) = make_float4(x[4], x[5], x[6], x[7]);
+        }
+        named_bar_sync(kFacBar, 128);
+        float l[8][8];     // lower triangle: P, then L
+        float dinv[8];     // 1 / L_jj
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+#pragma unroll
+          for (int c = 0; c <= r; ++c) l[r][c] = psm[r][c];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float piv = l[j][j];
+          bad |= !(piv > 0.f) || !isfinite(piv);
+          const float rs = rsqrtf(piv);
+          dinv[j] = rs;
+#pragma unroll
+          for (int r = j + 1; r < 8; ++r) l[r][j] *= rs;
+#pragma unroll
+          for (int r = j + 1; r < 8; ++r) {
+#pragma unroll
+            for (int c = j + 1; c <= r; ++c) l[r][c] = fmaf(-l[r][j], l[c][j], l[r][c]);
+          }
+        }
+        // ---- X~ (row i) and Y = X~ L^{-T}: forward substitution L y = x~.
+        if ((i >> 3) == K) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) x[j] -= (j == (i & 7)) ? 1.f : 0.f;   // static indices only
+        }
+        float y[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float acc = x[j];
+#pragma unroll
+          for (int m = 0; m < j; ++m) acc = fmaf(-l[j][m], y[m], acc);
+          y[j] = acc * dinv[j];
+        }
+        // ---- tf32 hi + lo operand (row i)
+        {
+          float yh[8], yl[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            yh[j] = to_tf32(y[j]);
+            yl[j] = to_tf32(y[j] - yh[j]);
+          }
+          store_op(ops + 0 * kOp, i, yh);
+          store_op(ops + 1 * kOp, i, yl);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(kFacBar, 128);
+        if (issuer) {
+          tc_fence_after();
+          // A -= Y Y^T: Y is the A operand (M x K) and, read K-major from the
+          // same rows, the B operand (K x N).  Three tf32 passes: hi hi, hi lo,
+          // lo hi; the lo lo product is below float32 rounding of the update.
+          const uint64_t yhi = smem_desc(opaddr + 0 * kOp, 2048, 128, kSwizzleNone);
+          const uint64_t ylo = smem_desc(opaddr + 1 * kOp, 2048, 128, kSwizzleNone);
+          const uint32_t d = tmem + tb * 256;
+          mma_tf32_ss(d, yhi, yhi, kIdescUpd, 1u);
+          mma_tf32_ss(d, yhi, ylo, kIdescUpd, 1u);
+          mma_tf32_ss(d, ylo, yhi, kIdescUpd, 1u);
+          mma_commit(&sh.upd);
+        }
+        ++steps_issued;
+      }
+      if (bad && i == 0) sh.bad = 1;   // every thread saw the same pivots
+      // One more commit covers every update MMA issued for this slot; wait for
+      // it (bounded), also on the error path, before TMEM is read or reused.
+      if (issuer) mma_commit(&sh.fdone);
+      ok = mbar_wait(&sh.fdone, nslot & 1) && steps_issued == 16;
+      if (!ok && !aborted(sh)) set_abort(sh, p.err);
+      if (named_bar_or(kFacBar, 128, !ok)) break;
+      tc_fence_after();
+      // M = lambda (2I - A), row i, as bf16 hi/lo (K-major, swizzled).
+      {
+        uint8_t* hi = p.M + (size_t)s * 65536;
+        uint8_t* lo = hi + 32768;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {       // 8 columns per 16-byte chunk
+            float h[8], l8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int col = c * 32 + q * 8 + e;
+              const float m = p.lam * ((col == i ? 2.f : 0.f) - __uint_as_float(r[q * 8 + e]));
+              h[e] = __bfloat162float(__float2bfloat16_rn(m));
+              l8[e] = m - h[e];
+            }
+            const int chunk = c * 4 + q;       // 0..15
+            const uint32_t off = (chunk / 8) * 16384u + sw128(i, chunk % 8);
+            *reinterpret_cast<uint4*>(hi + off) = make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]),
+                                                             pack_bf16(h[4], h[5]), pack_bf16(h[6], h[7]));
+            *reinterpret_cast<uint4*>(lo + off) = make_uint4(pack_bf16(l8[0], l8[1]), pack_bf16(l8[2], l8[3]),
+                                                             pack_bf16(l8[4], l8[5]), pack_bf16(l8[6], l8[7]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sh.tempty[tb]);
+      tb ^= 1;
+      if (tb == 0) tphase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0 && sh.bad) atomicOr(p.err, kDevErrNotSpd);
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                                 const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* M, float* Bm,
+                                 unsigned* err, cudaStream_t st) {
+  if (p.d_k != 128 || p.d_v != 128) return cudaErrorInvalidValue;
+  GramFactorParams prm;
+  memset(&prm, 0, sizeof(prm));
+  const int BH = p.B * p.H;
+  if (!make_bf16_rows_map(&prm.mK, K, p.n, BH * p.T, 64) || !make_bf16_rows_map(&prm.mV, V, p.n, BH * p.T, 64))
+    return cudaErrorInvalidValue;
+  if (p.n_txt > 0 && (!make_bf16_rows_map(&prm.mKt, Kt, p.n_txt, BH, 64) || !make_bf16_rows_map(&prm.mVt, Vt, p.n_txt, BH, 64)))
+    return cudaErrorInvalidValue;
+  const long long rows = (long long)BH * (p.T + 1) * 128;
+  if (!make_f32_rows_map(&prm.mB, Bm, rows, 128)) return cudaErrorInvalidValue;
+  prm.M = reinterpret_cast<uint8_t*>(M);
+  prm.err = err;
+  prm.BH = BH;
+  prm.T = p.T;
+  prm.n = p.n;
+  prm.n_txt = p.n_txt;
+  prm.lam = p.lambda;
+  const size_t smem = 1024 + kStages * kStageBytes + 2 * kOutChunk + 2 * kOp + 8 * 8 * 4 + sizeof(Shared);
+  cudaError_t e = cudaFuncSetAttribute(gramfactor_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int slots = BH * (p.T + 1);
+  const int grid = slots < sms ? slots : sms;
+  gramfactor_tc_kernel<<<grid, kThreads, smem, st>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace vda

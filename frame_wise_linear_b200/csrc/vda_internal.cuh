@@ -60,20 +60,17 @@ cudaError_t launch_readout_simt(const vda_problem& p, const TIn* Q, const TIn* G
 // (32 KB each, same 64 KB per slot).
 cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool split_bf16, cudaStream_t st);
 
-// Tensor-core factor step (vda_factor_tc.cu): bf16 path, d_k = 128; same
-// output as launch_factor with split_bf16.
-cudaError_t launch_factor_tc(const vda_problem& p, float* M, unsigned* err, cudaStream_t st);
-
 // Tensor-core scan (vda_scan_tc.cu): bf16 path, d_k = d_v = 128; M in the
 // split layout above, B_t float32 in the C region.
 cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
                            unsigned* err, cudaStream_t st);
 
-// Tensor-core Gram (vda_gram_tc.cu): bf16 inputs, d_k = d_v = 128.  Writes
-// the same A and B slots as launch_gram_simt.
-cudaError_t launch_gram_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                           const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* A, float* Bm,
-                           unsigned* err, cudaStream_t st);
+// Gram and factor in one kernel (vda_gramfactor_tc.cu): bf16 inputs,
+// d_k = d_v = 128.  Writes each slot's M_t (the bf16 hi/lo image described
+// under launch_factor) into M and B_t into Bm; A_t stays in TMEM.
+cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                                 const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* M, float* Bm,
+                                 unsigned* err, cudaStream_t st);
 
 // Tensor-core readout (vda_readout_tc.cu): bf16 Q, G, O, d_k = d_v = 128.
 cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,

@@ -174,7 +174,10 @@ def vda_forward_states(problem, Q, K, V, G, K_txt, V_txt, O, workspace, S_fwd, S
 
 
 VDA_TIMED_EVENTS = 5
-STAGES = ("gram", "factor", "scan", "readout")
+STAGES = ("gram", "factor", "scan", "readout")   # the intervals between the 5 events
+# Kernels one forward launches.  With bf16 inputs the Gram and the factor are
+# one kernel (the "factor" interval is then empty).
+LAUNCHES_PER_FORWARD = {VDA_DTYPE_F32: 4, VDA_DTYPE_BF16: 3}
 
 
 def vda_forward_timed(problem, Q, K, V, G, K_txt, V_txt, O, workspace, events, stream=None,

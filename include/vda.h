@@ -108,7 +108,9 @@ vda_status vda_forward_states(const vda_problem* p, const void* Q, const void* K
  * `n_events` cudaEvent_t handles (passed as void*), created by the caller;
  * events[0] is recorded before the first kernel and events[i] after stage i
  * (1 = Gram, 2 = factor-and-solve, 3 = scan, 4 = readout).  n_events must be
- * VDA_TIMED_EVENTS; elapsed time between events i-1 and i is stage i. */
+ * VDA_TIMED_EVENTS; elapsed time between events i-1 and i is stage i.  With
+ * bf16 inputs the Gram and the factor run as one kernel: stage 1 times both
+ * and events 1 and 2 are recorded back to back (stage 2 is empty). */
 #define VDA_TIMED_EVENTS 5
 vda_status vda_forward_timed(const vda_problem* p, const void* Q, const void* K, const void* V,
                              const void* G, const void* K_txt, const void* V_txt, void* O,
