@@ -26,15 +26,15 @@
 //               64-feature boxes with the 128-byte swizzle, 5-stage ring.
 //   warp 1      allocates TMEM (2 x 256 columns) and issues the Gram MMAs
 //               from one thread (both operands MN-major in shared memory).
-//   warps 2..5  B epilogue: TMEM -> registers -> 32-column swizzled chunks ->
-//               TMA stores of B_t.
-//   warps 6..9  factor group (one thread per row of A): lambda on the
-//               diagonal, the 16 block steps (its first thread issues the
-//               update MMAs), then M_t as bf16 hi/lo in the scan's operand
-//               layout.  The next slot's Gram runs meanwhile into the other
-//               TMEM buffer.
-// A buffer is reused once both the B epilogue and the factor group release
-// it.  A non-positive or non-finite pivot sets the NOT_SPD bit; every wait is
+//   warps 2..5  service warps, per slot: B_t out (TMEM -> 32-column swizzled
+//               chunks -> TMA stores), lambda onto A's diagonal in TMEM; then
+//               M_t of the slot the factor group has just swept, out of TMEM
+//               as bf16 hi/lo in the scan's operand layout, and the buffer
+//               back to the Gram.
+//   warps 6..9  factor group (one thread per row of A): the 16 block steps of
+//               the sweep; its first thread issues the update MMAs.  The next
+//               slot's Gram and service work run meanwhile, so the group goes
+//               from one slot's sweep straight to the next.  A non-positive or non-finite pivot sets the NOT_SPD bit; every wait is
 // bounded, and a wait that runs out sets the timeout bit and winds the CTA
 // down (waiting, bounded, for its own copies and MMAs).
 #include "sm100.cuh"
@@ -70,8 +70,10 @@ struct GramFactorParams {
 struct Shared {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[2];    // Gram chain of the buffer complete
+  uint64_t aready[2];   // B drained and lambda on the diagonal: the factor may start
+  uint64_t fin[2];      // the factor's sweep of the buffer complete: M may be written
+  uint64_t tempty[2];   // M written: the buffer may take the next Gram chain
   uint64_t upd;         // factor: one phase per block step
   uint64_t fdone;       // factor: one phase per slot, all its MMAs complete
   uint64_t drain;
@@ -126,7 +128,9 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.tfull[i], 1);
-      mbar_init(&sh.tempty[i], 256);   // 128 B-epilogue threads + 128 factor threads
+      mbar_init(&sh.aready[i], 128);
+      mbar_init(&sh.fin[i], 128);
+      mbar_init(&sh.tempty[i], 128);
     }
     mbar_init(&sh.upd, 1);
     mbar_init(&sh.fdone, 1);
@@ -239,32 +243,66 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
       mbar_wait(&sh.drain, 0);
     }
   } else if (warp < 6) {
-    // ------------------------------------------------------------ B epilogue
-    // B row by row (lane = feature i) into swizzled 32-column staging chunks,
-    // each stored by one TMA store.
+    // ------------------------------------------------------------ service warps
+    // Per slot, in order: B_t out (TMEM -> swizzled 32-column chunks -> TMA
+    // stores), lambda onto A's diagonal in TMEM, hand A to the factor group;
+    // then, once the factor group has swept the previous slot, M_t of that
+    // slot out of TMEM into global memory, and the buffer back to the Gram.
     const int quarter = warp % 4;            // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;     // feature index i of D
     const bool leader = (warp == 2 && lane == 0);
-    int tb = 0, nst = 0;
-    uint32_t tphase = 0;
-    for (int s = blockIdx.x; s < slots; s += gridDim.x) {
+    int nst = 0;
+    auto write_m = [&](int s, int tb) {     // M = lambda (2I - A_final), row `row`, bf16 hi/lo
+      const uint32_t trow = tmem + tb * 256 + ((uint32_t)(quarter * 32) << 16);
+      uint8_t* hi = p.M + (size_t)s * 65536;
+      uint8_t* lo = hi + 32768;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(trow + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {         // 8 columns per 16-byte chunk
+          float h[8], l8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int col = c * 32 + q * 8 + e;
+            const float m = p.lam * ((col == row ? 2.f : 0.f) - __uint_as_float(r[q * 8 + e]));
+            h[e] = __bfloat162float(__float2bfloat16_rn(m));
+            l8[e] = m - h[e];
+          }
+          const int chunk = c * 4 + q;         // 0..15
+          const uint32_t off = (chunk / 8) * 16384u + sw128(row, chunk % 8);
+          *reinterpret_cast<uint4*>(hi + off) = make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]),
+                                                           pack_bf16(h[4], h[5]), pack_bf16(h[6], h[7]));
+          *reinterpret_cast<uint4*>(lo + off) = make_uint4(pack_bf16(l8[0], l8[1]), pack_bf16(l8[2], l8[3]),
+                                                           pack_bf16(l8[4], l8[5]), pack_bf16(l8[6], l8[7]));
+        }
+      }
+    };
+    int prev_s = -1, prev_tb = 0;
+    uint32_t fphase = 0;                      // phase of fin[] for the previous slot
+    int j = 0;
+    for (int s = blockIdx.x; s < slots; s += gridDim.x, ++j) {
+      const int tb = j & 1;
+      const uint32_t tphase = (j >> 1) & 1;
       int rows, z;
       bool text;
       slot_info(p, s, rows, z, text);
-      const bool ok = !aborted(sh) && mbar_wait(&sh.tfull[tb], tphase);
+      bool ok = !aborted(sh) && mbar_wait(&sh.tfull[tb], tphase);
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
       if (named_bar_or(kEpiBar, 128, !ok)) break;   // one decision for the four warps
       tc_fence_after();
-      const uint32_t taddr = tmem + tb * 256 + 128 + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t trow = tmem + tb * 256 + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int chunk = 0; chunk < 4; ++chunk) {
         uint32_t r[32];
         if (rows > 0) {
-          tmem_ld_32x32b_x32(taddr + chunk * 32, r);
+          tmem_ld_32x32b_x32(trow + 128 + chunk * 32, r);
           tmem_ld_wait();
         } else {  // no tokens: B = 0
 #pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = 0u;
+          for (int q = 0; q < 32; ++q) r[q] = 0u;
         }
         uint8_t* stg = ostage + (nst & 1) * kOutChunk;
         if (leader) bulk_wait_read<1>();      // the store two chunks back has read this buffer
@@ -280,10 +318,52 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         }
         ++nst;
       }
+      // lambda on the diagonal (A = lambda I when the slot has no tokens).
+      {
+        uint32_t r[32];
+        const int c0 = (row / 32) * 32;
+        if (rows > 0) {
+          tmem_ld_32x32b_x32(trow + c0, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) r[q] = 0u;
+          uint32_t zr[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) zr[q] = 0u;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (c * 32 != c0) tmem_st_32x32b_x32(trow + c * 32, zr);
+        }
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (q == row - c0) r[q] = __float_as_uint(__uint_as_float(r[q]) + p.lam);
+        tmem_st_32x32b_x32(trow + c0, r);
+        tmem_st_wait();
+      }
       tc_fence_before();
-      mbar_arrive(&sh.tempty[tb]);
-      tb ^= 1;
-      if (tb == 0) tphase ^= 1;
+      mbar_arrive(&sh.aready[tb]);
+      if (prev_s >= 0) {
+        // M of the previous slot, once the factor group has swept it.
+        ok = !aborted(sh) && mbar_wait(&sh.fin[prev_tb], fphase);
+        if (!ok && !aborted(sh)) set_abort(sh, p.err);
+        if (named_bar_or(kEpiBar, 128, !ok)) break;
+        fphase ^= (prev_tb == 1) ? 1u : 0u;
+        tc_fence_after();
+        write_m(prev_s, prev_tb);
+        tc_fence_before();
+        mbar_arrive(&sh.tempty[prev_tb]);
+      }
+      prev_s = s;
+      prev_tb = tb;
+    }
+    if (prev_s >= 0) {                        // the same for the four warps
+      const bool ok = !aborted(sh) && mbar_wait(&sh.fin[prev_tb], fphase);
+      if (!ok && !aborted(sh)) set_abort(sh, p.err);
+      if (!named_bar_or(kEpiBar, 128, !ok)) {
+        tc_fence_after();
+        write_m(prev_s, prev_tb);
+      }
     }
     if (leader) bulk_wait<0>();               // B stores complete before exit
   } else {
@@ -291,44 +371,14 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
     const int i = (warp % 4) * 32 + lane;    // row of A = TMEM lane (warp % 4 = lane quarter)
     const bool issuer = (warp == 6 && lane == 0);
     const uint32_t opaddr = smem_u32(ops);
-    int tb = 0;
-    uint32_t tphase = 0;
     int nslot = 0;                            // slots factored by this CTA
     for (int s = blockIdx.x; s < slots; s += gridDim.x, ++nslot) {
-      int rows, z;
-      bool text;
-      slot_info(p, s, rows, z, text);
-      bool ok = !aborted(sh) && mbar_wait(&sh.tfull[tb], tphase);
+      const int tb = nslot & 1;
+      bool ok = !aborted(sh) && mbar_wait(&sh.aready[tb], (nslot >> 1) & 1);
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
       if (named_bar_or(kFacBar, 128, !ok)) break;
       tc_fence_after();
       const uint32_t trow = tmem + tb * 256 + ((uint32_t)((warp % 4) * 32) << 16);
-      // lambda on the diagonal (A = lambda I when the slot has no tokens).
-      {
-        uint32_t r[32];
-        const int c0 = (i / 32) * 32;
-        if (rows > 0) {
-          tmem_ld_32x32b_x32(trow + c0, r);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = 0u;
-          uint32_t zr[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) zr[j] = 0u;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            if (c * 32 != c0) tmem_st_32x32b_x32(trow + c * 32, zr);
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j == i - c0) r[j] = __float_as_uint(__uint_as_float(r[j]) + p.lam);
-        tmem_st_32x32b_x32(trow + c0, r);
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      named_bar_sync(kFacBar, 128);
-      tc_fence_after();
 
       bool bad = false;
       int steps_issued = 0;
@@ -346,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           tmem_ld_32x32b_x8(trow + 8 * K, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) x[j] = __uint_as_float(r[j]);
+          for (int q = 0; q < 8; ++q) x[q] = __uint_as_float(r[q]);
         }
         // ---- P = L L^T.  The 8 rows of the pivot block publish their pivot
         // columns; every thread factors P itself, in registers (rsqrt, no
@@ -364,39 +414,39 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           for (int c = 0; c <= r; ++c) l[r][c] = psm[r][c];
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float piv = l[j][j];
+        for (int jj = 0; jj < 8; ++jj) {
+          const float piv = l[jj][jj];
           bad |= !(piv > 0.f) || !isfinite(piv);
           const float rs = rsqrtf(piv);
-          dinv[j] = rs;
+          dinv[jj] = rs;
 #pragma unroll
-          for (int r = j + 1; r < 8; ++r) l[r][j] *= rs;
+          for (int r = jj + 1; r < 8; ++r) l[r][jj] *= rs;
 #pragma unroll
-          for (int r = j + 1; r < 8; ++r) {
+          for (int r = jj + 1; r < 8; ++r) {
 #pragma unroll
-            for (int c = j + 1; c <= r; ++c) l[r][c] = fmaf(-l[r][j], l[c][j], l[r][c]);
+            for (int c = jj + 1; c <= r; ++c) l[r][c] = fmaf(-l[r][jj], l[c][jj], l[r][c]);
           }
         }
         // ---- X~ (row i) and Y = X~ L^{-T}: forward substitution L y = x~.
         if ((i >> 3) == K) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) x[j] -= (j == (i & 7)) ? 1.f : 0.f;   // static indices only
+          for (int q = 0; q < 8; ++q) x[q] -= (q == (i & 7)) ? 1.f : 0.f;   // static indices only
         }
         float y[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float acc = x[j];
+        for (int q = 0; q < 8; ++q) {
+          float acc = x[q];
 #pragma unroll
-          for (int m = 0; m < j; ++m) acc = fmaf(-l[j][m], y[m], acc);
-          y[j] = acc * dinv[j];
+          for (int m = 0; m < q; ++m) acc = fmaf(-l[q][m], y[m], acc);
+          y[q] = acc * dinv[q];
         }
         // ---- tf32 hi + lo operand (row i)
         {
           float yh[8], yl[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            yh[j] = to_tf32(y[j]);
-            yl[j] = to_tf32(y[j] - yh[j]);
+          for (int q = 0; q < 8; ++q) {
+            yh[q] = to_tf32(y[q]);
+            yl[q] = to_tf32(y[q] - yh[q]);
           }
           store_op(ops + 0 * kOp, i, yh);
           store_op(ops + 1 * kOp, i, yl);
@@ -421,44 +471,13 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
       }
       if (bad && i == 0) sh.bad = 1;   // every thread saw the same pivots
       // One more commit covers every update MMA issued for this slot; wait for
-      // it (bounded), also on the error path, before TMEM is read or reused.
+      // it (bounded), also on the error path, before the buffer is handed on.
       if (issuer) mma_commit(&sh.fdone);
       ok = mbar_wait(&sh.fdone, nslot & 1) && steps_issued == 16;
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
       if (named_bar_or(kFacBar, 128, !ok)) break;
-      tc_fence_after();
-      // M = lambda (2I - A), row i, as bf16 hi/lo (K-major, swizzled).
-      {
-        uint8_t* hi = p.M + (size_t)s * 65536;
-        uint8_t* lo = hi + 32768;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(trow + c * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {       // 8 columns per 16-byte chunk
-            float h[8], l8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int col = c * 32 + q * 8 + e;
-              const float m = p.lam * ((col == i ? 2.f : 0.f) - __uint_as_float(r[q * 8 + e]));
-              h[e] = __bfloat162float(__float2bfloat16_rn(m));
-              l8[e] = m - h[e];
-            }
-            const int chunk = c * 4 + q;       // 0..15
-            const uint32_t off = (chunk / 8) * 16384u + sw128(i, chunk % 8);
-            *reinterpret_cast<uint4*>(hi + off) = make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]),
-                                                             pack_bf16(h[4], h[5]), pack_bf16(h[6], h[7]));
-            *reinterpret_cast<uint4*>(lo + off) = make_uint4(pack_bf16(l8[0], l8[1]), pack_bf16(l8[2], l8[3]),
-                                                             pack_bf16(l8[4], l8[5]), pack_bf16(l8[6], l8[7]));
-          }
-        }
-      }
       tc_fence_before();
-      mbar_arrive(&sh.tempty[tb]);
-      tb ^= 1;
-      if (tb == 0) tphase ^= 1;
+      mbar_arrive(&sh.fin[tb]);
     }
   }
 
