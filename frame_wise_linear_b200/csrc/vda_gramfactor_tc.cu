@@ -9,8 +9,8 @@
 //     M_t = lambda A_t^{-1}                                   (written as bf16 hi + lo)
 // The scan then runs S_t = M_t (S_{t-1} + B_t / lambda).
 //
-// Gram: one MMA chain D = K_t^T [K_t | V_t] (M = 128 features of K, N = 256,
-// K-dim = tokens) into a 256-column TMEM buffer, double-buffered.
+// Gram: per 16 tokens, two MMAs into TMEM: A += K^T K and B += K^T V (M = 128
+// features of K, N = 128, K-dim = tokens).
 // Factor: A_t stays where the chain left it, in TMEM (lane i = row i), and is
 // swept there: the sweep operator taken 8 pivots at a time in its Cholesky
 // form.  For a pivot block K with P = A_KK = L L^T and X = A[:, K],
@@ -21,20 +21,25 @@
 // row of Y; the rank-8 update is three kind::tf32 MMAs (Y hi/lo products above
 // float32 rounding, A negated).  A never goes through HBM.
 //
-// Design (persistent, one CTA per SM, 10 warps), slots round-robin over CTAs:
+// TMEM (512 columns): three 128-column A regions used in turn by successive
+// slots, and one 128-column B region.
+//
+// Design (persistent, one CTA per SM, 14 warps), slots round-robin over CTAs:
 //   warp 0      TMA producer: 64-token chunks of K_t and V_t, each as two
 //               64-feature boxes with the 128-byte swizzle, 5-stage ring.
-//   warp 1      allocates TMEM (2 x 256 columns) and issues the Gram MMAs
-//               from one thread (both operands MN-major in shared memory).
+//   warp 1      allocates TMEM and issues the Gram MMAs from one thread (both
+//               operands MN-major in shared memory), once the slot's A region
+//               is free (M of its previous slot written) and B is drained.
 //   warps 2..5  service warps, per slot: B_t out (TMEM -> 32-column swizzled
-//               chunks -> TMA stores), lambda onto A's diagonal in TMEM; then
-//               M_t of the slot the factor group has just swept, out of TMEM
-//               as bf16 hi/lo in the scan's operand layout, and the buffer
-//               back to the Gram.
-//   warps 6..9  factor group (one thread per row of A): the 16 block steps of
-//               the sweep; its first thread issues the update MMAs.  The next
-//               slot's Gram and service work run meanwhile, so the group goes
-//               from one slot's sweep straight to the next.  A non-positive or non-finite pivot sets the NOT_SPD bit; every wait is
+//               chunks -> TMA stores), lambda onto A's diagonal in TMEM, A to
+//               the slot's factor group; then M of the previous slot, once
+//               its sweep is complete, out of TMEM as bf16 hi/lo in the
+//               scan's operand layout, and its A region back to the Gram.
+//   warps 6..13 two factor groups of four warps (one thread per row of A),
+//               sweeping alternate slots, so that one group's pivot-block
+//               work overlaps the other's update MMAs; the first thread of a
+//               group issues its update MMAs.
+// A non-positive or non-finite pivot sets the NOT_SPD bit; every wait is
 // bounded, and a wait that runs out sets the timeout bit and winds the CTA
 // down (waiting, bounded, for its own copies and MMAs).
 #include "sm100.cuh"
@@ -49,13 +54,16 @@ constexpr int kStages = 5;
 constexpr int kChunk = 64;                    // tokens per stage
 constexpr int kBox = 64 * 64 * 2;             // one 64 x 64 bf16 box: 8 KB
 constexpr int kStageBytes = 4 * kBox;         // K lo/hi features, V lo/hi features
-constexpr int kThreads = 320;
-constexpr uint32_t kTmemCols = 512;           // two 256-column [A | B] buffers
+constexpr int kFacGroups = 2;                 // factor groups, each sweeping its own slot
+constexpr int kThreads = 32 * (6 + 4 * kFacGroups);
+constexpr int kARegions = 3;                  // TMEM: three 128-column A regions, then B
+constexpr uint32_t kBCol = 128 * kARegions;
+constexpr uint32_t kTmemCols = 512;
 constexpr int kOutChunk = 128 * 32 * 4;       // B staging: 32 float32 columns x 128 rows
 constexpr int kEpiBar = 1;                    // named barrier of the B epilogue warps
-constexpr int kFacBar = 2;                    // named barrier of the factor group
+constexpr int kFacBar0 = 2;                   // named barriers of the factor groups: 2, 3
 constexpr int kOp = 128 * 8 * 4;              // factor operand: 128 rows x 8 tf32 (4 KB)
-constexpr uint32_t kIdescGram = idesc_bf16_f32(128, 256, /*a MN*/ true, /*b MN*/ true);
+constexpr uint32_t kIdescGram = idesc_bf16_f32(128, 128, /*a MN*/ true, /*b MN*/ true);
 constexpr uint32_t kIdescUpd = idesc_tf32_f32(128, 128, /*negate A*/ true);
 
 struct GramFactorParams {
@@ -70,12 +78,13 @@ struct GramFactorParams {
 struct Shared {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t tfull[2];    // Gram chain of the buffer complete
-  uint64_t aready[2];   // B drained and lambda on the diagonal: the factor may start
-  uint64_t fin[2];      // the factor's sweep of the buffer complete: M may be written
-  uint64_t tempty[2];   // M written: the buffer may take the next Gram chain
-  uint64_t upd;         // factor: one phase per block step
-  uint64_t fdone;       // factor: one phase per slot, all its MMAs complete
+  uint64_t gdone;               // one phase per slot: its Gram chain is complete
+  uint64_t bfree;               // one phase per slot: B drained, the B region is free
+  uint64_t tempty[kARegions];   // M written: the A region may take the next Gram chain
+  uint64_t aready[kFacGroups];  // per group, one phase per slot: lambda on A's diagonal
+  uint64_t fin[kFacGroups];     // per group, one phase per slot: sweep complete
+  uint64_t upd[kFacGroups];     // per group, one phase per block step
+  uint64_t fdone[kFacGroups];   // per group, one phase per slot: all its MMAs complete
   uint64_t drain;
   uint32_t tmem_base;
   int bad;
@@ -113,9 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
   uint8_t* ostage = base + kStages * kStageBytes;   // 2 x B staging chunk
-  uint8_t* ops = ostage + 2 * kOutChunk;            // factor: Y hi | Y lo
-  float (*psm)[8] = reinterpret_cast<float (*)[8]>(ops + 2 * kOp);   // factor: the pivot block
-  Shared& sh = *reinterpret_cast<Shared*>(ops + 2 * kOp + 8 * 8 * 4);
+  uint8_t* ops0 = ostage + 2 * kOutChunk;           // per factor group: Y hi | Y lo
+  float* psm0 = reinterpret_cast<float*>(ops0 + kFacGroups * 2 * kOp);   // per group: the pivot block
+  Shared& sh = *reinterpret_cast<Shared*>(psm0 + kFacGroups * 64);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -126,14 +135,15 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
       mbar_init(&sh.full[i], 1);
       mbar_init(&sh.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.tfull[i], 1);
-      mbar_init(&sh.aready[i], 128);
-      mbar_init(&sh.fin[i], 128);
-      mbar_init(&sh.tempty[i], 128);
+    mbar_init(&sh.gdone, 1);
+    mbar_init(&sh.bfree, 128);
+    for (int i = 0; i < kARegions; ++i) mbar_init(&sh.tempty[i], 128);
+    for (int g = 0; g < kFacGroups; ++g) {
+      mbar_init(&sh.aready[g], 128);
+      mbar_init(&sh.fin[g], 128);
+      mbar_init(&sh.upd[g], 1);
+      mbar_init(&sh.fdone[g], 1);
     }
-    mbar_init(&sh.upd, 1);
-    mbar_init(&sh.fdone, 1);
     mbar_init(&sh.drain, 1);
     sh.bad = 0;
     sh.abort = 0;
@@ -199,19 +209,20 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int tb = 0;
-      uint32_t tphase = 0;
       const uint32_t sbase = smem_u32(stages);
-      for (int s = blockIdx.x; s < slots && !aborted(sh); s += gridDim.x) {
+      int j = 0;
+      for (int s = blockIdx.x; s < slots && !aborted(sh); s += gridDim.x, ++j) {
         int rows, z;
         bool text;
         slot_info(p, s, rows, z, text);
-        if (!mbar_wait(&sh.tempty[tb], tphase ^ 1)) {
+        const int reg = j % kARegions;
+        // The A region's previous slot has had its M written; the B region is drained.
+        if (!mbar_wait(&sh.tempty[reg], ((j / kARegions) & 1) ^ 1) || !mbar_wait(&sh.bfree, (j & 1) ^ 1)) {
           set_abort(sh, p.err);
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + tb * 256;
+        const uint32_t da = tmem + reg * 128, db = tmem + kBCol;
         bool first = true;
         for (int r0 = 0; r0 < rows; r0 += kChunk) {
           if (!mbar_wait(&sh.full[stage], phase)) {
@@ -222,9 +233,12 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           const uint32_t sa = sbase + stage * kStageBytes;
 #pragma unroll
           for (int k = 0; k < kChunk / 16; ++k) {
-            // 16 tokens = 16 rows of 128 bytes; MN blocks of 64 features 8 KB apart.
-            const uint64_t desc = smem_desc(sa + k * 16 * 128, kBox, 1024, kSwizzle128B);
-            mma_bf16_ss(d, desc, desc, kIdescGram, first ? 0u : 1u);
+            // 16 tokens = 16 rows of 128 bytes; MN blocks of 64 features 8 KB
+            // apart: K features in boxes 0-1, V features in boxes 2-3.
+            const uint64_t dk = smem_desc(sa + k * 16 * 128, kBox, 1024, kSwizzle128B);
+            const uint64_t dv = smem_desc(sa + 2 * kBox + k * 16 * 128, kBox, 1024, kSwizzle128B);
+            mma_bf16_ss(da, dk, dk, kIdescGram, first ? 0u : 1u);   // A = K^T K
+            mma_bf16_ss(db, dk, dv, kIdescGram, first ? 0u : 1u);   // B = K^T V
             first = false;
           }
           mma_commit(&sh.empty[stage]);
@@ -234,9 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           }
         }
         if (aborted(sh)) break;
-        mma_commit(&sh.tfull[tb]);   // with no tokens this only marks the buffer (A = lambda I, B = 0)
-        tb ^= 1;
-        if (tb == 0) tphase ^= 1;
+        mma_commit(&sh.gdone);   // with no tokens this only marks the slot (A = lambda I, B = 0)
       }
       // Make sure no MMA is still running before TMEM is released.
       mma_commit(&sh.drain);
@@ -245,15 +257,15 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
   } else if (warp < 6) {
     // ------------------------------------------------------------ service warps
     // Per slot, in order: B_t out (TMEM -> swizzled 32-column chunks -> TMA
-    // stores), lambda onto A's diagonal in TMEM, hand A to the factor group;
-    // then, once the factor group has swept the previous slot, M_t of that
-    // slot out of TMEM into global memory, and the buffer back to the Gram.
+    // stores), lambda onto A's diagonal in TMEM, hand A to the slot's factor
+    // group; then, once the previous slot's sweep is complete, M of that slot
+    // out of TMEM into global memory, and its A region back to the Gram.
     const int quarter = warp % 4;            // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;     // feature index i of D
     const bool leader = (warp == 2 && lane == 0);
     int nst = 0;
-    auto write_m = [&](int s, int tb) {     // M = lambda (2I - A_final), row `row`, bf16 hi/lo
-      const uint32_t trow = tmem + tb * 256 + ((uint32_t)(quarter * 32) << 16);
+    auto write_m = [&](int s, int reg) {    // M = lambda (2I - A_final), row `row`, bf16 hi/lo
+      const uint32_t trow = tmem + reg * 128 + ((uint32_t)(quarter * 32) << 16);
       uint8_t* hi = p.M + (size_t)s * 65536;
       uint8_t* lo = hi + 32768;
 #pragma unroll 1
@@ -280,25 +292,39 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         }
       }
     };
-    int prev_s = -1, prev_tb = 0;
-    uint32_t fphase = 0;                      // phase of fin[] for the previous slot
+    // M of slot number jm (this CTA's order) once its group's sweep is complete.
+    auto finish_m = [&](int jm, int sm) -> bool {
+      const int g = jm % kFacGroups;
+      const bool ok = !aborted(sh) && mbar_wait(&sh.fin[g], (jm / kFacGroups) & 1);
+      if (!ok && !aborted(sh)) set_abort(sh, p.err);
+      if (named_bar_or(kEpiBar, 128, !ok)) return false;   // one decision for the four warps
+      tc_fence_after();
+      write_m(sm, jm % kARegions);
+      tc_fence_before();
+      mbar_arrive(&sh.tempty[jm % kARegions]);
+      return true;
+    };
+    int prev_s = -1;
     int j = 0;
+    bool live = true;
     for (int s = blockIdx.x; s < slots; s += gridDim.x, ++j) {
-      const int tb = j & 1;
-      const uint32_t tphase = (j >> 1) & 1;
+      const int reg = j % kARegions;
       int rows, z;
       bool text;
       slot_info(p, s, rows, z, text);
-      bool ok = !aborted(sh) && mbar_wait(&sh.tfull[tb], tphase);
+      bool ok = !aborted(sh) && mbar_wait(&sh.gdone, j & 1);
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
-      if (named_bar_or(kEpiBar, 128, !ok)) break;   // one decision for the four warps
+      if (named_bar_or(kEpiBar, 128, !ok)) {
+        live = false;
+        break;
+      }
       tc_fence_after();
-      const uint32_t trow = tmem + tb * 256 + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int chunk = 0; chunk < 4; ++chunk) {
         uint32_t r[32];
         if (rows > 0) {
-          tmem_ld_32x32b_x32(trow + 128 + chunk * 32, r);
+          tmem_ld_32x32b_x32(tq + kBCol + chunk * 32, r);
           tmem_ld_wait();
         } else {  // no tokens: B = 0
 #pragma unroll
@@ -318,8 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         }
         ++nst;
       }
+      tc_fence_before();
+      mbar_arrive(&sh.bfree);
       // lambda on the diagonal (A = lambda I when the slot has no tokens).
       {
+        const uint32_t trow = tq + reg * 128;
         uint32_t r[32];
         const int c0 = (row / 32) * 32;
         if (rows > 0) {
@@ -342,52 +371,44 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         tmem_st_wait();
       }
       tc_fence_before();
-      mbar_arrive(&sh.aready[tb]);
-      if (prev_s >= 0) {
-        // M of the previous slot, once the factor group has swept it.
-        ok = !aborted(sh) && mbar_wait(&sh.fin[prev_tb], fphase);
-        if (!ok && !aborted(sh)) set_abort(sh, p.err);
-        if (named_bar_or(kEpiBar, 128, !ok)) break;
-        fphase ^= (prev_tb == 1) ? 1u : 0u;
-        tc_fence_after();
-        write_m(prev_s, prev_tb);
-        tc_fence_before();
-        mbar_arrive(&sh.tempty[prev_tb]);
+      mbar_arrive(&sh.aready[j % kFacGroups]);
+      if (prev_s >= 0 && !finish_m(j - 1, prev_s)) {
+        live = false;
+        break;
       }
       prev_s = s;
-      prev_tb = tb;
     }
-    if (prev_s >= 0) {                        // the same for the four warps
-      const bool ok = !aborted(sh) && mbar_wait(&sh.fin[prev_tb], fphase);
-      if (!ok && !aborted(sh)) set_abort(sh, p.err);
-      if (!named_bar_or(kEpiBar, 128, !ok)) {
-        tc_fence_after();
-        write_m(prev_s, prev_tb);
-      }
-    }
+    if (live && prev_s >= 0) finish_m(j - 1, prev_s);   // the same for the four warps
     if (leader) bulk_wait<0>();               // B stores complete before exit
   } else {
-    // ------------------------------------------------------------ factor group
+    // ------------------------------------------------------------ factor groups
+    // Group g sweeps this CTA's slots g, g + kFacGroups, ...: while one group
+    // waits on its update MMAs the other factors its pivot block.
+    const int g = (warp - 6) / 4;
     const int i = (warp % 4) * 32 + lane;    // row of A = TMEM lane (warp % 4 = lane quarter)
-    const bool issuer = (warp == 6 && lane == 0);
+    const bool issuer = ((warp - 6) % 4 == 0 && lane == 0);   // first thread of the group
+    const int bar = kFacBar0 + g;
+    uint8_t* ops = ops0 + g * 2 * kOp;
+    float (*psm)[8] = reinterpret_cast<float (*)[8]>(psm0 + g * 64);
     const uint32_t opaddr = smem_u32(ops);
-    int nslot = 0;                            // slots factored by this CTA
-    for (int s = blockIdx.x; s < slots; s += gridDim.x, ++nslot) {
-      const int tb = nslot & 1;
-      bool ok = !aborted(sh) && mbar_wait(&sh.aready[tb], (nslot >> 1) & 1);
+    int nslot = 0;                            // slots swept by this group
+    int j = g;                                // this CTA's slot number
+    for (int s = blockIdx.x + g * gridDim.x; s < slots; s += kFacGroups * gridDim.x, ++nslot, j += kFacGroups) {
+      const int reg = j % kARegions;
+      bool ok = !aborted(sh) && mbar_wait(&sh.aready[g], nslot & 1);
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
-      if (named_bar_or(kFacBar, 128, !ok)) break;
+      if (named_bar_or(bar, 128, !ok)) break;
       tc_fence_after();
-      const uint32_t trow = tmem + tb * 256 + ((uint32_t)((warp % 4) * 32) << 16);
+      const uint32_t trow = tmem + reg * 128 + ((uint32_t)((warp % 4) * 32) << 16);
 
       bool bad = false;
       int steps_issued = 0;
 #pragma unroll 1
       for (int K = 0; K < 16; ++K) {
         if (K > 0) {
-          const bool okw = mbar_wait(&sh.upd, (K - 1) & 1);
+          const bool okw = mbar_wait(&sh.upd[g], (K - 1) & 1);
           if (!okw) set_abort(sh, p.err);
-          if (named_bar_or(kFacBar, 128, !okw)) break;   // the same for every thread
+          if (named_bar_or(bar, 128, !okw)) break;   // the same for every thread
           tc_fence_after();
         }
         float x[8];
@@ -405,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           *reinterpret_cast<float4*>(&psm[i & 7][0]) = make_float4(x[0], x[1], x[2], x[3]);
           *reinterpret_cast<float4*>(&psm[i & 7][4]) = make_float4(x[4], x[5], x[6], x[7]);
         }
-        named_bar_sync(kFacBar, 128);
+        named_bar_sync(bar, 128);
         float l[8][8];     // lower triangle: P, then L
         float dinv[8];     // 1 / L_jj
 #pragma unroll
@@ -453,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        named_bar_sync(kFacBar, 128);
+        named_bar_sync(bar, 128);
         if (issuer) {
           tc_fence_after();
           // A -= Y Y^T: Y is the A operand (M x K) and, read K-major from the
@@ -461,23 +482,23 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           // lo hi; the lo lo product is below float32 rounding of the update.
           const uint64_t yhi = smem_desc(opaddr + 0 * kOp, 2048, 128, kSwizzleNone);
           const uint64_t ylo = smem_desc(opaddr + 1 * kOp, 2048, 128, kSwizzleNone);
-          const uint32_t d = tmem + tb * 256;
+          const uint32_t d = tmem + reg * 128;
           mma_tf32_ss(d, yhi, yhi, kIdescUpd, 1u);
           mma_tf32_ss(d, yhi, ylo, kIdescUpd, 1u);
           mma_tf32_ss(d, ylo, yhi, kIdescUpd, 1u);
-          mma_commit(&sh.upd);
+          mma_commit(&sh.upd[g]);
         }
         ++steps_issued;
       }
       if (bad && i == 0) sh.bad = 1;   // every thread saw the same pivots
       // One more commit covers every update MMA issued for this slot; wait for
       // it (bounded), also on the error path, before the buffer is handed on.
-      if (issuer) mma_commit(&sh.fdone);
-      ok = mbar_wait(&sh.fdone, nslot & 1) && steps_issued == 16;
+      if (issuer) mma_commit(&sh.fdone[g]);
+      ok = mbar_wait(&sh.fdone[g], nslot & 1) && steps_issued == 16;
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
-      if (named_bar_or(kFacBar, 128, !ok)) break;
+      if (named_bar_or(bar, 128, !ok)) break;
       tc_fence_before();
-      mbar_arrive(&sh.fin[tb]);
+      mbar_arrive(&sh.fin[g]);
     }
   }
 
@@ -510,7 +531,7 @@ cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, c
   prm.n = p.n;
   prm.n_txt = p.n_txt;
   prm.lam = p.lambda;
-  const size_t smem = 1024 + kStages * kStageBytes + 2 * kOutChunk + 2 * kOp + 8 * 8 * 4 + sizeof(Shared);
+  const size_t smem = 1024 + kStages * kStageBytes + 2 * kOutChunk + kFacGroups * (2 * kOp + 8 * 8 * 4) + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(gramfactor_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
