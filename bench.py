@@ -281,6 +281,21 @@ def config_of(w, n):
             "l2": f"inputs larger than L2 ({input_bytes(w) / 1e9:.2f} GB read per step vs 126 MB); no flush"}
 
 
+def max_over_ranks(ms, dist, device):
+    """The job's device time: the slowest rank's (ms on every rank afterwards)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([float(ms)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank, n_ranks, ms_per_step):
+    """Whole-job throughput: every rank's units over the job's time per step."""
+    return n_ranks * units_per_rank / (ms_per_step / 1e3)
+
+
 def input_bytes(w):
     es = 2 if w.dtype == 1 else 4
     return (w.B * w.H * (w.T * w.n * 2 * (w.d_k + w.d_v) + w.n_txt * (w.d_k + w.d_v))) * es
@@ -358,12 +373,9 @@ def run_b200(args, w):
     if w.dtype == 1:   # one kernel for the Gram and the factor: report them as one stage
         stage_ms = {"gram+factor": stage_ms["gram"] + stage_ms["factor"], "scan": stage_ms["scan"],
                     "readout": stage_ms["readout"]}
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, pg, dev)
     ms_step = ms / args.steps
-    value = ws_n * w.units / (ms_step / 1e3)
+    value = job_value(w.units, ws_n, ms_step)
 
     # dominant kernel roofline
     work = stage_work(w)
@@ -405,13 +417,10 @@ def run_b200(args, w):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, pg, dev)
     h2d = sum(v.numel() * v.element_size() for k, v in host.items() if (w.n_txt or k not in ("K_txt", "V_txt")))
     d2h = Oh.numel() * Oh.element_size()
-    e2e = {"value": ws_n * w.units / (e2e_ms / e2e_steps / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    e2e = {"value": job_value(w.units, ws_n, e2e_ms / e2e_steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": e2e_steps,
            "api": "vda_forward_host (C ABI, pinned host buffers)"}
     return finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks)
