@@ -102,8 +102,13 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
   unsigned* err = reinterpret_cast<unsigned*>(ws + L.err);
   float* M = reinterpret_cast<float*>(ws + L.M);
   float* C = reinterpret_cast<float*>(ws + L.C);
+  // float32 path: the states live in the workspace unless the caller wants
+  // them.  bf16 path: the workspace holds bf16 states for the readout; the
+  // caller's float32 state buffers, if any, are written besides.
   float* SF = S_fwd ? S_fwd : reinterpret_cast<float*>(ws + L.SF);
   float* SB = S_bwd ? S_bwd : reinterpret_cast<float*>(ws + L.SB);
+  __nv_bfloat16* SFb = reinterpret_cast<__nv_bfloat16*>(ws + L.SF);
+  __nv_bfloat16* SBb = reinterpret_cast<__nv_bfloat16*>(ws + L.SB);
   cudaError_t e = cudaMemsetAsync(err, 0, 256, st);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
   const TIn* q = static_cast<const TIn*>(Q);
@@ -130,13 +135,14 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
   }
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
   if constexpr (kBf16) {
-    if ((e = vda::launch_scan_tc(p, M, C, SF, SB, err, st)) != cudaSuccess) return cuda_fail(e, "scan launch");
+    if ((e = vda::launch_scan_tc(p, M, C, SFb, SBb, S_fwd, S_bwd, err, st)) != cudaSuccess)
+      return cuda_fail(e, "scan launch");
   } else {
     if ((e = vda::launch_scan_simt(p, M, C, SF, SB, st)) != cudaSuccess) return cuda_fail(e, "scan launch");
   }
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "event record");
   if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-    if ((e = vda::launch_readout_tc(p, q, g, SF, SB, static_cast<TIn*>(O), err, st)) != cudaSuccess)
+    if ((e = vda::launch_readout_tc(p, q, g, SFb, SBb, static_cast<TIn*>(O), err, st)) != cudaSuccess)
       return cuda_fail(e, "readout launch");
   } else {
     if ((e = vda::launch_readout_simt<TIn>(p, q, g, SF, SB, static_cast<TIn*>(O), st)) != cudaSuccess)

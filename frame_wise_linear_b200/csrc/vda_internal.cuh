@@ -37,8 +37,11 @@ inline Layout make_layout(const vda_problem& p) {
   L.err = off;  off += 256;
   L.M = off;    off = align_up(off + slots * p.d_k * p.d_k * sizeof(float), 256);
   L.C = off;    off = align_up(off + slots * p.d_k * p.d_v * sizeof(float), 256);
-  L.SF = off;   off = align_up(off + frames * p.d_k * p.d_v * sizeof(float), 256);
-  L.SB = off;   off = align_up(off + frames * p.d_k * p.d_v * sizeof(float), 256);
+  // The states for the readout: float32 on the float32 path; bfloat16 (the
+  // readout's MMA operand) on the bfloat16 path.
+  const size_t se = p.dtype == VDA_DTYPE_BF16 ? 2 : sizeof(float);
+  L.SF = off;   off = align_up(off + frames * p.d_k * p.d_v * se, 256);
+  L.SB = off;   off = align_up(off + frames * p.d_k * p.d_v * se, 256);
   L.total = off;
   return L;
 }
@@ -62,8 +65,10 @@ cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool sp
 
 // Tensor-core scan (vda_scan_tc.cu): bf16 path, d_k = d_v = 128; M in the
 // split layout above, B_t float32 in the C region.
-cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
-                           unsigned* err, cudaStream_t st);
+// S^f, S^b go to SFb, SBb as bfloat16 ([frames][d_k][d_v], the readout's
+// operand); also as float32 to SF, SB when both are non-null.
+cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, __nv_bfloat16* SFb,
+                           __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st);
 
 // Gram and factor in one kernel (vda_gramfactor_tc.cu): bf16 inputs,
 // d_k = d_v = 128.  Writes each slot's M_t (the bf16 hi/lo image described
@@ -73,9 +78,10 @@ cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, c
                                  unsigned* err, cudaStream_t st);
 
 // Tensor-core readout (vda_readout_tc.cu): bf16 Q, G, O, d_k = d_v = 128.
+// SF, SB: the bfloat16 states written by launch_scan_tc.
 cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,
-                              const float* SF, const float* SB, __nv_bfloat16* O, unsigned* err,
-                              cudaStream_t st);
+                              const __nv_bfloat16* SF, const __nv_bfloat16* SB, __nv_bfloat16* O,
+                              unsigned* err, cudaStream_t st);
 
 // TMA descriptor of a [items][rows][128] bf16 tensor, boxes of 64 features x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.

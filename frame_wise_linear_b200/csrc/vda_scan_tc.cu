@@ -12,7 +12,9 @@
 // MMA operand layout); X is split the same way; the product takes three MMA
 // passes, M_hi X_hi + M_hi X_lo + M_lo X_hi, accumulated in float32 (the
 // dropped M_lo X_lo term is below 2^-16 relative).  ||M_t||_2 <= 1, so the
-// per-step error does not grow along the chain.
+// per-step error does not grow along the chain.  Each state goes out as
+// bfloat16 in the readout's operand layout (row-major, d_k x d_v); float32
+// states are written as well when the caller asks for them.
 //
 // The recurrence is independent per column of S, so each chain is split over
 // kSplit CTAs of N = 128 / kSplit columns.  CTA layout (288 threads):
@@ -48,14 +50,14 @@ constexpr int kAhead = 4;                    // steps of M_t and B_t prefetched 
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, N, /*a MN*/ false, /*b MN*/ true);
 
 struct ScanTcParams {
-  CUtensorMap mSF, mSB; // [frames * 128][128] float32, 32 x 128 boxes
-  CUtensorMap mB;       // [slots * 128][128] float32, 32 x 128 boxes
-  const uint8_t* M;     // per slot 64 KB: M hi (32 KB) | M lo (32 KB)
-  const float* Bm;      // per slot 128 x 128 float
-  float* SF;
-  float* SB;
+  CUtensorMap mSFb, mSBb;  // states for the readout: [frames][128][128] bfloat16, 64 x 128 boxes
+  CUtensorMap mSF, mSB;    // optional float32 states: [frames * 128][128], 32 x 128 boxes
+  CUtensorMap mB;          // [slots * 128][128] float32, 32 x 128 boxes
+  const uint8_t* M;        // per slot 64 KB: M hi (32 KB) | M lo (32 KB)
+  const float* Bm;         // per slot 128 x 128 float
   unsigned* err;
   int T;
+  int f32_out;             // also write the float32 states
   float lam;
 };
 
@@ -200,24 +202,42 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     float srow[kCols];
 #pragma unroll
     for (int j = 0; j < kCols; ++j) srow[j] = 0.f;
-    // S_t row m -> swizzled staging (32-column boxes) -> TMA store.  Runs
-    // while the next step's MMAs do: S_{t+1} needs only srow.
+    // S_t row m -> swizzled staging -> TMA store, while the next step's MMAs
+    // run (S_{t+1} needs only srow): as bfloat16, the readout's operand (this
+    // CTA's 64 columns are one 128-byte-swizzled box), and, when asked for,
+    // as float32 (two 32-column boxes) through the same buffer.
+    const bool leader = (warp == 0 && lane == 0);
     auto store_state = [&](int s) {
       const int t = dir == 0 ? s : T + 1 - s;
-      if (warp == 0 && lane == 0) bulk_wait_read<0>();   // the previous store has read the buffer
+      const int frame = bh * T + (t - 1);
+      if (leader) bulk_wait_read<0>();      // the previous store has read the buffer
       named_bar_sync(kEpiBar, 32 * kRowWarps);
 #pragma unroll
-      for (int q = 0; q < kCols / 4; ++q)
-        *reinterpret_cast<float4*>(sstage + hc * 16384 + sw128(m, q)) =
-            make_float4(srow[4 * q], srow[4 * q + 1], srow[4 * q + 2], srow[4 * q + 3]);
+      for (int q = 0; q < kCols / 8; ++q)
+        *reinterpret_cast<uint4*>(sstage + sw128(m, (kCols / 8) * hc + q)) =
+            make_uint4(pack_bf16(srow[8 * q], srow[8 * q + 1]), pack_bf16(srow[8 * q + 2], srow[8 * q + 3]),
+                       pack_bf16(srow[8 * q + 4], srow[8 * q + 5]), pack_bf16(srow[8 * q + 6], srow[8 * q + 7]));
       fence_proxy_async_smem();
       named_bar_sync(kEpiBar, 32 * kRowWarps);
-      if (warp == 0 && lane == 0) {
-        const CUtensorMap* map = dir == 0 ? &p.mSF : &p.mSB;
-        const int y = ((bh * T) + (t - 1)) * 128;
-#pragma unroll
-        for (int b = 0; b < N / 32; ++b) tma_store_2d(map, sstage + b * 16384, c0 + 32 * b, y);
+      if (leader) {
+        tma_store_3d(dir == 0 ? &p.mSFb : &p.mSBb, sstage, c0, 0, frame);
         bulk_commit();
+      }
+      if (p.f32_out) {                        // the same for every thread
+        if (leader) bulk_wait_read<0>();
+        named_bar_sync(kEpiBar, 32 * kRowWarps);
+#pragma unroll
+        for (int q = 0; q < kCols / 4; ++q)
+          *reinterpret_cast<float4*>(sstage + hc * 16384 + sw128(m, q)) =
+              make_float4(srow[4 * q], srow[4 * q + 1], srow[4 * q + 2], srow[4 * q + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(kEpiBar, 32 * kRowWarps);
+        if (leader) {
+          const CUtensorMap* map = dir == 0 ? &p.mSF : &p.mSB;
+#pragma unroll
+          for (int b = 0; b < N / 32; ++b) tma_store_2d(map, sstage + b * 16384, c0 + 32 * b, frame * 128);
+          bulk_commit();
+        }
       }
     };
     // The loop never breaks: after a timeout the waits are skipped, so the
@@ -261,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       }
     }
     if (T >= 1) store_state(T);
-    if (warp == 0 && lane == 0) bulk_wait<0>();   // S stores complete before exit
+    if (leader) bulk_wait<0>();               // S stores complete before exit
   }
 
   tc_fence_before();
@@ -272,19 +292,21 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
 
 }  // namespace
 
-cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, float* SF, float* SB,
-                           unsigned* err, cudaStream_t st) {
+cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, __nv_bfloat16* SFb,
+                           __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st) {
   ScanTcParams prm;
   memset(&prm, 0, sizeof(prm));
-  const long long rows = (long long)p.B * p.H * p.T * 128;
+  const int frames = p.B * p.H * p.T;
   const long long brows = (long long)p.B * p.H * (p.T + 1) * 128;
-  if (!make_f32_rows_map(&prm.mSF, SF, rows, 128) || !make_f32_rows_map(&prm.mSB, SB, rows, 128) ||
+  if (!make_bf16_rows_map(&prm.mSFb, SFb, 128, frames, 128) || !make_bf16_rows_map(&prm.mSBb, SBb, 128, frames, 128) ||
       !make_f32_rows_map(&prm.mB, Bm, brows, 128))
+    return cudaErrorInvalidValue;
+  prm.f32_out = (SF != nullptr && SB != nullptr) ? 1 : 0;
+  if (prm.f32_out && (!make_f32_rows_map(&prm.mSF, SF, (long long)frames * 128, 128) ||
+                      !make_f32_rows_map(&prm.mSB, SB, (long long)frames * 128, 128)))
     return cudaErrorInvalidValue;
   prm.M = reinterpret_cast<const uint8_t*>(M);
   prm.Bm = Bm;
-  prm.SF = SF;
-  prm.SB = SB;
   prm.err = err;
   prm.T = p.T;
   prm.lam = p.lambda;

@@ -25,8 +25,11 @@
  *     K_txt: [B, H, n_txt, d_k]     V_txt   : [B, H, n_txt, d_v]
  *     S_fwd, S_bwd (states)          : [B, H, T, d_k, d_v], float32
  * Inputs and O share one element type, vda_problem.dtype: float32 or
- * bfloat16.  The state and every accumulation are float32; O is rounded to
- * its type with round-to-nearest-even.
+ * bfloat16.  The state recurrence and every accumulation are float32; O is
+ * rounded to its type with round-to-nearest-even.  With bfloat16 inputs the
+ * readout takes the two states as bfloat16 operands (O = sigmoid(G) *
+ * (Q S^f + Q S^b) with S^f, S^b rounded to bfloat16, accumulated in
+ * float32); the states returned by vda_forward_states are the float32 ones.
  *
  * Ownership.  The caller owns every buffer.  Device pointers must be CUDA
  * device memory of the current device, 16-byte aligned.  The library

@@ -47,11 +47,15 @@ def _p(**kw):
     return vda.make_problem(**base)
 
 
-def test_workspace_size_valid(lib):
-    p = _p()
+@pytest.mark.parametrize("dtype,state_bytes", [(vda.VDA_DTYPE_BF16, 2), (vda.VDA_DTYPE_F32, 4)])
+def test_workspace_size_valid(lib, dtype, state_bytes):
+    # error word, M and B_t per slot (float32), S^f and S^b per frame (bf16 on
+    # the bf16 path, where they are the readout's operands; float32 otherwise)
+    p = _p(dtype=dtype)
     nb = vda.vda_workspace_size(p)
-    slots = 1 * 2 * 4
-    assert nb >= 256 + slots * 128 * 128 * 4 * 2 + 6 * 128 * 128 * 4 * 2
+    slots, frames = 1 * 2 * 4, 1 * 2 * 3
+    assert nb >= 256 + slots * 128 * 128 * 4 * 2 + frames * 128 * 128 * state_bytes * 2
+    assert nb < 256 + slots * 128 * 128 * 4 * 2 + frames * 128 * 128 * state_bytes * 2 + 5 * 256
     assert vda.vda_host_workspace_size(p) > nb
 
 
