@@ -131,7 +131,7 @@ vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
   if constexpr (!kBf16) {
-    if ((e = vda::launch_factor(p, M, err, false, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
+    if ((e = vda::launch_factor(p, M, err, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
   }
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
   if constexpr (kBf16) {

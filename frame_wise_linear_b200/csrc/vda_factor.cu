@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kThreads = 160;
 
-template <int D, bool kSplitOut>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 3) factor_sweep_kernel(float* __restrict__ Mreg, float lam,
                                                                    unsigned* __restrict__ err) {
   // xs[b][0] = column k, xs[b][1] = column k + 1, both before the pair of pivots.
@@ -58,36 +58,28 @@ __global__ void __launch_bounds__(kThreads, 3) factor_sweep_kernel(float* __rest
 #pragma unroll
     for (int c = 0; c < 8; ++c) a[r][c] *= -lam;
 
-  if constexpr (kSplitOut) {
-    sweep::store_split(a, R, C, reinterpret_cast<uint8_t*>(A));
-  } else {
-    sweep::store_f32<D>(a, R, C, A);
-  }
+  sweep::store_f32<D>(a, R, C, A);
 }
 
-template <int D, bool kSplit>
+template <int D>
 cudaError_t launch_d(const vda_problem& p, float* M, unsigned* err, cudaStream_t st) {
   const unsigned slots = (unsigned)(p.B * p.H * (p.T + 1));
-  factor_sweep_kernel<D, kSplit><<<slots, kThreads, 0, st>>>(M, p.lambda, err);
+  factor_sweep_kernel<D><<<slots, kThreads, 0, st>>>(M, p.lambda, err);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool split_bf16, cudaStream_t st) {
-  if (split_bf16) {
-    if (p.d_k != 128) return cudaErrorInvalidValue;
-    return launch_d<128, true>(p, M, err, st);
-  }
+cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, cudaStream_t st) {
   switch (p.d_k) {
-    case 16: return launch_d<16, false>(p, M, err, st);
-    case 32: return launch_d<32, false>(p, M, err, st);
-    case 48: return launch_d<48, false>(p, M, err, st);
-    case 64: return launch_d<64, false>(p, M, err, st);
-    case 80: return launch_d<80, false>(p, M, err, st);
-    case 96: return launch_d<96, false>(p, M, err, st);
-    case 112: return launch_d<112, false>(p, M, err, st);
-    case 128: return launch_d<128, false>(p, M, err, st);
+    case 16: return launch_d<16>(p, M, err, st);
+    case 32: return launch_d<32>(p, M, err, st);
+    case 48: return launch_d<48>(p, M, err, st);
+    case 64: return launch_d<64>(p, M, err, st);
+    case 80: return launch_d<80>(p, M, err, st);
+    case 96: return launch_d<96>(p, M, err, st);
+    case 112: return launch_d<112>(p, M, err, st);
+    case 128: return launch_d<128>(p, M, err, st);
   }
   return cudaErrorInvalidValue;
 }

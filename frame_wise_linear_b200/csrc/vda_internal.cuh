@@ -57,11 +57,9 @@ template <typename TIn>
 cudaError_t launch_readout_simt(const vda_problem& p, const TIn* Q, const TIn* G,
                                 const float* SF, const float* SB, TIn* O, cudaStream_t st);
 
-// Factor step (vda_factor.cu): overwrites each slot's A_t in M with
-// M_t = lambda A_t^{-1}, as float32 row-major or, with split_bf16 (d_k = 128),
-// as bf16 hi and lo halves in the K-major 128-byte-swizzled MMA operand image
-// (32 KB each, same 64 KB per slot).
-cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, bool split_bf16, cudaStream_t st);
+// Factor step of the float32 path (vda_factor.cu): overwrites each slot's A_t
+// in M with M_t = lambda A_t^{-1}, float32 row-major.
+cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, cudaStream_t st);
 
 // Tensor-core scan (vda_scan_tc.cu): bf16 path, d_k = d_v = 128; M in the
 // split layout above, B_t float32 in the C region.
@@ -71,8 +69,9 @@ cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm
                            __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st);
 
 // Gram and factor in one kernel (vda_gramfactor_tc.cu): bf16 inputs,
-// d_k = d_v = 128.  Writes each slot's M_t (the bf16 hi/lo image described
-// under launch_factor) into M and B_t into Bm; A_t stays in TMEM.
+// d_k = d_v = 128.  Writes each slot's M_t into M as bf16 hi and lo halves
+// (32 KB each) of the K-major, 128-byte-swizzled image of the scan's MMA A
+// operand, and B_t into Bm; A_t stays in TMEM.
 cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
                                  const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* M, float* Bm,
                                  unsigned* err, cudaStream_t st);

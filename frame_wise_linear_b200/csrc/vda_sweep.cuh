@@ -1,6 +1,6 @@
 // The symmetric sweep operator on a d x d SPD matrix held as 8x8 register
-// blocks of its lower triangle (one block per thread), shared by the
-// stand-alone factor kernel and the fused Gram + factor kernel.
+// blocks of its lower triangle (one block per thread): the factor step of the
+// float32 path.
 //
 // Sweeping pivot k maps a_kk -> -1/a_kk, a_ik -> a_ik/a_kk and
 // a_ij -> a_ij - a_ik a_kj / a_kk (in-place Gauss-Jordan with diagonal pivots,
@@ -12,7 +12,6 @@
 // column from the two.
 #pragma once
 
-#include "sm100.cuh"
 #include "vda_internal.cuh"
 
 namespace vda {
@@ -143,49 +142,6 @@ __device__ __forceinline__ bool invert(float (&a)[8][8], int R, int C, bool acti
     pair(std::integral_constant<int, 6>{});
   }
   return bad;
-}
-
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Writes 8 consecutive k-values of row m of M as bf16 hi and lo chunks of the
-// K-major, 128-byte-swizzled MMA operand image (two 64-column halves of 16 KB).
-__device__ __forceinline__ void store_split_chunk(uint8_t* hi, uint8_t* lo, int m, int kchunk, const float (&v)[8]) {
-  float h[8], l[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    h[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
-    l[i] = v[i] - h[i];
-  }
-  const uint32_t off = (kchunk / 8) * 16384u + sm100::sw128(m, kchunk % 8);
-  *reinterpret_cast<uint4*>(hi + off) = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
-  *reinterpret_cast<uint4*>(lo + off) = make_uint4(pack2(l[0], l[1]), pack2(l[2], l[3]), pack2(l[4], l[5]), pack2(l[6], l[7]));
-}
-
-// Writes this thread's block of the symmetric result and its transpose as
-// bf16 hi (bytes [0, 32K)) and lo ([32K, 64K)) halves of the K-major,
-// 128-byte-swizzled MMA operand image of a 128 x 128 matrix.
-__device__ __forceinline__ void store_split(const float (&a)[8][8], int R, int C, uint8_t* img) {
-  uint8_t* hi = img;
-  uint8_t* lo = img + 32768;
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    float v[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) v[c] = a[r][c];
-    store_split_chunk(hi, lo, 8 * R + r, C, v);
-  }
-  if (R != C) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float v[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) v[r] = a[r][c];
-      store_split_chunk(hi, lo, 8 * C + c, R, v);
-    }
-  }
 }
 
 // Writes this thread's block and its transpose into a row-major D x D matrix.
