@@ -49,6 +49,7 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ tr
 
 struct ReadoutTcParams {
   CUtensorMap mQ, mG, mO;
+  CUtensorMap mSF, mSB;      // the same states as tiles: 64 columns x 128 rows, 128-byte swizzle
   const __nv_bfloat16* SF;   // [frames][128][128]
   const __nv_bfloat16* SB;
   unsigned* err;
@@ -62,6 +63,7 @@ struct Shared {
   uint64_t t_full[2], t_empty[2];
   uint64_t sig_full, sig_empty;
   uint64_t p_full[2];   // S staging slots
+  uint64_t s0_full;     // the first frame's states, loaded straight into the operand buffer
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -110,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     mbar_init(&sh.sig_empty, 1);
     mbar_init(&sh.p_full[0], 1);
     mbar_init(&sh.p_full[1], 1);
+    mbar_init(&sh.s0_full, 1);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     fence_barrier_init();
@@ -122,6 +125,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     tma_prefetch_desc(&p.mQ);
     tma_prefetch_desc(&p.mG);
     tma_prefetch_desc(&p.mO);
+    tma_prefetch_desc(&p.mSF);
+    tma_prefetch_desc(&p.mSB);
   }
   tc_fence_before();
   __syncthreads();
@@ -267,21 +272,24 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
   } else {
     // ------------------------------------------------------------ S prep
     // S^f and S^b (bfloat16) of each frame of this CTA's range, in order.
-    // The frame's 8 pieces (16 rows of S^f and of S^b, 4 KB each, contiguous)
-    // arrive by bulk copy in a 2-slot ring, issued by the first prep thread
-    // as slots free up, so no global load goes through the load/store unit (a
-    // burst of them there stalls the epilogue's shared-memory traffic).
-    // Thread pt keeps row 16 j + pt / 16, columns 8 (pt % 16) .. + 7 of every
-    // piece j in registers; once the MMAs release the operand buffer it writes
-    // them there (swizzled) and the next frame's pieces start.
+    // The first frame's go straight into the operand buffer, which is free
+    // at the start: four TMA tile loads (64 columns x 128 rows, swizzled as
+    // the MMA reads them), one round trip.  Every later frame's 8 pieces (16
+    // rows of S^f and of S^b, 4 KB each, contiguous) arrive by bulk copy in a
+    // 2-slot ring, issued by the first prep thread as slots free up, so no
+    // global load goes through the load/store unit (a burst of them there
+    // stalls the epilogue's shared-memory traffic).  Thread pt keeps row
+    // 16 j + pt / 16, columns 8 (pt % 16) .. + 7 of every piece j in
+    // registers; once the MMAs release the operand buffer it writes them
+    // there (swizzled) and the next frame's pieces start.
     const int pt = threadIdx.x - 320;         // 0..255
     const int prow = pt / 16;                 // row inside a piece
     const int pchunk = pt % 16;               // 8-column chunk
     const int u_first = t_begin / p.tiles_per_unit;
     const int u_last = t_end > t_begin ? (t_end - 1) / p.tiles_per_unit : u_first - 1;
-    const int n_pieces = (u_last - u_first + 1) * kPieces;
+    const int n_pieces = (u_last - u_first) * kPieces;   // frames after the first
     auto issue = [&](int g) {                 // piece g of the sequence into slot g % 2
-      const int u = u_first + g / kPieces, j = g % kPieces;
+      const int u = u_first + 1 + g / kPieces, j = g % kPieces;
       const size_t off = ((size_t)u * 128 + (size_t)j * kPieceRows) * 128;
       uint8_t* dst = sstage + (g & 1) * kPiece;
       mbar_expect_tx(&sh.p_full[g & 1], kPiece);
@@ -289,12 +297,32 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       bulk_load(dst + kPieceHalf, p.SB + off, kPieceHalf, &sh.p_full[g & 1]);
     };
     int issued = 0;
-    if (pt == 0) {
+    bool first_issued = false;
+    if (pt == 0 && u_first <= u_last) {
+      const uint64_t pol = policy_evict_first();
+      mbar_expect_tx(&sh.s0_full, kSig);
+      tma_load_3d(sig, &p.mSF, &sh.s0_full, 0, 0, u_first, pol);
+      tma_load_3d(sig + kBox, &p.mSF, &sh.s0_full, 64, 0, u_first, pol);
+      tma_load_3d(sig + kTile, &p.mSB, &sh.s0_full, 0, 0, u_first, pol);
+      tma_load_3d(sig + kTile + kBox, &p.mSB, &sh.s0_full, 64, 0, u_first, pol);
+      first_issued = true;
       for (; issued < 2 && issued < n_pieces; ++issued) issue(issued);
     }
     uint32_t seph = 0;
     int g = 0;                                 // pieces consumed
-    for (int u = u_first; u <= u_last; ++u) {
+    bool s0_waited = false, stop = false;
+    if (u_first <= u_last) {                   // the same for every prep thread
+      // The first frame: hand the operand buffer to the MMAs once it has landed.
+      const bool ok = mbar_wait(&sh.s0_full, 0);
+      s0_waited = true;
+      if (!ok) set_abort(sh, p.err);
+      stop = named_bar_or(3, 256, !ok);        // one decision for all prep threads
+      if (!stop) {
+        mbar_arrive(&sh.sig_full);
+        seph ^= 1;                             // the MMAs release the buffer once per frame
+      }
+    }
+    for (int u = u_first + 1; u <= u_last && !stop; ++u) {
       if (pt == 0 && u + 1 <= u_last) {
         // Read about a frame from now: bring into L2 first.
         bulk_prefetch_l2(p.SF + (size_t)(u + 1) * 128 * 128, 128 * 128 * 2);
@@ -325,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       fence_proxy_async_smem();
       mbar_arrive(&sh.sig_full);
     }
+    if (pt == 0 && first_issued && !s0_waited) mbar_wait(&sh.s0_full, 0);
     if (pt == 0) {   // let the copies still in flight land before exit
       for (int c = g; c < issued; ++c) mbar_wait(&sh.p_full[c & 1], (c >> 1) & 1);
     }
@@ -345,7 +374,8 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
   memset(&prm, 0, sizeof(prm));
   const int units = p.B * p.H * p.T;
   if (!make_bf16_rows_map(&prm.mQ, Q, p.n, units, kRows) || !make_bf16_rows_map(&prm.mG, G, p.n, units, kRows) ||
-      !make_bf16_rows_map(&prm.mO, O, p.n, units, kRows))
+      !make_bf16_rows_map(&prm.mO, O, p.n, units, kRows) || !make_bf16_rows_map(&prm.mSF, SF, 128, units, 128) ||
+      !make_bf16_rows_map(&prm.mSB, SB, 128, units, 128))
     return cudaErrorInvalidValue;
   prm.SF = SF;
   prm.SB = SB;
