@@ -319,6 +319,16 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start before the previous kernel on its stream has
+// finished; griddep_wait() blocks the calling thread until that kernel has
+// completed and its memory is visible.  griddep_launch_dependents() lets the
+// next such kernel start launching (its CTAs then take SMs as they free up).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier that also ORs a predicate over the participating threads:
 // every thread gets the same answer (one decision for a group of warps).
 __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {

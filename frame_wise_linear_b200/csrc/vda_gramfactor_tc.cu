@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  griddep_launch_dependents();   // the scan's CTAs may take SMs as this grid's finish
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

@@ -298,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     };
     int issued = 0;
     bool first_issued = false;
+    if (pt == 0) griddep_wait();              // the states come from the previous kernel
     if (pt == 0 && u_first <= u_last) {
       const uint64_t pol = policy_evict_first();
       mbar_expect_tx(&sh.s0_full, kSig);
@@ -390,8 +391,20 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long tiles = (long long)units * prm.tiles_per_unit;
   const int grid = (int)(tiles < sms ? tiles : sms);
-  readout_tc_kernel<<<grid, kThreads, smem, st>>>(prm);
-  return cudaGetLastError();
+  // Launched with programmatic stream serialization: its CTAs start as the
+  // scan's CTAs finish (or on SMs the scan leaves free) and begin loading Q
+  // and G; only the state loads wait for the scan (griddep_wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, readout_tc_kernel, prm);
 }
 
 }  // namespace vda

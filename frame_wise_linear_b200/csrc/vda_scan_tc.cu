@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  griddep_launch_dependents();   // the readout's CTAs may take SMs as this grid's finish
 
   if (warp == kMmaWarp) {
     if (lane == 0) {
@@ -144,6 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         bulk_prefetch_l2(p.M + slot_of(s) * (size_t)kMBytes, kMBytes);
         bulk_prefetch_l2(p.Bm + slot_of(s) * 128 * 128, 128 * 128 * 4);
       };
+      tma_prefetch_desc(&p.mB);
+      griddep_wait();                // M_t and B_t come from the previous kernel
       int issued = 0;
       issue_b(0);
       issue_load(0);
@@ -313,9 +316,20 @@ cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm
   const size_t smem = 1024 + 2 * kMBytes + 2 * kXHalf + kSStage + kBBuf + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(kSplit, 2, p.B * p.H);
-  scan_tc_kernel<<<grid, kThreads, smem, st>>>(prm);
-  return cudaGetLastError();
+  // Launched with programmatic stream serialization: its CTAs start as the
+  // Gram+factor kernel's CTAs finish, and its load thread waits for that
+  // kernel (griddep_wait) before reading M_t and B_t.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kSplit, 2, p.B * p.H);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, scan_tc_kernel, prm);
 }
 
 }  // namespace vda
