@@ -23,8 +23,9 @@
 //               and B_t, stage the previous state (swizzled) for a TMA store
 //               while the step's MMAs run, then read S_t back from TMEM;
 //   warp 8      one thread: bulk-copies M_t (64 KB) into a 2-stage ring and
-//               B_t (this CTA's columns) by TMA, ahead of time, and issues
-//               the 24 MMAs of each step.
+//               B_t (this CTA's columns) by TMA as soon as the row warps have
+//               copied the previous one into registers, and issues the 24
+//               MMAs of each step.
 // Every wait is bounded; a timeout sets the error bit and the CTA winds down.
 #include "sm100.cuh"
 #include "vda_internal.cuh"
@@ -63,7 +64,7 @@ struct ScanTcParams {
 
 struct Shared {
   uint64_t m_full[2], m_empty[2];
-  uint64_t x_full, d_full, b_full;
+  uint64_t x_full, d_full, b_full, b_empty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     mbar_init(&sh.x_full, 32 * kRowWarps);
     mbar_init(&sh.d_full, 1);
     mbar_init(&sh.b_full, 1);
+    mbar_init(&sh.b_empty, 32 * kRowWarps);
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     fence_barrier_init();
@@ -125,7 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       // ---------------------------------------------------- loads + MMAs
       // B_s: one box per 32 columns, into the buffer the row warps build X from.
       const uint64_t pol = policy_evict_first();
+      int b_last = -1;                         // last step whose B_s load was issued
       auto issue_b = [&](int s) {
+        b_last = s;
         mbar_expect_tx(&sh.b_full, kBBuf);
 #pragma unroll
         for (int b = 0; b < N / 32; ++b)
@@ -160,12 +164,17 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       const uint32_t xaddr = smem_u32(xbuf);
       for (int s = 0; s <= T; ++s) {
         const int st = s & 1;
+        // The row warps have copied B_s into registers: the buffer takes B_{s+1}.
+        if (!mbar_wait(&sh.b_empty, s & 1)) {
+          set_abort(sh, p.err);
+          break;
+        }
+        if (s + 1 <= T) issue_b(s + 1);
         if (!mbar_wait(&sh.m_full[st], (s >> 1) & 1) || !mbar_wait(&sh.x_full, s & 1)) {
           set_abort(sh, p.err);
           break;
         }
         tc_fence_after();
-        if (s + 1 <= T) issue_b(s + 1);        // X_s is built: the B buffer is free
         prefetch(s + kAhead);
         const uint32_t ma = maddr + st * kMBytes;
 #pragma unroll
@@ -193,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       }
       if (aborted(sh)) {  // copies still in flight land before exit
         for (int s = issued > 2 ? issued - 2 : 0; s < issued; ++s) mbar_wait(&sh.m_full[s & 1], (s >> 1) & 1);
+        if (b_last >= 0) mbar_wait(&sh.b_full, b_last & 1);
       }
       mma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
@@ -249,16 +259,24 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       // X row m = S_{s-1} row m + B_s row m / lambda, split into hi / lo, MN-major swizzled.
       const bool okb = !aborted(sh) && mbar_wait(&sh.b_full, s & 1);
       if (!okb && !aborted(sh)) set_abort(sh, p.err);
+      // B box hc (32 columns) into registers first, and the buffer back to
+      // the load thread at once, so B_{s+1} is on its way while X_s is built.
+      float bv[kCols];
+#pragma unroll
+      for (int q = 0; q < kCols / 4; ++q) {
+        const float4 b4 = *reinterpret_cast<const float4*>(bbuf + hc * 16384 + sw128(m, q));
+        bv[4 * q] = b4.x;
+        bv[4 * q + 1] = b4.y;
+        bv[4 * q + 2] = b4.z;
+        bv[4 * q + 3] = b4.w;
+      }
+      mbar_arrive(&sh.b_empty);
 #pragma unroll
       for (int q = 0; q < kCols / 8; ++q) {
         float h[8], l[8];
-        // B box hc (32 columns); this chunk of 8 columns is 16-byte chunks 2q, 2q + 1.
-        const float4 b0 = *reinterpret_cast<const float4*>(bbuf + hc * 16384 + sw128(m, 2 * q));
-        const float4 b1 = *reinterpret_cast<const float4*>(bbuf + hc * 16384 + sw128(m, 2 * q + 1));
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float x = fmaf(bv[i], inv_lam, srow[8 * q + i]);
+          const float x = fmaf(bv[8 * q + i], inv_lam, srow[8 * q + i]);
           h[i] = __bfloat162float(__float2bfloat16_rn(x));
           l[i] = x - h[i];
         }
