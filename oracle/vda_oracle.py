@@ -1,4 +1,5 @@
-"""Float64 CPU oracle for the Video Delta Attention (VDA) linear branch, forward.
+"""Float64 CPU oracle for the Video Delta Attention (VDA) linear branch:
+forward, and the backward (the gradients of the forward).
 
 TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
 execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
@@ -61,6 +62,8 @@ __all__ = [
     "sigmoid",
     "vda_head",
     "vda_forward",
+    "vda_head_backward",
+    "vda_backward",
 ]
 
 
@@ -224,3 +227,103 @@ def vda_forward(Q, K, V, G, K_txt, V_txt, lam: float, heads=None, return_states:
     if return_states:
         return O, states
     return O
+
+
+def vda_head_backward(Q, K, V, G, K_txt, V_txt, lam: float, dO):
+    """Gradients of one head's VDA forward, for the scalar L = sum(dO * O).
+
+    The pages give no backward; this is the exact derivative of ``vda_head``
+    (the reverse-mode chain rule through its steps), lam held fixed.  Inputs
+    as ``vda_head``; ``dO`` has O's shape.  Returns a dict of float64 arrays
+    dQ, dK, dV, dG, dK_txt, dV_txt (the last two None without text tokens).
+
+    Steps, with S_t = S^fwd_t + S^bwd_t and P_t = Q_t S_t:
+      dG_t = dO_t * P_t * s_t (1 - s_t), s_t = sigmoid(G_t);
+      dP_t = dO_t * s_t;  dQ_t = dP_t S_t^T;  E_t = Q_t^T dP_t.
+      The forward scan's adjoint runs from t = T down to 1:
+        Gf_t = A_t^{-1} (E_t + lam Gf_{t+1}),  Gf_{T+1} = 0,
+      and the backward scan's from t = 1 up to T:
+        Gb_t = A_t^{-1} (E_t + lam Gb_{t-1}),  Gb_0 = 0
+      (Gf_t is the gradient of lam S^fwd_{t-1} + B_t, the right-hand side of
+      frame t's solve; likewise Gb_t).  S_0 seeds both scans, so
+      G_0 = A_txt^{-1} lam (Gf_1 + Gb_T).  Each solve S = A^{-1} R gives
+      dR = A^{-1} dS and dA = -dR S^T, hence for t = 1..T
+        dB_t = Gf_t + Gb_t,   dA_t = -(Gf_t S^fwd_t^T + Gb_t S^bwd_t^T),
+      and for the text dB_0 = G_0, dA_0 = -G_0 S_0^T.  Through the normal
+      equations A = K^T K + lam I, B = K^T V:
+        dK = K (dA + dA^T) + V dB^T,   dV = K dB.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    T, _, d_k = K.shape
+    d_v = V.shape[2]
+    has_text = K_txt is not None and np.asarray(K_txt).shape[0] > 0
+    S0 = text_state(K_txt, V_txt, lam, d_k, d_v)
+    SF = scan_forward(S0, K, V, lam)
+    SB = scan_backward(S0, K, V, lam)
+    A = [normal_equations(K[t], V[t], lam)[0] for t in range(T)]
+
+    gate = sigmoid(G)
+    dQ = np.empty(Q.shape)
+    dG = np.empty(G.shape)
+    E = np.empty((T, d_k, d_v))
+    for t in range(T):
+        S = SF[t] + SB[t]
+        P = Q[t] @ S
+        dG[t] = dO[t] * P * gate[t] * (1.0 - gate[t])
+        dP = dO[t] * gate[t]
+        dQ[t] = dP @ S.T
+        E[t] = Q[t].T @ dP
+
+    Gf = np.empty((T, d_k, d_v))
+    nxt = np.zeros((d_k, d_v))
+    for t in range(T - 1, -1, -1):
+        Gf[t] = spd_solve(A[t], E[t] + lam * nxt)
+        nxt = Gf[t]
+    Gb = np.empty((T, d_k, d_v))
+    prv = np.zeros((d_k, d_v))
+    for t in range(T):
+        Gb[t] = spd_solve(A[t], E[t] + lam * prv)
+        prv = Gb[t]
+
+    dK = np.empty(K.shape)
+    dV = np.empty(V.shape)
+    for t in range(T):
+        dB = Gf[t] + Gb[t]
+        dA = -(Gf[t] @ SF[t].T + Gb[t] @ SB[t].T)
+        dK[t] = K[t] @ (dA + dA.T) + V[t] @ dB.T
+        dV[t] = K[t] @ dB
+
+    dK_txt = dV_txt = None
+    if has_text:
+        K_txt = np.asarray(K_txt, dtype=np.float64)
+        V_txt = np.asarray(V_txt, dtype=np.float64)
+        A0, _ = normal_equations(K_txt, V_txt, lam)
+        G0 = spd_solve(A0, lam * (Gf[0] + Gb[T - 1]))
+        dA0 = -G0 @ S0.T
+        dK_txt = K_txt @ (dA0 + dA0.T) + V_txt @ G0.T
+        dV_txt = K_txt @ G0
+    return {"dQ": dQ, "dK": dK, "dV": dV, "dG": dG, "dK_txt": dK_txt, "dV_txt": dV_txt}
+
+
+def vda_backward(Q, K, V, G, K_txt, V_txt, lam: float, dO, heads=None):
+    """``vda_head_backward`` over the [B, H, T, n, d] layout (or a list of
+    (b, h) pairs, stacked on a leading axis, as ``vda_forward``)."""
+    Bn, Hn = np.shape(Q)[0], np.shape(Q)[1]
+    pairs = [(b, h) for b in range(Bn) for h in range(Hn)] if heads is None else list(heads)
+    res = []
+    for b, h in pairs:
+        kt = None if K_txt is None else K_txt[b, h]
+        vt = None if V_txt is None else V_txt[b, h]
+        res.append(vda_head_backward(Q[b, h], K[b, h], V[b, h], G[b, h], kt, vt, lam, dO[b, h]))
+    out = {}
+    for k in res[0]:
+        if res[0][k] is None:
+            out[k] = None
+            continue
+        arr = np.stack([r[k] for r in res])
+        out[k] = arr.reshape((Bn, Hn) + arr.shape[1:]) if heads is None else arr
+    return out
