@@ -272,6 +272,50 @@ vda_status vda_forward_host(const vda_problem* p, const void* Q, const void* K, 
   return vda_sync_status(base + off, stream);
 }
 
+vda_status vda_backward_workspace_size(const vda_problem* p, size_t* bytes) {
+  g_msg[0] = 0;
+  vda_status s = check_problem(p);
+  if (s != VDA_OK) return s;
+  if (p->dtype != VDA_DTYPE_BF16)
+    return fail(VDA_ERR_UNSUPPORTED, "the backward supports bfloat16 inputs only");
+  if (!bytes) return fail(VDA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = vda::backward_workspace_bytes(*p);
+  return VDA_OK;
+}
+
+vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                        const void* K_txt, const void* V_txt, const void* dO, void* dQ, void* dK, void* dV,
+                        void* dG, void* dK_txt, void* dV_txt, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  size_t need = 0;
+  vda_status s = vda_backward_workspace_size(p, &need);
+  if (s != VDA_OK) return s;
+  if ((s = check_pointers(*p, Q, K, V, G, K_txt, V_txt, dO)) != VDA_OK) return s;
+  const void* outs[4] = {dQ, dK, dV, dG};
+  const char* names[4] = {"dQ", "dK", "dV", "dG"};
+  for (int i = 0; i < 4; ++i) {
+    if (!outs[i]) return fail(VDA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(outs[i])) return fail(VDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  if (p->n_txt > 0 && (!dK_txt || !dV_txt || !aligned16(dK_txt) || !aligned16(dV_txt)))
+    return fail(VDA_ERR_INVALID_ARG, "dK_txt / dV_txt NULL or not 16-byte aligned with n_txt = %d", p->n_txt);
+  if (!workspace) return fail(VDA_ERR_WORKSPACE, "workspace is NULL");
+  if ((uintptr_t)workspace & 255u) return fail(VDA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (workspace_bytes < need)
+    return fail(VDA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  using bf = __nv_bfloat16;
+  const char* where = "";
+  cudaError_t e = vda::run_backward(*p, static_cast<const bf*>(Q), static_cast<const bf*>(K),
+                                    static_cast<const bf*>(V), static_cast<const bf*>(G),
+                                    static_cast<const bf*>(K_txt), static_cast<const bf*>(V_txt),
+                                    static_cast<const bf*>(dO), static_cast<bf*>(dQ), static_cast<bf*>(dK),
+                                    static_cast<bf*>(dV), static_cast<bf*>(dG), static_cast<bf*>(dK_txt),
+                                    static_cast<bf*>(dV_txt), static_cast<char*>(workspace),
+                                    static_cast<cudaStream_t>(stream), &where);
+  if (e != cudaSuccess) return cuda_fail(e, where);
+  return VDA_OK;
+}
+
 vda_status vda_sync_status(void* workspace, void* stream) {
   g_msg[0] = 0;
   if (!workspace) return fail(VDA_ERR_WORKSPACE, "workspace is NULL");

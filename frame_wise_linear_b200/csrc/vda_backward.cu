@@ -1,0 +1,288 @@
+// VDA backward (bf16 inputs, d_k = d_v = 128): the gradients of O with
+// respect to Q, K, V, G, K_txt and V_txt for L = sum(dO * O).
+//
+// The pages give the forward only; this is its exact derivative (the chain
+// rule through "VDN-MiniMax-H3" (aiezz.com) section 03's normal-equation
+// solve, text injection and gate, and the bidirectional scan of "VDN-H3"
+// (comfyui-wiki.com)).  With S_t = S^f_t + S^b_t and P_t = Q_t S_t:
+//   dG_t = dO_t * P_t * s (1 - s),  dP_t = dO_t * s  (s = sigmoid(G_t));
+//   dQ_t = dP_t S_t^T;  E_t = Q_t^T dP_t.
+//   The forward scan's adjoint, run backward in time, and the backward
+//   scan's, run forward in time, have the scan's own form:
+//     Gf_t = M_t (Gf_{t+1} + E_t / lambda),   Gb_t = M_t (Gb_{t-1} + E_t / lambda),
+//   so the scan kernel computes them (E in place of B; its direction 0
+//   gives Gb, its direction 1 gives Gf).
+//   dB_t = Gf_t + Gb_t,  dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T);
+//   text: G_0 = M_0 (Gf_1 + Gb_T), S_0 = M_0 B_0 / lambda, dB_0 = G_0,
+//   dA_0 = -G_0 S_0^T;
+//   dK = K (dA + dA^T) + V dB^T,  dV = K dB  (frames and text alike).
+//
+// Steps: the forward's Gram+factor and scan kernels (float32 states), then
+// element-wise kernels here and plain batched GEMMs in cuBLAS (bf16 operands
+// with float32 accumulation for the token-sized products, float32 for the
+// 128 x 128 ones), and the scan kernel twice more for the adjoints.
+#include <cublas_v2.h>
+
+#include <mutex>
+
+#include "sm100.cuh"
+#include "vda_internal.cuh"
+
+namespace vda {
+namespace {
+
+constexpr int kD = 128;
+constexpr size_t kMat = (size_t)kD * kD;   // elements of one 128 x 128 matrix
+
+__device__ __forceinline__ float sigmoid_f(float g) { return 1.f / (1.f + __expf(-g)); }
+
+// S = bf16(S^f + S^b), element-wise over `count` floats.
+__global__ void sum_states_kernel(const float* __restrict__ SF, const float* __restrict__ SB,
+                                  __nv_bfloat16* __restrict__ S, size_t count) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
+    S[i] = __float2bfloat16_rn(SF[i] + SB[i]);
+}
+
+// P (in place) -> dP = dO * s; dG = dO * P * s (1 - s).
+__global__ void gate_backward_kernel(__nv_bfloat16* __restrict__ P, const __nv_bfloat16* __restrict__ G,
+                                     const __nv_bfloat16* __restrict__ dO, __nv_bfloat16* __restrict__ dG,
+                                     size_t count) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x) {
+    const float s = sigmoid_f(__bfloat162float(G[i]));
+    const float d = __bfloat162float(dO[i]);
+    const float p = __bfloat162float(P[i]);
+    dG[i] = __float2bfloat16_rn(d * p * s * (1.f - s));
+    P[i] = __float2bfloat16_rn(d * s);
+  }
+}
+
+// One slot's right-hand operands of the Gram backward: W1 = dA + dA^T and
+// dB = Gf + Gb (or the text's dA_0 and G_0 with the second input null), both
+// bf16, row-major.  One CTA per slot, 256 threads.
+__global__ void slot_operands_kernel(const float* __restrict__ dA, const float* __restrict__ Gf,
+                                     const float* __restrict__ Gb, __nv_bfloat16* __restrict__ W1,
+                                     __nv_bfloat16* __restrict__ dBout, size_t in_stride, size_t out_stride) {
+  const float* a = dA + blockIdx.x * in_stride;
+  const float* f = Gf + blockIdx.x * in_stride;
+  const float* b = Gb ? Gb + blockIdx.x * in_stride : nullptr;
+  __nv_bfloat16* w = W1 + blockIdx.x * out_stride;
+  __nv_bfloat16* db = dBout + blockIdx.x * out_stride;
+  for (int e = threadIdx.x; e < kD * kD; e += blockDim.x) {
+    const int r = e / kD, c = e % kD;
+    w[e] = __float2bfloat16_rn(a[e] + a[c * kD + r]);
+    db[e] = __float2bfloat16_rn(b ? f[e] + b[e] : f[e]);
+  }
+}
+
+// M_0 (fp32, row-major) from the bf16 hi/lo operand image of each head's
+// text slot, and X_0 = Gf_1 + Gb_T.  One CTA per head.
+__global__ void text_inputs_kernel(const uint8_t* __restrict__ Mimg, const float* __restrict__ Gf,
+                                   const float* __restrict__ Gb, float* __restrict__ M0, float* __restrict__ X0,
+                                   int T) {
+  const int bh = blockIdx.x;
+  const uint8_t* img = Mimg + (size_t)bh * (T + 1) * 65536;   // the text slot
+  const float* gf1 = Gf + ((size_t)bh * T + 0) * kMat;
+  const float* gbT = Gb + ((size_t)bh * T + (T - 1)) * kMat;
+  for (int e = threadIdx.x; e < kD * kD; e += blockDim.x) {
+    const int r = e / kD, c = e % kD;
+    const int chunk = c / 8;
+    const uint32_t off = (chunk / 8) * 16384u + sm100::sw128(r, chunk % 8) + (c % 8) * 2;
+    const float hi = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(img + off));
+    const float lo = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(img + 32768 + off));
+    M0[(size_t)bh * kMat + e] = hi + lo;
+    X0[(size_t)bh * kMat + e] = gf1[e] + gbT[e];
+  }
+}
+
+// Per device, created on first use and kept until exit: the cuBLAS handle.
+struct Blas {
+  std::mutex mu;
+  cublasHandle_t h = nullptr;
+};
+constexpr int kMaxDevices = 64;
+Blas g_blas[kMaxDevices];
+
+int grid_for(size_t count) {
+  size_t b = (count + 255) / 256;
+  return (int)(b > 148 * 16 ? 148 * 16 : (b ? b : 1));
+}
+
+// Row-major C[m x n] = op(A) op(B) for a batch, through cuBLAS's column-major
+// convention (C^T = op(B)^T op(A)^T).  ta / tb: the row-major operand is used
+// transposed.  Types: bf16 operands with float32 accumulation (C bf16 or
+// float32), or float32 throughout.
+cublasStatus_t gemm_rm(cublasHandle_t h, bool ta, bool tb, int m, int n, int k, float alpha, const void* A,
+                       cudaDataType at, int lda, long long sa, const void* B, cudaDataType bt, int ldb,
+                       long long sb, float beta, void* C, cudaDataType ct, int ldc, long long sc, int batch) {
+  return cublasGemmStridedBatchedEx(h, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, n, m, k,
+                                    &alpha, B, bt, ldb, sb, A, at, lda, sa, &beta, C, ct, ldc, sc, batch,
+                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+}
+
+struct BwdLayout {
+  Layout fwd;
+  size_t SF32, SB32, Sb, P, E, Gf, Gb, dA, W, M0, X0, G0, S0, dA0, total;
+};
+
+BwdLayout make_bwd_layout(const vda_problem& p) {
+  BwdLayout L;
+  L.fwd = make_layout(p);
+  const size_t bh = (size_t)p.B * p.H, frames = bh * p.T, slots = bh * (p.T + 1);
+  size_t off = L.fwd.total;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 256); return o; };
+  L.SF32 = take(frames * kMat * 4);
+  L.SB32 = take(frames * kMat * 4);
+  L.Sb = take(frames * kMat * 2);
+  L.P = take(frames * (size_t)p.n * kD * 2);
+  L.E = take(slots * kMat * 4);
+  L.Gf = take(frames * kMat * 4);
+  L.Gb = take(frames * kMat * 4);
+  L.dA = take(frames * kMat * 4);
+  L.W = take(slots * 2 * kMat * 2);       // per slot: W1 | dB, bf16
+  L.M0 = take(bh * kMat * 4);
+  L.X0 = take(bh * kMat * 4);
+  L.G0 = take(bh * kMat * 4);
+  L.S0 = take(bh * kMat * 4);
+  L.dA0 = take(bh * kMat * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(const vda_problem& p) { return make_bwd_layout(p).total; }
+
+cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                         const __nv_bfloat16* V, const __nv_bfloat16* G, const __nv_bfloat16* Kt,
+                         const __nv_bfloat16* Vt, const __nv_bfloat16* dO, __nv_bfloat16* dQ, __nv_bfloat16* dK,
+                         __nv_bfloat16* dV, __nv_bfloat16* dG, __nv_bfloat16* dKt, __nv_bfloat16* dVt, char* ws,
+                         cudaStream_t st, const char** where) {
+  const BwdLayout L = make_bwd_layout(p);
+  const int BH = p.B * p.H, T = p.T, n = p.n, frames = BH * T;
+  const size_t slot_stride = (size_t)(T + 1) * kMat;   // elements between a head's slot blocks
+  unsigned* err = reinterpret_cast<unsigned*>(ws + L.fwd.err);
+  float* M = reinterpret_cast<float*>(ws + L.fwd.M);
+  float* Bm = reinterpret_cast<float*>(ws + L.fwd.C);
+  __nv_bfloat16* SFb = reinterpret_cast<__nv_bfloat16*>(ws + L.fwd.SF);
+  __nv_bfloat16* SBb = reinterpret_cast<__nv_bfloat16*>(ws + L.fwd.SB);
+  float* SF32 = reinterpret_cast<float*>(ws + L.SF32);
+  float* SB32 = reinterpret_cast<float*>(ws + L.SB32);
+  __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(ws + L.Sb);
+  __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(ws + L.P);
+  float* E = reinterpret_cast<float*>(ws + L.E);
+  float* Gf = reinterpret_cast<float*>(ws + L.Gf);
+  float* Gb = reinterpret_cast<float*>(ws + L.Gb);
+  float* dA = reinterpret_cast<float*>(ws + L.dA);
+  __nv_bfloat16* W = reinterpret_cast<__nv_bfloat16*>(ws + L.W);
+  float* M0 = reinterpret_cast<float*>(ws + L.M0);
+  float* X0 = reinterpret_cast<float*>(ws + L.X0);
+  float* G0 = reinterpret_cast<float*>(ws + L.G0);
+  float* S0 = reinterpret_cast<float*>(ws + L.S0);
+  float* dA0 = reinterpret_cast<float*>(ws + L.dA0);
+  const cudaDataType bf = CUDA_R_16BF, f32 = CUDA_R_32F;
+  cudaError_t e;
+#define VDA_TRY(expr, what)                 \
+  if ((e = (expr)) != cudaSuccess) {        \
+    *where = what;                          \
+    return e;                               \
+  }
+#define VDA_BLAS(expr, what)                            \
+  if ((expr) != CUBLAS_STATUS_SUCCESS) {                \
+    *where = what;                                      \
+    return cudaErrorUnknown;                            \
+  }
+
+  int dev = 0;
+  VDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  Blas& bl = g_blas[dev];
+  std::lock_guard<std::mutex> lock(bl.mu);
+  if (!bl.h) VDA_BLAS(cublasCreate(&bl.h), "cublasCreate");
+  cublasHandle_t h = bl.h;
+  VDA_BLAS(cublasSetStream(h, st), "cublasSetStream");
+  VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
+
+  // 1. The forward's M_t, B_t and float32 states.
+  VDA_TRY(cudaMemsetAsync(err, 0, 256, st), "clearing the error word");
+  VDA_TRY(launch_gramfactor_tc(p, K, V, Kt, Vt, M, Bm, err, st), "gram+factor launch");
+  VDA_TRY(launch_scan_tc(p, M, Bm, SFb, SBb, SF32, SB32, err, st), "scan launch");
+
+  // 2. The readout's gradients: P = Q S, then dP, dG, dQ = dP S^T, E = Q^T dP.
+  const size_t sc = (size_t)frames * kMat;
+  sum_states_kernel<<<grid_for(sc), 256, 0, st>>>(SF32, SB32, Sb, sc);
+  VDA_TRY(cudaGetLastError(), "sum_states launch");
+  const long long ntok = (long long)n * kD;
+  VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, Q, bf, kD, ntok, Sb, bf, kD, kMat, 0.f, P, bf, kD, ntok, frames),
+           "P = Q S");
+  const size_t pc = (size_t)frames * n * kD;
+  gate_backward_kernel<<<grid_for(pc), 256, 0, st>>>(P, G, dO, dG, pc);
+  VDA_TRY(cudaGetLastError(), "gate_backward launch");
+  VDA_BLAS(gemm_rm(h, false, true, n, kD, kD, 1.f, P, bf, kD, ntok, Sb, bf, kD, kMat, 0.f, dQ, bf, kD, ntok, frames),
+           "dQ = dP S^T");
+  // E in the slot layout the scan reads (B_t's), the text slots zero.
+  VDA_TRY(cudaMemset2DAsync(E, slot_stride * 4, 0, kMat * 4, BH, st), "clearing E's text slots");
+  for (int b = 0; b < BH; ++b) {
+    const size_t f0 = (size_t)b * T;
+    VDA_BLAS(gemm_rm(h, true, false, kD, kD, n, 1.f, Q + f0 * ntok, bf, kD, ntok, P + f0 * ntok, bf, kD, ntok,
+                     0.f, E + (size_t)b * slot_stride + kMat, f32, kD, kMat, T),
+             "E = Q^T dP");
+  }
+
+  // 3. The scans' adjoints: the scan kernel with E for B; direction 0 gives
+  //    Gb (forward in time), direction 1 gives Gf.
+  VDA_TRY(launch_scan_tc(p, M, E, SFb, SBb, Gb, Gf, err, st), "adjoint scan launch");
+
+  // 4. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T), then W1 = dA + dA^T and dB.
+  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, Gf, f32, kD, kMat, SF32, f32, kD, kMat, 0.f, dA, f32, kD, kMat,
+                   frames), "dA (forward part)");
+  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, Gb, f32, kD, kMat, SB32, f32, kD, kMat, 1.f, dA, f32, kD, kMat,
+                   frames), "dA (backward part)");
+  for (int b = 0; b < BH; ++b) {
+    const size_t f0 = (size_t)b * T;
+    __nv_bfloat16* w = W + ((size_t)b * (T + 1) + 1) * 2 * kMat;   // frame slots of head b
+    slot_operands_kernel<<<T, 256, 0, st>>>(dA + f0 * kMat, Gf + f0 * kMat, Gb + f0 * kMat, w, w + kMat, kMat,
+                                            2 * kMat);
+  }
+  VDA_TRY(cudaGetLastError(), "slot_operands launch");
+  // The text: G_0 = M_0 (Gf_1 + Gb_T), S_0 = M_0 B_0 / lambda, dA_0 = -G_0 S_0^T.
+  if (p.n_txt > 0) {
+    text_inputs_kernel<<<BH, 256, 0, st>>>(reinterpret_cast<const uint8_t*>(M), Gf, Gb, M0, X0, T);
+    VDA_TRY(cudaGetLastError(), "text_inputs launch");
+    VDA_BLAS(gemm_rm(h, false, false, kD, kD, kD, 1.f, M0, f32, kD, kMat, X0, f32, kD, kMat, 0.f, G0, f32, kD, kMat,
+                     BH), "G_0");
+    VDA_BLAS(gemm_rm(h, false, false, kD, kD, kD, 1.f / p.lambda, M0, f32, kD, kMat, Bm, f32, kD,
+                     (long long)slot_stride, 0.f, S0, f32, kD, kMat, BH), "S_0");
+    VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, G0, f32, kD, kMat, S0, f32, kD, kMat, 0.f, dA0, f32, kD, kMat,
+                     BH), "dA_0");
+    slot_operands_kernel<<<BH, 256, 0, st>>>(dA0, G0, nullptr, W, W + kMat, kMat, (T + 1) * 2 * kMat);
+    VDA_TRY(cudaGetLastError(), "slot_operands launch");
+  }
+
+  // 5. dK = K W1 + V dB^T, dV = K dB, for the frames and the text.
+  for (int b = 0; b < BH; ++b) {
+    const size_t f0 = (size_t)b * T;
+    const __nv_bfloat16* w = W + ((size_t)b * (T + 1) + 1) * 2 * kMat;
+    const long long ws2 = 2 * (long long)kMat;
+    VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K + f0 * ntok, bf, kD, ntok, w, bf, kD, ws2, 0.f,
+                     dK + f0 * ntok, bf, kD, ntok, T), "dK = K W1");
+    VDA_BLAS(gemm_rm(h, false, true, n, kD, kD, 1.f, V + f0 * ntok, bf, kD, ntok, w + kMat, bf, kD, ws2, 1.f,
+                     dK + f0 * ntok, bf, kD, ntok, T), "dK += V dB^T");
+    VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K + f0 * ntok, bf, kD, ntok, w + kMat, bf, kD, ws2, 0.f,
+                     dV + f0 * ntok, bf, kD, ntok, T), "dV = K dB");
+  }
+  if (p.n_txt > 0) {
+    const long long nt = (long long)p.n_txt * kD;
+    const long long wst = (long long)(T + 1) * 2 * kMat;
+    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, W, bf, kD, wst, 0.f, dKt, bf, kD, nt, BH),
+             "dK_txt = K_txt W1");
+    VDA_BLAS(gemm_rm(h, false, true, p.n_txt, kD, kD, 1.f, Vt, bf, kD, nt, W + kMat, bf, kD, wst, 1.f, dKt, bf, kD,
+                     nt, BH), "dK_txt += V_txt dB^T");
+    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, W + kMat, bf, kD, wst, 0.f, dVt, bf, kD,
+                     nt, BH), "dV_txt = K_txt dB");
+  }
+#undef VDA_TRY
+#undef VDA_BLAS
+  return cudaSuccess;
+}
+
+}  // namespace vda

@@ -82,6 +82,15 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
                               const __nv_bfloat16* SF, const __nv_bfloat16* SB, __nv_bfloat16* O,
                               unsigned* err, cudaStream_t st);
 
+// Backward (vda_backward.cu): bf16 inputs, d_k = d_v = 128.  Workspace bytes,
+// and the whole backward enqueued on `st` (on failure *where names the step).
+size_t backward_workspace_bytes(const vda_problem& p);
+cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                         const __nv_bfloat16* V, const __nv_bfloat16* G, const __nv_bfloat16* Kt,
+                         const __nv_bfloat16* Vt, const __nv_bfloat16* dO, __nv_bfloat16* dQ, __nv_bfloat16* dK,
+                         __nv_bfloat16* dV, __nv_bfloat16* dG, __nv_bfloat16* dKt, __nv_bfloat16* dVt, char* ws,
+                         cudaStream_t st, const char** where);
+
 // TMA descriptor of a [items][rows][128] bf16 tensor, boxes of 64 features x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
 bool make_bf16_rows_map(CUtensorMap* m, const void* ptr, int rows, int items, int box_rows);

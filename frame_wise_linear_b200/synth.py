@@ -31,7 +31,7 @@ import numpy as np
 
 # Stream index of every tensor; fixed so that a tensor's values do not depend
 # on which other tensors a workload draws.
-_STREAM = {"Q": 0, "K": 1, "V": 2, "G": 3, "K_txt": 4, "V_txt": 5, "U": 6, "W": 7, "E": 8}
+_STREAM = {"Q": 0, "K": 1, "V": 2, "G": 3, "K_txt": 4, "V_txt": 5, "U": 6, "W": 7, "E": 8, "dO": 9}
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
@@ -219,4 +219,36 @@ def make_inputs_torch(w: Workload | str, seed: int = 0, device="cuda", pin: bool
                 if tdt == torch.bfloat16:
                     t = t.view(torch.int16).view(torch.bfloat16)
                 out[k][b, h].copy_(t)
+    return out
+
+
+def head_grad_out(w: Workload | str, b: int, h: int, seed: int = 0) -> np.ndarray:
+    """One (b, h)'s output gradient dO for the backward, N(0, 1) of O's shape,
+    in storage form (BF16 bits as uint16, or float32); its own stream."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    x = _rng(seed, "dO", b, h).standard_normal((w.T, w.n, w.d_v), dtype=np.float32)
+    return to_bf16_bits(x) if w.dtype == DTYPE_BF16 else x
+
+
+def head_grad_out_widened(w: Workload | str, b: int, h: int, seed: int = 0) -> np.ndarray:
+    """``head_grad_out`` as the exact float64 values the device sees."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    return widen(head_grad_out(w, b, h, seed), w.dtype)
+
+
+def grad_out_torch(w: Workload | str, seed: int = 0, device="cuda"):
+    """dO for every (b, h) as a [B, H, T, n, d_v] torch tensor on `device`."""
+    import torch
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    tdt = torch.bfloat16 if w.dtype == DTYPE_BF16 else torch.float32
+    out = torch.empty((w.B, w.H, w.T, w.n, w.d_v), dtype=tdt, device=device)
+    for b in range(w.B):
+        for h in range(w.H):
+            t = torch.from_numpy(head_grad_out(w, b, h, seed))
+            if tdt == torch.bfloat16:
+                t = t.view(torch.int16).view(torch.bfloat16)
+            out[b, h].copy_(t)
     return out

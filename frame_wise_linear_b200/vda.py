@@ -39,6 +39,8 @@ SYMBOLS = (
     "vda_host_workspace_size",
     "vda_forward_host",
     "vda_forward_noalloc",
+    "vda_backward_workspace_size",
+    "vda_backward",
     "vda_sync_status",
     "vda_status_string",
     "vda_last_error",
@@ -89,6 +91,10 @@ def load(path: str | None = None):
         lib.vda_forward_timed.restype = st
         lib.vda_forward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.vda_forward_noalloc.restype = st
+        lib.vda_backward_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+        lib.vda_backward_workspace_size.restype = st
+        lib.vda_backward.argtypes = [P] + [vp] * 13 + [vp, ctypes.c_size_t, vp]
+        lib.vda_backward.restype = st
         lib.vda_sync_status.argtypes = [vp, vp]
         lib.vda_sync_status.restype = st
         lib.vda_status_string.argtypes = [st]
@@ -137,6 +143,25 @@ def vda_workspace_size(problem: vda_problem) -> int:
     out = ctypes.c_size_t(0)
     _check(load().vda_workspace_size(ctypes.byref(problem), ctypes.byref(out)), "vda_workspace_size")
     return out.value
+
+
+def vda_backward_workspace_size(problem: vda_problem) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load().vda_backward_workspace_size(ctypes.byref(problem), ctypes.byref(out)),
+           "vda_backward_workspace_size")
+    return out.value
+
+
+def vda_backward(problem, Q, K, V, G, K_txt, V_txt, dO, dQ, dK, dV, dG, dK_txt, dV_txt, workspace,
+                 stream=None, workspace_bytes=None, check=True) -> int:
+    """Gradients of sum(dO * O) into dQ, dK, dV, dG, dK_txt, dV_txt (device buffers)."""
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    s = load().vda_backward(ctypes.byref(problem), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(K_txt),
+                            _ptr(V_txt), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dG), _ptr(dK_txt),
+                            _ptr(dV_txt), _ptr(workspace), wb, _stream(stream))
+    if check:
+        _check(s, "vda_backward")
+    return s
 
 
 def vda_host_workspace_size(problem: vda_problem) -> int:

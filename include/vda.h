@@ -166,6 +166,25 @@ vda_status vda_forward_noalloc(const vda_problem* p, const void* Q, const void* 
                                const void* G, const void* K_txt, const void* V_txt, void* O,
                                void* stream);
 
+/* Backward of vda_forward: the gradients of L = sum(dO * O) with respect to
+ * Q, K, V, G, K_txt and V_txt (lambda held fixed).  The pages give the
+ * forward only; this is its exact derivative (the chain rule through the
+ * gate, the readout, both scans, the text state and the normal equations).
+ * bfloat16 inputs with d_k = d_v = 128 only (VDA_ERR_UNSUPPORTED otherwise).
+ * dO, dQ, dK, dV, dG have the shapes of O, Q, K, V, G; dK_txt, dV_txt those
+ * of K_txt, V_txt (ignored, may be NULL, when n_txt == 0); all bfloat16,
+ * device memory, 16-byte aligned, written, not accumulated into.  The call
+ * recomputes the forward's transitions and states in `workspace` (at least
+ * vda_backward_workspace_size() bytes, 256-byte aligned); its device error
+ * word is read by vda_sync_status() as for vda_forward.  Asynchronous on
+ * `stream`; the plain batched GEMMs run in cuBLAS, whose handle the library
+ * creates per device on first use and keeps until exit. */
+vda_status vda_backward_workspace_size(const vda_problem* p, size_t* bytes);
+vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, const void* V,
+                        const void* G, const void* K_txt, const void* V_txt, const void* dO,
+                        void* dQ, void* dK, void* dV, void* dG, void* dK_txt, void* dV_txt,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of
  * `workspace`: VDA_OK, VDA_ERR_NOT_SPD or VDA_ERR_TIMEOUT (first one set),
  * or VDA_ERR_CUDA if the stream reports an error.  Blocking. */
