@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end leg (default min(K, 10))")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--direction", choices=("forward", "backward"), default="forward",
+                    help="backward: time vda_backward (the gradients) instead; a separate line, not the headline")
     return ap.parse_args()
 
 
@@ -462,12 +464,94 @@ def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
     return 0
 
 
+BWD_METRIC = "VDA backward frames*heads/sec (gradients of Q, K, V, G and the text) at 768p shape; % of B200 roofline"
+
+
+def backward_roofline(w, peaks):
+    """Algorithmic work of one backward: Q, K, V, G, dO read; dQ, dK, dV, dG written (and the text's);
+    tensor flops of the Gram, P = Q S, dQ, E and the two products of dK and one of dV per token."""
+    es = 2 if w.dtype == 1 else 4
+    bh = w.B * w.H
+    frames = bh * w.T
+    tok = frames * w.n
+    nbytes = tok * (3 * w.d_k + 6 * w.d_v) * es + bh * w.n_txt * 2 * (w.d_k + w.d_v) * es
+    flops = 2.0 * tok * w.d_k * (w.d_k + w.d_v) + 2.0 * tok * 3 * w.d_k * w.d_v + 2.0 * tok * w.d_k * (w.d_k + 2 * w.d_v)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    return dict(bytes=nbytes, tensor_flops=flops, t_roof_s=max(t_hbm, t_tc), bound="hbm" if t_hbm >= t_tc else "tensor")
+
+
+def run_backward(args, w):
+    """K timed vda_backward calls on one GPU: whole-call throughput and its roofline."""
+    import torch
+    from frame_wise_linear_b200 import build as _build
+    from frame_wise_linear_b200 import synth, vda
+    if args.gpus != 1:
+        raise SystemExit("--direction backward runs on one GPU")
+    dev = torch.device("cuda", 0)
+    _build.build()
+    vda.load()
+    peaks, peaks_kind = load_peaks()
+    d = synth.make_inputs_torch(w, seed=0, device=dev)
+    dO = synth.grad_out_torch(w, seed=0, device=dev)
+    prob = vda.make_problem(**w.problem())
+    wsp = torch.empty(vda.vda_backward_workspace_size(prob), dtype=torch.uint8, device=dev)
+    txt = w.n_txt > 0
+    outs = [torch.empty_like(d[k]) for k in ("Q", "K", "V", "G")]
+    touts = [torch.empty_like(d["K_txt"]), torch.empty_like(d["V_txt"])] if txt else [None, None]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vda.vda_backward(prob, d["Q"], d["K"], d["V"], d["G"], d["K_txt"] if txt else None,
+                         d["V_txt"] if txt else None, dO, *outs, *touts, wsp, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    vda.vda_sync_status(wsp, stream=stream)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    vda.vda_sync_status(wsp, stream=stream)
+    ms_step = start.elapsed_time(end) / args.steps
+    rf = backward_roofline(w, peaks)
+    line = {
+        "metric": BWD_METRIC, "direction": "backward", "value": job_value(w.units, 1, ms_step), "unit": UNIT,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == 1 else "f32", "data": "synthetic",
+        "config": config_of(w, 1),
+        "roofline": {"kernel": "whole vda_backward call", "bound": rf["bound"],
+                     "achieved": rf["bytes"] / (ms_step / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "frac": rf["t_roof_s"] / (ms_step / 1e3), "traffic": None},
+        "roofline_path": {"t_roof_us": rf["t_roof_s"] * 1e6, "bound": rf["bound"], "bytes": rf["bytes"],
+                          "frac": rf["t_roof_s"] / (ms_step / 1e3)},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     from frame_wise_linear_b200 import synth
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.direction == "backward":
+        return run_backward(args, w)
     return run_b200(args, w)
 
 
