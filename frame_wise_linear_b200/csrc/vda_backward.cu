@@ -17,10 +17,12 @@
 //   dA_0 = -G_0 S_0^T;
 //   dK = K (dA + dA^T) + V dB^T,  dV = K dB  (frames and text alike).
 //
-// Steps: the forward's Gram+factor and scan kernels (float32 states), then
-// element-wise kernels here and plain batched GEMMs in cuBLAS (bf16 operands
-// with float32 accumulation for the token-sized products, float32 for the
-// 128 x 128 ones), and the scan kernel twice more for the adjoints.
+// Steps: the forward's Gram+factor and scan kernels (float32 states); the
+// readout's backward in one tensor-core pass over the tokens (dQ, dG, E);
+// the scan kernel once more for both adjoints; then element-wise kernels
+// here and plain batched GEMMs in cuBLAS, one call per product over all
+// frames (float32 data on TF32 tensor cores for the 128 x 128 products, bf16
+// operands with float32 accumulation for the token-sized ones).
 #include <cublas_v2.h>
 
 #include <mutex>
@@ -34,43 +36,40 @@ namespace {
 constexpr int kD = 128;
 constexpr size_t kMat = (size_t)kD * kD;   // elements of one 128 x 128 matrix
 
-__device__ __forceinline__ float sigmoid_f(float g) { return 1.f / (1.f + __expf(-g)); }
-
-// S = bf16(S^f + S^b), element-wise over `count` floats.
-__global__ void sum_states_kernel(const float* __restrict__ SF, const float* __restrict__ SB,
-                                  __nv_bfloat16* __restrict__ S, size_t count) {
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
-    S[i] = __float2bfloat16_rn(SF[i] + SB[i]);
-}
-
-// P (in place) -> dP = dO * s; dG = dO * P * s (1 - s).
-__global__ void gate_backward_kernel(__nv_bfloat16* __restrict__ P, const __nv_bfloat16* __restrict__ G,
-                                     const __nv_bfloat16* __restrict__ dO, __nv_bfloat16* __restrict__ dG,
-                                     size_t count) {
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x) {
-    const float s = sigmoid_f(__bfloat162float(G[i]));
-    const float d = __bfloat162float(dO[i]);
-    const float p = __bfloat162float(P[i]);
-    dG[i] = __float2bfloat16_rn(d * p * s * (1.f - s));
-    P[i] = __float2bfloat16_rn(d * s);
+// S = bf16(S^f + S^b), element-wise, four floats per thread and pass.
+__global__ void sum_states_kernel(const float4* __restrict__ SF, const float4* __restrict__ SB,
+                                  uint2* __restrict__ S, size_t count4) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count4; i += (size_t)gridDim.x * blockDim.x) {
+    const float4 f = SF[i], b = SB[i];
+    __nv_bfloat162 lo = __floats2bfloat162_rn(f.x + b.x, f.y + b.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(f.z + b.z, f.w + b.w);
+    S[i] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
   }
 }
 
-// One slot's right-hand operands of the Gram backward: W1 = dA + dA^T and
-// dB = Gf + Gb (or the text's dA_0 and G_0 with the second input null), both
-// bf16, row-major.  One CTA per slot, 256 threads.
-__global__ void slot_operands_kernel(const float* __restrict__ dA, const float* __restrict__ Gf,
-                                     const float* __restrict__ Gb, __nv_bfloat16* __restrict__ W1,
-                                     __nv_bfloat16* __restrict__ dBout, size_t in_stride, size_t out_stride) {
-  const float* a = dA + blockIdx.x * in_stride;
-  const float* f = Gf + blockIdx.x * in_stride;
-  const float* b = Gb ? Gb + blockIdx.x * in_stride : nullptr;
-  __nv_bfloat16* w = W1 + blockIdx.x * out_stride;
-  __nv_bfloat16* db = dBout + blockIdx.x * out_stride;
-  for (int e = threadIdx.x; e < kD * kD; e += blockDim.x) {
-    const int r = e / kD, c = e % kD;
-    w[e] = __float2bfloat16_rn(a[e] + a[c * kD + r]);
-    db[e] = __float2bfloat16_rn(b ? f[e] + b[e] : f[e]);
+// The right-hand operands of the Gram backward, per matrix m: W1 = dA + dA^T
+// and dB = Gf + Gb (Gb null: dB = Gf), bf16, row-major, written to
+// W + m * 2 * 128^2 (W1) and the 128^2 elements after it (dB).  One CTA of
+// 32 x 8 threads per 32 x 32 tile: grid (16, matrices); the transposed tile
+// goes through shared memory so every global access is coalesced.
+__global__ void operands_kernel(const float* __restrict__ dA, const float* __restrict__ Gf,
+                                const float* __restrict__ Gb, __nv_bfloat16* __restrict__ W) {
+  __shared__ float tt[32][33];
+  const size_t m = blockIdx.y;
+  const int r0 = (blockIdx.x / 4) * 32, c0 = (blockIdx.x % 4) * 32;
+  const float* a = dA + m * kMat;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) tt[ty + 8 * i][tx] = a[(size_t)(c0 + ty + 8 * i) * kD + r0 + tx];
+  __syncthreads();
+  __nv_bfloat16* w1 = W + m * 2 * kMat;
+  __nv_bfloat16* db = w1 + kMat;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty + 8 * i, c = c0 + tx;
+    const size_t e = (size_t)r * kD + c;
+    w1[e] = __float2bfloat16_rn(a[e] + tt[tx][ty + 8 * i]);
+    db[e] = __float2bfloat16_rn(Gb ? Gf[m * kMat + e] + Gb[m * kMat + e] : Gf[m * kMat + e]);
   }
 }
 
@@ -113,32 +112,36 @@ int grid_for(size_t count) {
 // float32), or float32 throughout.
 cublasStatus_t gemm_rm(cublasHandle_t h, bool ta, bool tb, int m, int n, int k, float alpha, const void* A,
                        cudaDataType at, int lda, long long sa, const void* B, cudaDataType bt, int ldb,
-                       long long sb, float beta, void* C, cudaDataType ct, int ldc, long long sc, int batch) {
+                       long long sb, float beta, void* C, cudaDataType ct, int ldc, long long sc, int batch,
+                       cublasComputeType_t ctype = CUBLAS_COMPUTE_32F) {
   return cublasGemmStridedBatchedEx(h, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, n, m, k,
-                                    &alpha, B, bt, ldb, sb, A, at, lda, sa, &beta, C, ct, ldc, sc, batch,
-                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+                                    &alpha, B, bt, ldb, sb, A, at, lda, sa, &beta, C, ct, ldc, sc, batch, ctype,
+                                    CUBLAS_GEMM_DEFAULT);
 }
 
 struct BwdLayout {
   Layout fwd;
-  size_t SF32, SB32, Sb, P, E, Gf, Gb, dA, W, M0, X0, G0, S0, dA0, total;
+  size_t SF32, SB32, Sb, E, Gf, Gb, dA, W, Wt, M0, X0, G0, S0, dA0, total;
 };
 
+// Frame-indexed blocks ([frames][128][128]) for everything after the
+// forward's, so each token-sized product is one batched GEMM; the text's
+// per-head matrices in blocks of their own.
 BwdLayout make_bwd_layout(const vda_problem& p) {
   BwdLayout L;
   L.fwd = make_layout(p);
-  const size_t bh = (size_t)p.B * p.H, frames = bh * p.T, slots = bh * (p.T + 1);
+  const size_t bh = (size_t)p.B * p.H, frames = bh * p.T;
   size_t off = L.fwd.total;
   auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 256); return o; };
   L.SF32 = take(frames * kMat * 4);
   L.SB32 = take(frames * kMat * 4);
   L.Sb = take(frames * kMat * 2);
-  L.P = take(frames * (size_t)p.n * kD * 2);
-  L.E = take(slots * kMat * 4);
+  L.E = take(frames * kMat * 4);
   L.Gf = take(frames * kMat * 4);
   L.Gb = take(frames * kMat * 4);
   L.dA = take(frames * kMat * 4);
-  L.W = take(slots * 2 * kMat * 2);       // per slot: W1 | dB, bf16
+  L.W = take(frames * 2 * kMat * 2);      // per frame: W1 | dB, bf16
+  L.Wt = take(bh * 2 * kMat * 2);         // per head, the text's
   L.M0 = take(bh * kMat * 4);
   L.X0 = take(bh * kMat * 4);
   L.G0 = take(bh * kMat * 4);
@@ -168,12 +171,12 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   float* SF32 = reinterpret_cast<float*>(ws + L.SF32);
   float* SB32 = reinterpret_cast<float*>(ws + L.SB32);
   __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(ws + L.Sb);
-  __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(ws + L.P);
   float* E = reinterpret_cast<float*>(ws + L.E);
   float* Gf = reinterpret_cast<float*>(ws + L.Gf);
   float* Gb = reinterpret_cast<float*>(ws + L.Gb);
   float* dA = reinterpret_cast<float*>(ws + L.dA);
   __nv_bfloat16* W = reinterpret_cast<__nv_bfloat16*>(ws + L.W);
+  __nv_bfloat16* Wt = reinterpret_cast<__nv_bfloat16*>(ws + L.Wt);
   float* M0 = reinterpret_cast<float*>(ws + L.M0);
   float* X0 = reinterpret_cast<float*>(ws + L.X0);
   float* G0 = reinterpret_cast<float*>(ws + L.G0);
@@ -207,77 +210,60 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   VDA_TRY(launch_gramfactor_tc(p, K, V, Kt, Vt, M, Bm, err, st), "gram+factor launch");
   VDA_TRY(launch_scan_tc(p, M, Bm, SFb, SBb, SF32, SB32, err, st), "scan launch");
 
-  // 2. The readout's gradients: P = Q S, then dP, dG, dQ = dP S^T, E = Q^T dP.
+  // 2. The readout's gradients in one pass over the tokens: P = Q S, dP,
+  //    dG, dQ = dP S^T and E = Q^T dP (vda_readout_bwd_tc.cu).
   const size_t sc = (size_t)frames * kMat;
-  sum_states_kernel<<<grid_for(sc), 256, 0, st>>>(SF32, SB32, Sb, sc);
+  sum_states_kernel<<<grid_for(sc / 4), 256, 0, st>>>(reinterpret_cast<const float4*>(SF32),
+                                                      reinterpret_cast<const float4*>(SB32),
+                                                      reinterpret_cast<uint2*>(Sb), sc / 4);
   VDA_TRY(cudaGetLastError(), "sum_states launch");
-  const long long ntok = (long long)n * kD;
-  VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, Q, bf, kD, ntok, Sb, bf, kD, kMat, 0.f, P, bf, kD, ntok, frames),
-           "P = Q S");
-  const size_t pc = (size_t)frames * n * kD;
-  gate_backward_kernel<<<grid_for(pc), 256, 0, st>>>(P, G, dO, dG, pc);
-  VDA_TRY(cudaGetLastError(), "gate_backward launch");
-  VDA_BLAS(gemm_rm(h, false, true, n, kD, kD, 1.f, P, bf, kD, ntok, Sb, bf, kD, kMat, 0.f, dQ, bf, kD, ntok, frames),
-           "dQ = dP S^T");
-  // E in the slot layout the scan reads (B_t's), the text slots zero.
-  VDA_TRY(cudaMemset2DAsync(E, slot_stride * 4, 0, kMat * 4, BH, st), "clearing E's text slots");
-  for (int b = 0; b < BH; ++b) {
-    const size_t f0 = (size_t)b * T;
-    VDA_BLAS(gemm_rm(h, true, false, kD, kD, n, 1.f, Q + f0 * ntok, bf, kD, ntok, P + f0 * ntok, bf, kD, ntok,
-                     0.f, E + (size_t)b * slot_stride + kMat, f32, kD, kMat, T),
-             "E = Q^T dP");
-  }
+  VDA_TRY(launch_readout_bwd_tc(p, Q, G, dO, Sb, dQ, dG, E, err, st), "readout backward launch");
 
-  // 3. The scans' adjoints: the scan kernel with E for B; direction 0 gives
-  //    Gb (forward in time), direction 1 gives Gf.
-  VDA_TRY(launch_scan_tc(p, M, E, SFb, SBb, Gb, Gf, err, st), "adjoint scan launch");
+  // 3. The scans' adjoints: the scan kernel with E (frame-indexed, nothing
+  //    at the text step) for B; direction 0 gives Gb (forward in time),
+  //    direction 1 gives Gf.
+  VDA_TRY(launch_scan_tc(p, M, E, SFb, SBb, Gb, Gf, err, st, /*b_frames=*/true), "adjoint scan launch");
 
-  // 4. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T), then W1 = dA + dA^T and dB.
+  // 4. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T) (float32 data, TF32 tensor
+  //    cores), then W1 = dA + dA^T and dB.
+  VDA_BLAS(cublasSetMathMode(h, CUBLAS_TF32_TENSOR_OP_MATH), "cublasSetMathMode");
   VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, Gf, f32, kD, kMat, SF32, f32, kD, kMat, 0.f, dA, f32, kD, kMat,
-                   frames), "dA (forward part)");
+                   frames, CUBLAS_COMPUTE_32F_FAST_TF32), "dA (forward part)");
   VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, Gb, f32, kD, kMat, SB32, f32, kD, kMat, 1.f, dA, f32, kD, kMat,
-                   frames), "dA (backward part)");
-  for (int b = 0; b < BH; ++b) {
-    const size_t f0 = (size_t)b * T;
-    __nv_bfloat16* w = W + ((size_t)b * (T + 1) + 1) * 2 * kMat;   // frame slots of head b
-    slot_operands_kernel<<<T, 256, 0, st>>>(dA + f0 * kMat, Gf + f0 * kMat, Gb + f0 * kMat, w, w + kMat, kMat,
-                                            2 * kMat);
-  }
-  VDA_TRY(cudaGetLastError(), "slot_operands launch");
+                   frames, CUBLAS_COMPUTE_32F_FAST_TF32), "dA (backward part)");
+  operands_kernel<<<dim3(16, frames), dim3(32, 8), 0, st>>>(dA, Gf, Gb, W);
+  VDA_TRY(cudaGetLastError(), "operands launch");
   // The text: G_0 = M_0 (Gf_1 + Gb_T), S_0 = M_0 B_0 / lambda, dA_0 = -G_0 S_0^T.
   if (p.n_txt > 0) {
     text_inputs_kernel<<<BH, 256, 0, st>>>(reinterpret_cast<const uint8_t*>(M), Gf, Gb, M0, X0, T);
     VDA_TRY(cudaGetLastError(), "text_inputs launch");
     VDA_BLAS(gemm_rm(h, false, false, kD, kD, kD, 1.f, M0, f32, kD, kMat, X0, f32, kD, kMat, 0.f, G0, f32, kD, kMat,
-                     BH), "G_0");
+                     BH, CUBLAS_COMPUTE_32F_FAST_TF32), "G_0");
     VDA_BLAS(gemm_rm(h, false, false, kD, kD, kD, 1.f / p.lambda, M0, f32, kD, kMat, Bm, f32, kD,
-                     (long long)slot_stride, 0.f, S0, f32, kD, kMat, BH), "S_0");
+                     (long long)slot_stride, 0.f, S0, f32, kD, kMat, BH, CUBLAS_COMPUTE_32F_FAST_TF32), "S_0");
     VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, G0, f32, kD, kMat, S0, f32, kD, kMat, 0.f, dA0, f32, kD, kMat,
-                     BH), "dA_0");
-    slot_operands_kernel<<<BH, 256, 0, st>>>(dA0, G0, nullptr, W, W + kMat, kMat, (T + 1) * 2 * kMat);
-    VDA_TRY(cudaGetLastError(), "slot_operands launch");
+                     BH, CUBLAS_COMPUTE_32F_FAST_TF32), "dA_0");
+    operands_kernel<<<dim3(16, BH), dim3(32, 8), 0, st>>>(dA0, G0, nullptr, Wt);
+    VDA_TRY(cudaGetLastError(), "operands launch");
   }
+  VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
 
   // 5. dK = K W1 + V dB^T, dV = K dB, for the frames and the text.
-  for (int b = 0; b < BH; ++b) {
-    const size_t f0 = (size_t)b * T;
-    const __nv_bfloat16* w = W + ((size_t)b * (T + 1) + 1) * 2 * kMat;
-    const long long ws2 = 2 * (long long)kMat;
-    VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K + f0 * ntok, bf, kD, ntok, w, bf, kD, ws2, 0.f,
-                     dK + f0 * ntok, bf, kD, ntok, T), "dK = K W1");
-    VDA_BLAS(gemm_rm(h, false, true, n, kD, kD, 1.f, V + f0 * ntok, bf, kD, ntok, w + kMat, bf, kD, ws2, 1.f,
-                     dK + f0 * ntok, bf, kD, ntok, T), "dK += V dB^T");
-    VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K + f0 * ntok, bf, kD, ntok, w + kMat, bf, kD, ws2, 0.f,
-                     dV + f0 * ntok, bf, kD, ntok, T), "dV = K dB");
-  }
+  const long long ntok = (long long)n * kD;
+  const long long w2 = 2 * (long long)kMat;
+  VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K, bf, kD, ntok, W, bf, kD, w2, 0.f, dK, bf, kD, ntok, frames),
+           "dK = K W1");
+  VDA_BLAS(gemm_rm(h, false, true, n, kD, kD, 1.f, V, bf, kD, ntok, W + kMat, bf, kD, w2, 1.f, dK, bf, kD, ntok,
+                   frames), "dK += V dB^T");
+  VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K, bf, kD, ntok, W + kMat, bf, kD, w2, 0.f, dV, bf, kD, ntok,
+                   frames), "dV = K dB");
   if (p.n_txt > 0) {
     const long long nt = (long long)p.n_txt * kD;
-    const long long wst = (long long)(T + 1) * 2 * kMat;
-    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, W, bf, kD, wst, 0.f, dKt, bf, kD, nt, BH),
+    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, Wt, bf, kD, w2, 0.f, dKt, bf, kD, nt, BH),
              "dK_txt = K_txt W1");
-    VDA_BLAS(gemm_rm(h, false, true, p.n_txt, kD, kD, 1.f, Vt, bf, kD, nt, W + kMat, bf, kD, wst, 1.f, dKt, bf, kD,
+    VDA_BLAS(gemm_rm(h, false, true, p.n_txt, kD, kD, 1.f, Vt, bf, kD, nt, Wt + kMat, bf, kD, w2, 1.f, dKt, bf, kD,
                      nt, BH), "dK_txt += V_txt dB^T");
-    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, W + kMat, bf, kD, wst, 0.f, dVt, bf, kD,
+    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, Wt + kMat, bf, kD, w2, 0.f, dVt, bf, kD,
                      nt, BH), "dV_txt = K_txt dB");
   }
 #undef VDA_TRY

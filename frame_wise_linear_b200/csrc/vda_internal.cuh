@@ -65,8 +65,11 @@ cudaError_t launch_factor(const vda_problem& p, float* M, unsigned* err, cudaStr
 // split layout above, B_t float32 in the C region.
 // S^f, S^b go to SFb, SBb as bfloat16 ([frames][d_k][d_v], the readout's
 // operand); also as float32 to SF, SB when both are non-null.
+// b_frames: Bm is [frames][128][128] (no text slots) and the text step adds
+// nothing, the form of the backward's adjoint scans.
 cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, __nv_bfloat16* SFb,
-                           __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st);
+                           __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st,
+                           bool b_frames = false);
 
 // Gram and factor in one kernel (vda_gramfactor_tc.cu): bf16 inputs,
 // d_k = d_v = 128.  Writes each slot's M_t into M as bf16 hi and lo halves
@@ -81,6 +84,13 @@ cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, c
 cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,
                               const __nv_bfloat16* SF, const __nv_bfloat16* SB, __nv_bfloat16* O,
                               unsigned* err, cudaStream_t st);
+
+// Backward of the gated readout (vda_readout_bwd_tc.cu): bf16 Q, G, dO and
+// S = S^f + S^b ([frames][128][128]); writes dQ and dG (bf16, the tokens'
+// layout) and E = Q^T dP (float32, [frames][128][128]).
+cudaError_t launch_readout_bwd_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,
+                                  const __nv_bfloat16* dO, const __nv_bfloat16* S, __nv_bfloat16* dQ,
+                                  __nv_bfloat16* dG, float* E, unsigned* err, cudaStream_t st);
 
 // Backward (vda_backward.cu): bf16 inputs, d_k = d_v = 128.  Workspace bytes,
 // and the whole backward enqueued on `st` (on failure *where names the step).

@@ -59,6 +59,7 @@ struct ScanTcParams {
   unsigned* err;
   int T;
   int f32_out;             // also write the float32 states
+  int b_frames;            // B is [frames * 128][128] with no text rows; the text step adds nothing
   float lam;
 };
 
@@ -98,6 +99,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   const int T = p.T;
   const size_t slot0 = (size_t)bh * (T + 1);
   auto slot_of = [&](int s) -> size_t { return slot0 + (s == 0 ? 0 : (dir == 0 ? s : T + 1 - s)); };
+  // First row of B_s: its slot's, or, for frame-indexed B, its frame's (the
+  // text step reads frame 1's rows and the row warps ignore them).
+  auto brow_of = [&](int s) -> size_t {
+    if (!p.b_frames) return slot_of(s) * 128;
+    const int t = s == 0 ? 1 : (dir == 0 ? s : T + 1 - s);
+    return ((size_t)bh * T + (t - 1)) * 128;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -133,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         mbar_expect_tx(&sh.b_full, kBBuf);
 #pragma unroll
         for (int b = 0; b < N / 32; ++b)
-          tma_load_2d(bbuf + b * 16384, &p.mB, &sh.b_full, c0 + 32 * b, (int)(slot_of(s) * 128), pol);
+          tma_load_2d(bbuf + b * 16384, &p.mB, &sh.b_full, c0 + 32 * b, (int)brow_of(s), pol);
       };
       auto issue_load = [&](int s) {
         const int st = s & 1;
@@ -147,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       auto prefetch = [&](int s) {
         if (blockIdx.x != 0 || s > T) return;
         bulk_prefetch_l2(p.M + slot_of(s) * (size_t)kMBytes, kMBytes);
-        bulk_prefetch_l2(p.Bm + slot_of(s) * 128 * 128, 128 * 128 * 4);
+        bulk_prefetch_l2(p.Bm + brow_of(s) * 128, 128 * 128 * 4);
       };
       tma_prefetch_desc(&p.mB);
       griddep_wait();                // M_t and B_t come from the previous kernel
@@ -271,12 +279,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         bv[4 * q + 3] = b4.w;
       }
       mbar_arrive(&sh.b_empty);
+      const bool no_b = p.b_frames && s == 0;   // frame-indexed B: nothing at the text step
 #pragma unroll
       for (int q = 0; q < kCols / 8; ++q) {
         float h[8], l[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float x = fmaf(bv[8 * q + i], inv_lam, srow[8 * q + i]);
+          const float x = no_b ? srow[8 * q + i] : fmaf(bv[8 * q + i], inv_lam, srow[8 * q + i]);
           h[i] = __bfloat162float(__float2bfloat16_rn(x));
           l[i] = x - h[i];
         }
@@ -314,11 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
 }  // namespace
 
 cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm, __nv_bfloat16* SFb,
-                           __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st) {
+                           __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st,
+                           bool b_frames) {
   ScanTcParams prm;
   memset(&prm, 0, sizeof(prm));
   const int frames = p.B * p.H * p.T;
-  const long long brows = (long long)p.B * p.H * (p.T + 1) * 128;
+  const long long brows = b_frames ? (long long)frames * 128 : (long long)p.B * p.H * (p.T + 1) * 128;
+  prm.b_frames = b_frames ? 1 : 0;
   if (!make_bf16_rows_map(&prm.mSFb, SFb, 128, frames, 128) || !make_bf16_rows_map(&prm.mSBb, SBb, 128, frames, 128) ||
       !make_f32_rows_map(&prm.mB, Bm, brows, 128))
     return cudaErrorInvalidValue;
