@@ -19,10 +19,10 @@
 //
 // Steps: the forward's Gram+factor and scan kernels (float32 states); the
 // readout's backward in one tensor-core pass over the tokens (dQ, dG, E);
-// the scan kernel once more for both adjoints; then element-wise kernels
-// here and plain batched GEMMs in cuBLAS, one call per product over all
-// frames (float32 data on TF32 tensor cores for the 128 x 128 products, bf16
-// operands with float32 accumulation for the token-sized ones).
+// the scan kernel once more for both adjoints; the 128 x 128 products as
+// plain batched GEMMs in cuBLAS (float32 data on TF32 tensor cores, one call
+// per product over all frames) and element-wise kernels here; then the Gram
+// products' backward in one tensor-core pass over the tokens (dK, dV).
 #include <cublas_v2.h>
 
 #include <mutex>
@@ -182,7 +182,7 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   float* G0 = reinterpret_cast<float*>(ws + L.G0);
   float* S0 = reinterpret_cast<float*>(ws + L.S0);
   float* dA0 = reinterpret_cast<float*>(ws + L.dA0);
-  const cudaDataType bf = CUDA_R_16BF, f32 = CUDA_R_32F;
+  const cudaDataType f32 = CUDA_R_32F;
   cudaError_t e;
 #define VDA_TRY(expr, what)                 \
   if ((e = (expr)) != cudaSuccess) {        \
@@ -248,24 +248,9 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   }
   VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
 
-  // 5. dK = K W1 + V dB^T, dV = K dB, for the frames and the text.
-  const long long ntok = (long long)n * kD;
-  const long long w2 = 2 * (long long)kMat;
-  VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K, bf, kD, ntok, W, bf, kD, w2, 0.f, dK, bf, kD, ntok, frames),
-           "dK = K W1");
-  VDA_BLAS(gemm_rm(h, false, true, n, kD, kD, 1.f, V, bf, kD, ntok, W + kMat, bf, kD, w2, 1.f, dK, bf, kD, ntok,
-                   frames), "dK += V dB^T");
-  VDA_BLAS(gemm_rm(h, false, false, n, kD, kD, 1.f, K, bf, kD, ntok, W + kMat, bf, kD, w2, 0.f, dV, bf, kD, ntok,
-                   frames), "dV = K dB");
-  if (p.n_txt > 0) {
-    const long long nt = (long long)p.n_txt * kD;
-    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, Wt, bf, kD, w2, 0.f, dKt, bf, kD, nt, BH),
-             "dK_txt = K_txt W1");
-    VDA_BLAS(gemm_rm(h, false, true, p.n_txt, kD, kD, 1.f, Vt, bf, kD, nt, Wt + kMat, bf, kD, w2, 1.f, dKt, bf, kD,
-                     nt, BH), "dK_txt += V_txt dB^T");
-    VDA_BLAS(gemm_rm(h, false, false, p.n_txt, kD, kD, 1.f, Kt, bf, kD, nt, Wt + kMat, bf, kD, w2, 0.f, dVt, bf, kD,
-                     nt, BH), "dV_txt = K_txt dB");
-  }
+  // 5. dK = K W1 + V dB^T, dV = K dB, for the frames and the text, in one
+  //    pass over the tokens (vda_gram_bwd_tc.cu).
+  VDA_TRY(launch_gram_bwd_tc(p, K, V, W, Kt, Vt, Wt, dK, dV, dKt, dVt, err, st), "gram backward launch");
 #undef VDA_TRY
 #undef VDA_BLAS
   return cudaSuccess;

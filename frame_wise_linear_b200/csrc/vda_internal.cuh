@@ -92,6 +92,14 @@ cudaError_t launch_readout_bwd_tc(const vda_problem& p, const __nv_bfloat16* Q, 
                                   const __nv_bfloat16* dO, const __nv_bfloat16* S, __nv_bfloat16* dQ,
                                   __nv_bfloat16* dG, float* E, unsigned* err, cudaStream_t st);
 
+// Backward of the Gram products (vda_gram_bwd_tc.cu): dK = K W1 + V dB^T and
+// dV = K dB per frame (W: [frames][256][128] bf16, W1 rows then dB rows) and
+// per head for the text (Wt: [heads][256][128]; skipped when n_txt == 0).
+cudaError_t launch_gram_bwd_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                               const __nv_bfloat16* W, const __nv_bfloat16* Kt, const __nv_bfloat16* Vt,
+                               const __nv_bfloat16* Wt, __nv_bfloat16* dK, __nv_bfloat16* dV, __nv_bfloat16* dKt,
+                               __nv_bfloat16* dVt, unsigned* err, cudaStream_t st);
+
 // Backward (vda_backward.cu): bf16 inputs, d_k = d_v = 128.  Workspace bytes,
 // and the whole backward enqueued on `st` (on failure *where names the step).
 size_t backward_workspace_bytes(const vda_problem& p);

@@ -13,7 +13,9 @@
 // the same TMEM buffer and E += Q^T dP (A = Q MN-major, B = dP MN-major)
 // accumulates over the frame's tiles in a TMEM block of its own.  dQ leaves
 // from registers by direct stores (shared memory holds the S operand and two
-// stages of Q, G and dO: 224 KB); E leaves the same way once per frame.
+// stages of Q, G and dO: 224 KB), after a shuffle transpose inside 8-lane
+// groups so each store instruction writes four whole 128-byte row segments;
+// E leaves the same way once per frame.
 //
 // Design (persistent, one CTA per SM, 10 warps); each CTA takes a contiguous
 // range of whole frames, so E needs no cross-CTA reduction:
@@ -76,6 +78,28 @@ __device__ __forceinline__ void set_abort(Shared& sh, unsigned* err) {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 8 x 8 transpose of 16-byte chunks across the 8 lanes of a group (j = lane
+// % 8): chunk k of lane j becomes chunk j of lane k.  Then the group's 8
+// lanes hold one 128-byte row segment per chunk index, so a store writes
+// whole lines (three butterfly stages of shuffles).
+__device__ __forceinline__ void transpose8(uint4 (&x)[8], int j) {
+#pragma unroll
+  for (int s = 1; s < 8; s <<= 1) {
+    const bool hi = (j & s) != 0;
+#pragma unroll
+    for (int k0 = 0; k0 < 8; ++k0) {
+      if (k0 & s) continue;
+      const int k1 = k0 | s;
+      uint4 t = hi ? x[k0] : x[k1];
+      t.x = __shfl_xor_sync(0xffffffffu, t.x, s);
+      t.y = __shfl_xor_sync(0xffffffffu, t.y, s);
+      t.z = __shfl_xor_sync(0xffffffffu, t.z, s);
+      t.w = __shfl_xor_sync(0xffffffffu, t.w, s);
+      if (hi) x[k0] = t; else x[k1] = t;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __grid_constant__ ReadoutBwdParams p) {
@@ -309,23 +333,28 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
       if (named_bar_or(1 + half, 128, !ok)) return false;
       tc_fence_after();
       const uint32_t taddr = tmem + tb * 128 + half * 64 + lane_off;
-      const bool valid = y + row < p.n;
-      __nv_bfloat16* dst = p.dQ + ((size_t)u * p.n + (valid ? y + row : 0)) * 128 + half * 64;
-#pragma unroll 1
+      // Row `row`'s 64 columns as 8 chunks, transposed across 8-lane groups:
+      // chunk k of lane (g, j) is then chunk j of row 8 g + k of the quarter.
+      uint4 ch[8];
+#pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(taddr + c * 32, r);
         tmem_ld_wait();
-        if (valid) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 v = make_uint4(pack_bf16(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
-                                       pack_bf16(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-                                       pack_bf16(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-                                       pack_bf16(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
-            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * q) = v;
-          }
-        }
+        for (int q = 0; q < 4; ++q)
+          ch[c * 4 + q] = make_uint4(pack_bf16(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                                     pack_bf16(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                                     pack_bf16(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                                     pack_bf16(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+      }
+      transpose8(ch, lane & 7);
+      const int r0 = quarter * 32 + 8 * (lane >> 3);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int tr = y + r0 + k;             // token row; rows past n skipped
+        if (tr < p.n)
+          *reinterpret_cast<uint4*>(p.dQ + ((size_t)u * p.n + tr) * 128 + half * 64 + (lane & 7) * 8) = ch[k];
       }
       tc_fence_before();
       mbar_arrive(&sh.t_empty[tb]);
@@ -334,15 +363,20 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
     // E_t of frame u (complete once the frame's last dQ is): row = d_k index.
     auto drain_e = [&](int u) {
       const uint32_t taddr = tmem + kECol + half * 64 + lane_off;
-      float* dst = p.E + ((size_t)u * 128 + row) * 128 + half * 64;
-#pragma unroll 1
+      const int r0 = quarter * 32 + 8 * (lane >> 3);
+#pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(taddr + c * 32, r);
         tmem_ld_wait();
+        uint4 ch[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4*>(dst + c * 32 + 4 * q) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        for (int q = 0; q < 8; ++q) ch[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        transpose8(ch, lane & 7);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(p.E + ((size_t)u * 128 + r0 + k) * 128 + half * 64 + c * 32 + (lane & 7) * 4) =
+              ch[k];
       }
       tc_fence_before();
       mbar_arrive(&sh.e_empty);
