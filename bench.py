@@ -501,9 +501,28 @@ def run_backward(args, w):
     touts = [torch.empty_like(d["K_txt"]), torch.empty_like(d["V_txt"])] if txt else [None, None]
     stream = torch.cuda.current_stream(dev)
 
+    ins = (prob, d["Q"], d["K"], d["V"], d["G"], d["K_txt"] if txt else None, d["V_txt"] if txt else None)
+    O = torch.empty_like(d["G"])
+
     def step():
-        vda.vda_backward(prob, d["Q"], d["K"], d["V"], d["G"], d["K_txt"] if txt else None,
-                         d["V_txt"] if txt else None, dO, *outs, *touts, wsp, stream=stream)
+        vda.vda_backward(*ins, dO, *outs, *touts, wsp, stream=stream)
+
+    def fwd():
+        vda.vda_forward(*ins, O, wsp, stream=stream)
+
+    def step_ff():
+        vda.vda_backward_from_forward(*ins, dO, *outs, *touts, wsp, stream=stream)
+
+    def timed(fn, k):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(k):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / k
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -523,9 +542,23 @@ def run_backward(args, w):
         step()
     end.record(stream)
     torch.cuda.synchronize(dev)
+    ms_step = start.elapsed_time(end) / args.steps
+    # The backward on the state a forward call left in the workspace (a
+    # training step's form), and the whole forward + backward step.
+    fwd()
+    for _ in range(max(args.warmup, 3)):
+        step_ff()
+    ms_ff = timed(step_ff, args.steps)
+
+    def train():
+        fwd()
+        step_ff()
+
+    for _ in range(max(args.warmup, 3)):
+        train()
+    ms_train = timed(train, args.steps)
     clocks = sampler.stop()
     vda.vda_sync_status(wsp, stream=stream)
-    ms_step = start.elapsed_time(end) / args.steps
     rf = backward_roofline(w, peaks)
     line = {
         "metric": BWD_METRIC, "direction": "backward", "value": job_value(w.units, 1, ms_step), "unit": UNIT,
@@ -538,6 +571,10 @@ def run_backward(args, w):
                      "frac": rf["t_roof_s"] / (ms_step / 1e3), "traffic": None},
         "roofline_path": {"t_roof_us": rf["t_roof_s"] * 1e6, "bound": rf["bound"], "bytes": rf["bytes"],
                           "frac": rf["t_roof_s"] / (ms_step / 1e3)},
+        "from_forward": {"call": "vda_backward_from_forward after vda_forward (no recompute)", "ms_per_call": ms_ff,
+                         "value": job_value(w.units, 1, ms_ff), "frac": rf["t_roof_s"] / (ms_ff / 1e3)},
+        "train_step": {"calls": "vda_forward + vda_backward_from_forward", "ms_per_step": ms_train,
+                       "value": job_value(w.units, 1, ms_train)},
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

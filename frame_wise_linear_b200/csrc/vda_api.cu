@@ -283,10 +283,12 @@ vda_status vda_backward_workspace_size(const vda_problem* p, size_t* bytes) {
   return VDA_OK;
 }
 
-vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, const void* V, const void* G,
-                        const void* K_txt, const void* V_txt, const void* dO, void* dQ, void* dK, void* dV,
-                        void* dG, void* dK_txt, void* dV_txt, void* workspace, size_t workspace_bytes,
-                        void* stream) {
+namespace {
+
+vda_status backward_impl(const vda_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                         const void* K_txt, const void* V_txt, const void* dO, void* dQ, void* dK, void* dV,
+                         void* dG, void* dK_txt, void* dV_txt, void* workspace, size_t workspace_bytes, void* stream,
+                         bool from_forward) {
   size_t need = 0;
   vda_status s = vda_backward_workspace_size(p, &need);
   if (s != VDA_OK) return s;
@@ -311,9 +313,27 @@ vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, cons
                                     static_cast<const bf*>(dO), static_cast<bf*>(dQ), static_cast<bf*>(dK),
                                     static_cast<bf*>(dV), static_cast<bf*>(dG), static_cast<bf*>(dK_txt),
                                     static_cast<bf*>(dV_txt), static_cast<char*>(workspace),
-                                    static_cast<cudaStream_t>(stream), &where);
+                                    static_cast<cudaStream_t>(stream), &where, from_forward);
   if (e != cudaSuccess) return cuda_fail(e, where);
   return VDA_OK;
+}
+
+}  // namespace
+
+vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                        const void* K_txt, const void* V_txt, const void* dO, void* dQ, void* dK, void* dV,
+                        void* dG, void* dK_txt, void* dV_txt, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return backward_impl(p, Q, K, V, G, K_txt, V_txt, dO, dQ, dK, dV, dG, dK_txt, dV_txt, workspace, workspace_bytes,
+                       stream, false);
+}
+
+vda_status vda_backward_from_forward(const vda_problem* p, const void* Q, const void* K, const void* V,
+                                     const void* G, const void* K_txt, const void* V_txt, const void* dO, void* dQ,
+                                     void* dK, void* dV, void* dG, void* dK_txt, void* dV_txt, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  return backward_impl(p, Q, K, V, G, K_txt, V_txt, dO, dQ, dK, dV, dG, dK_txt, dV_txt, workspace, workspace_bytes,
+                       stream, true);
 }
 
 vda_status vda_sync_status(void* workspace, void* stream) {

@@ -17,11 +17,13 @@
 //   dA_0 = -G_0 S_0^T;
 //   dK = K (dA + dA^T) + V dB^T,  dV = K dB  (frames and text alike).
 //
-// Steps: the forward's Gram+factor and scan kernels (float32 states); the
+// Steps: the forward's Gram+factor and scan kernels (bf16 states), unless a
+// vda_forward call has just left them in the workspace; the
 // readout's backward in one tensor-core pass over the tokens (dQ, dG, E);
 // the scan kernel once more for both adjoints; the 128 x 128 products as
-// plain batched GEMMs in cuBLAS (float32 data on TF32 tensor cores, one call
-// per product over all frames) and element-wise kernels here; then the Gram
+// plain batched GEMMs in cuBLAS (one call per product over all frames: bf16
+// adjoints and states for dA, float32 data on TF32 tensor cores for the
+// text's) and element-wise kernels here; then the Gram
 // products' backward in one tensor-core pass over the tokens (dK, dV).
 #include <cublas_v2.h>
 
@@ -36,14 +38,22 @@ namespace {
 constexpr int kD = 128;
 constexpr size_t kMat = (size_t)kD * kD;   // elements of one 128 x 128 matrix
 
-// S = bf16(S^f + S^b), element-wise, four floats per thread and pass.
-__global__ void sum_states_kernel(const float4* __restrict__ SF, const float4* __restrict__ SB,
-                                  uint2* __restrict__ S, size_t count4) {
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count4; i += (size_t)gridDim.x * blockDim.x) {
-    const float4 f = SF[i], b = SB[i];
-    __nv_bfloat162 lo = __floats2bfloat162_rn(f.x + b.x, f.y + b.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(f.z + b.z, f.w + b.w);
-    S[i] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+// S = bf16(S^f + S^b) from the bf16 states, eight elements per thread and
+// pass (16-byte accesses).
+__global__ void sum_states_kernel(const uint4* __restrict__ SF, const uint4* __restrict__ SB, uint4* __restrict__ S,
+                                  size_t count8) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count8; i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 f = SF[i], b = SB[i];
+    const __nv_bfloat162* f2 = reinterpret_cast<const __nv_bfloat162*>(&f);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+    uint4 o;
+    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 x = __bfloat1622float2(f2[j]), y = __bfloat1622float2(b2[j]);
+      o2[j] = __floats2bfloat162_rn(x.x + y.x, x.y + y.y);
+    }
+    S[i] = o;
   }
 }
 
@@ -121,24 +131,25 @@ cublasStatus_t gemm_rm(cublasHandle_t h, bool ta, bool tb, int m, int n, int k, 
 
 struct BwdLayout {
   Layout fwd;
-  size_t SF32, SB32, Sb, E, Gf, Gb, dA, W, Wt, M0, X0, G0, S0, dA0, total;
+  size_t Sb, E, Gf, Gb, GfB, GbB, dA, W, Wt, M0, X0, G0, S0, dA0, total;
 };
 
-// Frame-indexed blocks ([frames][128][128]) for everything after the
-// forward's, so each token-sized product is one batched GEMM; the text's
-// per-head matrices in blocks of their own.
+// After the forward's regions (whose M_t, B_t and bf16 states a preceding
+// vda_forward leaves in place): frame-indexed blocks ([frames][128][128]),
+// so each product is one batched call; the text's per-head matrices in
+// blocks of their own.
 BwdLayout make_bwd_layout(const vda_problem& p) {
   BwdLayout L;
   L.fwd = make_layout(p);
   const size_t bh = (size_t)p.B * p.H, frames = bh * p.T;
   size_t off = L.fwd.total;
   auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 256); return o; };
-  L.SF32 = take(frames * kMat * 4);
-  L.SB32 = take(frames * kMat * 4);
   L.Sb = take(frames * kMat * 2);
   L.E = take(frames * kMat * 4);
   L.Gf = take(frames * kMat * 4);
   L.Gb = take(frames * kMat * 4);
+  L.GfB = take(frames * kMat * 2);        // the adjoints as bf16, the dA products' operands
+  L.GbB = take(frames * kMat * 2);
   L.dA = take(frames * kMat * 4);
   L.W = take(frames * 2 * kMat * 2);      // per frame: W1 | dB, bf16
   L.Wt = take(bh * 2 * kMat * 2);         // per head, the text's
@@ -159,7 +170,7 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
                          const __nv_bfloat16* V, const __nv_bfloat16* G, const __nv_bfloat16* Kt,
                          const __nv_bfloat16* Vt, const __nv_bfloat16* dO, __nv_bfloat16* dQ, __nv_bfloat16* dK,
                          __nv_bfloat16* dV, __nv_bfloat16* dG, __nv_bfloat16* dKt, __nv_bfloat16* dVt, char* ws,
-                         cudaStream_t st, const char** where) {
+                         cudaStream_t st, const char** where, bool from_forward) {
   const BwdLayout L = make_bwd_layout(p);
   const int BH = p.B * p.H, T = p.T, n = p.n, frames = BH * T;
   const size_t slot_stride = (size_t)(T + 1) * kMat;   // elements between a head's slot blocks
@@ -168,12 +179,12 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   float* Bm = reinterpret_cast<float*>(ws + L.fwd.C);
   __nv_bfloat16* SFb = reinterpret_cast<__nv_bfloat16*>(ws + L.fwd.SF);
   __nv_bfloat16* SBb = reinterpret_cast<__nv_bfloat16*>(ws + L.fwd.SB);
-  float* SF32 = reinterpret_cast<float*>(ws + L.SF32);
-  float* SB32 = reinterpret_cast<float*>(ws + L.SB32);
   __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(ws + L.Sb);
   float* E = reinterpret_cast<float*>(ws + L.E);
   float* Gf = reinterpret_cast<float*>(ws + L.Gf);
   float* Gb = reinterpret_cast<float*>(ws + L.Gb);
+  __nv_bfloat16* GfB = reinterpret_cast<__nv_bfloat16*>(ws + L.GfB);
+  __nv_bfloat16* GbB = reinterpret_cast<__nv_bfloat16*>(ws + L.GbB);
   float* dA = reinterpret_cast<float*>(ws + L.dA);
   __nv_bfloat16* W = reinterpret_cast<__nv_bfloat16*>(ws + L.W);
   __nv_bfloat16* Wt = reinterpret_cast<__nv_bfloat16*>(ws + L.Wt);
@@ -182,7 +193,7 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   float* G0 = reinterpret_cast<float*>(ws + L.G0);
   float* S0 = reinterpret_cast<float*>(ws + L.S0);
   float* dA0 = reinterpret_cast<float*>(ws + L.dA0);
-  const cudaDataType f32 = CUDA_R_32F;
+  const cudaDataType bf = CUDA_R_16BF, f32 = CUDA_R_32F;
   cudaError_t e;
 #define VDA_TRY(expr, what)                 \
   if ((e = (expr)) != cudaSuccess) {        \
@@ -205,32 +216,37 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   VDA_BLAS(cublasSetStream(h, st), "cublasSetStream");
   VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
 
-  // 1. The forward's M_t, B_t and float32 states.
-  VDA_TRY(cudaMemsetAsync(err, 0, 256, st), "clearing the error word");
-  VDA_TRY(launch_gramfactor_tc(p, K, V, Kt, Vt, M, Bm, err, st), "gram+factor launch");
-  VDA_TRY(launch_scan_tc(p, M, Bm, SFb, SBb, SF32, SB32, err, st), "scan launch");
+  // 1. The forward's M_t, B_t and bf16 states: recomputed, or left in the
+  //    workspace by the vda_forward call that preceded this one (whose
+  //    error bits stay set for vda_sync_status).
+  if (!from_forward) {
+    VDA_TRY(cudaMemsetAsync(err, 0, 256, st), "clearing the error word");
+    VDA_TRY(launch_gramfactor_tc(p, K, V, Kt, Vt, M, Bm, err, st), "gram+factor launch");
+    VDA_TRY(launch_scan_tc(p, M, Bm, SFb, SBb, nullptr, nullptr, err, st), "scan launch");
+  }
 
   // 2. The readout's gradients in one pass over the tokens: P = Q S, dP,
   //    dG, dQ = dP S^T and E = Q^T dP (vda_readout_bwd_tc.cu).
   const size_t sc = (size_t)frames * kMat;
-  sum_states_kernel<<<grid_for(sc / 4), 256, 0, st>>>(reinterpret_cast<const float4*>(SF32),
-                                                      reinterpret_cast<const float4*>(SB32),
-                                                      reinterpret_cast<uint2*>(Sb), sc / 4);
+  sum_states_kernel<<<grid_for(sc / 8), 256, 0, st>>>(reinterpret_cast<const uint4*>(SFb),
+                                                      reinterpret_cast<const uint4*>(SBb),
+                                                      reinterpret_cast<uint4*>(Sb), sc / 8);
   VDA_TRY(cudaGetLastError(), "sum_states launch");
   VDA_TRY(launch_readout_bwd_tc(p, Q, G, dO, Sb, dQ, dG, E, err, st), "readout backward launch");
 
   // 3. The scans' adjoints: the scan kernel with E (frame-indexed, nothing
   //    at the text step) for B; direction 0 gives Gb (forward in time),
   //    direction 1 gives Gf.
-  VDA_TRY(launch_scan_tc(p, M, E, SFb, SBb, Gb, Gf, err, st, /*b_frames=*/true), "adjoint scan launch");
+  VDA_TRY(launch_scan_tc(p, M, E, GbB, GfB, Gb, Gf, err, st, /*b_frames=*/true), "adjoint scan launch");
 
-  // 4. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T) (float32 data, TF32 tensor
-  //    cores), then W1 = dA + dA^T and dB.
+  // 4. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T) from the bf16 adjoints and
+  //    states (float32 accumulation), then W1 = dA + dA^T and dB (from the
+  //    float32 adjoints).
+  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GfB, bf, kD, kMat, SFb, bf, kD, kMat, 0.f, dA, f32, kD, kMat,
+                   frames), "dA (forward part)");
+  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GbB, bf, kD, kMat, SBb, bf, kD, kMat, 1.f, dA, f32, kD, kMat,
+                   frames), "dA (backward part)");
   VDA_BLAS(cublasSetMathMode(h, CUBLAS_TF32_TENSOR_OP_MATH), "cublasSetMathMode");
-  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, Gf, f32, kD, kMat, SF32, f32, kD, kMat, 0.f, dA, f32, kD, kMat,
-                   frames, CUBLAS_COMPUTE_32F_FAST_TF32), "dA (forward part)");
-  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, Gb, f32, kD, kMat, SB32, f32, kD, kMat, 1.f, dA, f32, kD, kMat,
-                   frames, CUBLAS_COMPUTE_32F_FAST_TF32), "dA (backward part)");
   operands_kernel<<<dim3(16, frames), dim3(32, 8), 0, st>>>(dA, Gf, Gb, W);
   VDA_TRY(cudaGetLastError(), "operands launch");
   // The text: G_0 = M_0 (Gf_1 + Gb_T), S_0 = M_0 B_0 / lambda, dA_0 = -G_0 S_0^T.

@@ -101,13 +101,15 @@ cudaError_t launch_gram_bwd_tc(const vda_problem& p, const __nv_bfloat16* K, con
                                __nv_bfloat16* dVt, unsigned* err, cudaStream_t st);
 
 // Backward (vda_backward.cu): bf16 inputs, d_k = d_v = 128.  Workspace bytes,
-// and the whole backward enqueued on `st` (on failure *where names the step).
+// and the whole backward enqueued on `st` (on failure *where names the step);
+// from_forward: the workspace holds what a vda_forward call with the same
+// problem and inputs left there (M_t, B_t, bf16 states), not recomputed.
 size_t backward_workspace_bytes(const vda_problem& p);
 cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                          const __nv_bfloat16* V, const __nv_bfloat16* G, const __nv_bfloat16* Kt,
                          const __nv_bfloat16* Vt, const __nv_bfloat16* dO, __nv_bfloat16* dQ, __nv_bfloat16* dK,
                          __nv_bfloat16* dV, __nv_bfloat16* dG, __nv_bfloat16* dKt, __nv_bfloat16* dVt, char* ws,
-                         cudaStream_t st, const char** where);
+                         cudaStream_t st, const char** where, bool from_forward);
 
 // TMA descriptor of a [items][rows][128] bf16 tensor, boxes of 64 features x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.

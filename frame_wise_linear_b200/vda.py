@@ -41,6 +41,7 @@ SYMBOLS = (
     "vda_forward_noalloc",
     "vda_backward_workspace_size",
     "vda_backward",
+    "vda_backward_from_forward",
     "vda_sync_status",
     "vda_status_string",
     "vda_last_error",
@@ -95,6 +96,8 @@ def load(path: str | None = None):
         lib.vda_backward_workspace_size.restype = st
         lib.vda_backward.argtypes = [P] + [vp] * 13 + [vp, ctypes.c_size_t, vp]
         lib.vda_backward.restype = st
+        lib.vda_backward_from_forward.argtypes = [P] + [vp] * 13 + [vp, ctypes.c_size_t, vp]
+        lib.vda_backward_from_forward.restype = st
         lib.vda_sync_status.argtypes = [vp, vp]
         lib.vda_sync_status.restype = st
         lib.vda_status_string.argtypes = [st]
@@ -161,6 +164,18 @@ def vda_backward(problem, Q, K, V, G, K_txt, V_txt, dO, dQ, dK, dV, dG, dK_txt, 
                             _ptr(dV_txt), _ptr(workspace), wb, _stream(stream))
     if check:
         _check(s, "vda_backward")
+    return s
+
+
+def vda_backward_from_forward(problem, Q, K, V, G, K_txt, V_txt, dO, dQ, dK, dV, dG, dK_txt, dV_txt, workspace,
+                              stream=None, workspace_bytes=None, check=True) -> int:
+    """As vda_backward, reusing what a preceding vda_forward left in `workspace` (same problem and inputs)."""
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    s = load().vda_backward_from_forward(ctypes.byref(problem), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(K_txt),
+                                         _ptr(V_txt), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dG),
+                                         _ptr(dK_txt), _ptr(dV_txt), _ptr(workspace), wb, _stream(stream))
+    if check:
+        _check(s, "vda_backward_from_forward")
     return s
 
 

@@ -185,6 +185,20 @@ vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, cons
                         void* dQ, void* dK, void* dV, void* dG, void* dK_txt, void* dV_txt,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* The same gradients without recomputing the forward: `workspace` (at least
+ * vda_backward_workspace_size() bytes) must hold what a vda_forward call with
+ * the same problem and the same Q, K, V, G, K_txt, V_txt left there, enqueued
+ * before this call in stream order, with nothing written to the workspace in
+ * between (vda_forward's own workspace layout is a prefix of the backward's).
+ * The library does not check this precondition: other contents give wrong
+ * gradients, not an error.  The error word is not cleared, so a failure of
+ * that forward (VDA_ERR_NOT_SPD, VDA_ERR_TIMEOUT) still reaches
+ * vda_sync_status().  Arguments, layout and errors as for vda_backward. */
+vda_status vda_backward_from_forward(const vda_problem* p, const void* Q, const void* K, const void* V,
+                                     const void* G, const void* K_txt, const void* V_txt, const void* dO,
+                                     void* dQ, void* dK, void* dV, void* dG, void* dK_txt, void* dV_txt,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of
  * `workspace`: VDA_OK, VDA_ERR_NOT_SPD or VDA_ERR_TIMEOUT (first one set),
  * or VDA_ERR_CUDA if the stream reports an error.  Blocking. */

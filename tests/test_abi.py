@@ -146,3 +146,24 @@ def test_no_device_fails_loudly(lib):
     need = vda.vda_workspace_size(p)
     s = vda.vda_forward(p, *([ok] * 7), ok, stream=0, workspace_bytes=need, check=False)
     assert s == vda.VDA_ERR_CUDA
+
+
+@pytest.mark.skipif(_has_cuda(), reason="only meaningful where no CUDA device exists")
+@pytest.mark.parametrize("entry", ["vda_backward", "vda_backward_from_forward"])
+def test_backward_entry_points_checked_and_fail_loudly(lib, entry):
+    """Both backward entry points: bf16 only, pointer and workspace checks, then a CUDA error with no GPU."""
+    import ctypes
+    fn = getattr(vda, entry)
+    size = ctypes.c_size_t(0)
+    p32 = _p(dtype=vda.VDA_DTYPE_F32)
+    assert lib.vda_backward_workspace_size(ctypes.byref(p32), ctypes.byref(size)) == vda.VDA_ERR_UNSUPPORTED
+    p = _p()
+    need = vda.vda_backward_workspace_size(p)
+    ok = 1 << 20
+    args = [ok] * 13
+    assert fn(p32, *args, ok, stream=0, workspace_bytes=need, check=False) == vda.VDA_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[7] = 0                                  # dQ
+    assert fn(p, *bad, ok, stream=0, workspace_bytes=need, check=False) == vda.VDA_ERR_INVALID_ARG
+    assert fn(p, *args, ok, stream=0, workspace_bytes=need - 1, check=False) == vda.VDA_ERR_WORKSPACE
+    assert fn(p, *args, ok, stream=0, workspace_bytes=need, check=False) == vda.VDA_ERR_CUDA

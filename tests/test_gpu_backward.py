@@ -26,7 +26,7 @@ SMALL = {
 NAMES = ("dQ", "dK", "dV", "dG", "dK_txt", "dV_txt")
 
 
-def _run_gpu(w, seed=0):
+def _run_gpu(w, seed=0, from_forward=False, raw=False):
     import torch
     from frame_wise_linear_b200 import vda
     from vda_testutil import from_device
@@ -39,10 +39,18 @@ def _run_gpu(w, seed=0):
     txt = w.n_txt > 0
     out["dK_txt"] = torch.empty_like(d["K_txt"]) if txt else None
     out["dV_txt"] = torch.empty_like(d["V_txt"]) if txt else None
-    vda.vda_backward(prob, d["Q"], d["K"], d["V"], d["G"], d["K_txt"] if txt else None,
-                     d["V_txt"] if txt else None, dO, out["dQ"], out["dK"], out["dV"], out["dG"],
-                     out["dK_txt"], out["dV_txt"], ws)
+    args = (prob, d["Q"], d["K"], d["V"], d["G"], d["K_txt"] if txt else None, d["V_txt"] if txt else None)
+    if from_forward:
+        # The forward's own output, then the backward on what it left in the workspace.
+        O = torch.empty_like(d["G"])
+        vda.vda_forward(*args, O, ws)
+        vda.vda_backward_from_forward(*args, dO, out["dQ"], out["dK"], out["dV"], out["dG"], out["dK_txt"],
+                                      out["dV_txt"], ws)
+    else:
+        vda.vda_backward(*args, dO, out["dQ"], out["dK"], out["dV"], out["dG"], out["dK_txt"], out["dV_txt"], ws)
     vda.vda_sync_status(ws)
+    if raw:
+        return out
     return {k: (from_device(v) if v is not None else None) for k, v in out.items()}
 
 
@@ -82,3 +90,27 @@ def test_backward_768p_sampled_heads():
     got = _run_gpu(w)
     errs = _compare(w, got, [(0, 0), (0, 17)])
     assert max(errs.values()) <= BWD_TOL, errs
+
+
+@pytest.mark.parametrize("name", ["bwd_small", "bwd_no_text", "bwd_tail"])
+def test_backward_from_forward_small(name):
+    """vda_backward_from_forward after vda_forward: the oracle's gradients, and bit for bit the recomputing call's."""
+    import torch
+    w = SMALL[name]
+    got = _run_gpu(w, from_forward=True)
+    errs = _compare(w, got, [(b, h) for b in range(w.B) for h in range(w.H)])
+    assert max(errs.values()) <= BWD_TOL, errs
+    a = _run_gpu(w, raw=True)
+    b = _run_gpu(w, from_forward=True, raw=True)
+    for k in NAMES:
+        if a[k] is not None:
+            assert torch.equal(a[k], b[k]), k
+
+
+def test_backward_from_forward_768p_equals_recompute():
+    import torch
+    w = synth.WORKLOADS["768p"]
+    a = _run_gpu(w, raw=True)
+    b = _run_gpu(w, from_forward=True, raw=True)
+    for k in NAMES:
+        assert torch.equal(a[k], b[k]), k
