@@ -103,10 +103,14 @@ __global__ void text_inputs_kernel(const uint8_t* __restrict__ Mimg, const float
   }
 }
 
-// Per device, created on first use and kept until exit: the cuBLAS handle.
+// Per device, created on first use and kept until exit: the cuBLAS handle,
+// and the side stream (non-blocking) with the fork / join events of the
+// text's work.
 struct Blas {
   std::mutex mu;
   cublasHandle_t h = nullptr;
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
 };
 constexpr int kMaxDevices = 64;
 Blas g_blas[kMaxDevices];
@@ -212,6 +216,11 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   Blas& bl = g_blas[dev];
   std::lock_guard<std::mutex> lock(bl.mu);
   if (!bl.h) VDA_BLAS(cublasCreate(&bl.h), "cublasCreate");
+  if (!bl.side) {
+    VDA_TRY(cudaStreamCreateWithFlags(&bl.side, cudaStreamNonBlocking), "side stream");
+    VDA_TRY(cudaEventCreateWithFlags(&bl.fork, cudaEventDisableTiming), "fork event");
+    VDA_TRY(cudaEventCreateWithFlags(&bl.join, cudaEventDisableTiming), "join event");
+  }
   cublasHandle_t h = bl.h;
   VDA_BLAS(cublasSetStream(h, st), "cublasSetStream");
   VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
@@ -239,19 +248,16 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   //    direction 1 gives Gf.
   VDA_TRY(launch_scan_tc(p, M, E, GbB, GfB, Gb, Gf, err, st, /*b_frames=*/true), "adjoint scan launch");
 
-  // 4. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T) from the bf16 adjoints and
-  //    states (float32 accumulation), then W1 = dA + dA^T and dB (from the
-  //    float32 adjoints).
-  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GfB, bf, kD, kMat, SFb, bf, kD, kMat, 0.f, dA, f32, kD, kMat,
-                   frames), "dA (forward part)");
-  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GbB, bf, kD, kMat, SBb, bf, kD, kMat, 1.f, dA, f32, kD, kMat,
-                   frames), "dA (backward part)");
-  VDA_BLAS(cublasSetMathMode(h, CUBLAS_TF32_TENSOR_OP_MATH), "cublasSetMathMode");
-  operands_kernel<<<dim3(16, frames), dim3(32, 8), 0, st>>>(dA, Gf, Gb, W);
-  VDA_TRY(cudaGetLastError(), "operands launch");
-  // The text: G_0 = M_0 (Gf_1 + Gb_T), S_0 = M_0 B_0 / lambda, dA_0 = -G_0 S_0^T.
-  if (p.n_txt > 0) {
-    text_inputs_kernel<<<BH, 256, 0, st>>>(reinterpret_cast<const uint8_t*>(M), Gf, Gb, M0, X0, T);
+  // 4. The text's operands on the side stream (five small launches that
+  //    overlap the frames' work below): G_0 = M_0 (Gf_1 + Gb_T),
+  //    S_0 = M_0 B_0 / lambda, dA_0 = -G_0 S_0^T (TF32 tensor cores).
+  const bool text = p.n_txt > 0;
+  if (text) {
+    VDA_TRY(cudaEventRecord(bl.fork, st), "fork event");
+    VDA_TRY(cudaStreamWaitEvent(bl.side, bl.fork, 0), "fork wait");
+    VDA_BLAS(cublasSetStream(h, bl.side), "cublasSetStream");
+    VDA_BLAS(cublasSetMathMode(h, CUBLAS_TF32_TENSOR_OP_MATH), "cublasSetMathMode");
+    text_inputs_kernel<<<BH, 256, 0, bl.side>>>(reinterpret_cast<const uint8_t*>(M), Gf, Gb, M0, X0, T);
     VDA_TRY(cudaGetLastError(), "text_inputs launch");
     VDA_BLAS(gemm_rm(h, false, false, kD, kD, kD, 1.f, M0, f32, kD, kMat, X0, f32, kD, kMat, 0.f, G0, f32, kD, kMat,
                      BH, CUBLAS_COMPUTE_32F_FAST_TF32), "G_0");
@@ -259,12 +265,25 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
                      (long long)slot_stride, 0.f, S0, f32, kD, kMat, BH, CUBLAS_COMPUTE_32F_FAST_TF32), "S_0");
     VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, G0, f32, kD, kMat, S0, f32, kD, kMat, 0.f, dA0, f32, kD, kMat,
                      BH, CUBLAS_COMPUTE_32F_FAST_TF32), "dA_0");
-    operands_kernel<<<dim3(16, BH), dim3(32, 8), 0, st>>>(dA0, G0, nullptr, Wt);
+    operands_kernel<<<dim3(16, BH), dim3(32, 8), 0, bl.side>>>(dA0, G0, nullptr, Wt);
     VDA_TRY(cudaGetLastError(), "operands launch");
+    VDA_TRY(cudaEventRecord(bl.join, bl.side), "join event");
+    VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
+    VDA_BLAS(cublasSetStream(h, st), "cublasSetStream");
   }
-  VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
 
-  // 5. dK = K W1 + V dB^T, dV = K dB, for the frames and the text, in one
+  // 5. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T) from the bf16 adjoints and
+  //    states (float32 accumulation), then W1 = dA + dA^T and dB (from the
+  //    float32 adjoints).
+  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GfB, bf, kD, kMat, SFb, bf, kD, kMat, 0.f, dA, f32, kD, kMat,
+                   frames), "dA (forward part)");
+  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GbB, bf, kD, kMat, SBb, bf, kD, kMat, 1.f, dA, f32, kD, kMat,
+                   frames), "dA (backward part)");
+  operands_kernel<<<dim3(16, frames), dim3(32, 8), 0, st>>>(dA, Gf, Gb, W);
+  VDA_TRY(cudaGetLastError(), "operands launch");
+  if (text) VDA_TRY(cudaStreamWaitEvent(st, bl.join, 0), "join wait");
+
+  // 6. dK = K W1 + V dB^T, dV = K dB, for the frames and the text, in one
   //    pass over the tokens (vda_gram_bwd_tc.cu).
   VDA_TRY(launch_gram_bwd_tc(p, K, V, W, Kt, Vt, Wt, dK, dV, dKt, dVt, err, st), "gram backward launch");
 #undef VDA_TRY

@@ -178,7 +178,9 @@ vda_status vda_forward_noalloc(const vda_problem* p, const void* Q, const void* 
  * vda_backward_workspace_size() bytes, 256-byte aligned); its device error
  * word is read by vda_sync_status() as for vda_forward.  Asynchronous on
  * `stream`; the plain batched GEMMs run in cuBLAS, whose handle the library
- * creates per device on first use and keeps until exit. */
+ * creates per device on first use and keeps until exit, as it does a
+ * non-blocking side stream that the text's small steps fork onto and join
+ * back from (events) within the call. */
 vda_status vda_backward_workspace_size(const vda_problem* p, size_t* bytes);
 vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, const void* V,
                         const void* G, const void* K_txt, const void* V_txt, const void* dO,
