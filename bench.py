@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end leg (default min(K, 10))")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", choices=("bhtnd", "btnhd"), default="bhtnd",
+                    help="token tensors as [B, H, T, n, d] (default) or token-major [B, T*n, H, d]")
     ap.add_argument("--direction", choices=("forward", "backward"), default="forward",
                     help="backward: time vda_backward (the gradients) instead; a separate line, not the headline")
     return ap.parse_args()
@@ -278,10 +280,15 @@ def run_reference(args, w):
     return 0
 
 
-def config_of(w, n):
+LAYOUTS = {"bhtnd": 0, "btnhd": 1}
+LAYOUT_NAMES = {0: "[B,H,T,n,d]", 1: "[B,T*n,H,d]"}
+
+
+def config_of(w, n, layout=0):
     return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} n={w.n} d_k={w.d_k} d_v={w.d_v} "
                         f"n_txt={w.n_txt} lambda={w.lam} {'bf16' if w.dtype == 1 else 'f32'}",
             "B": w.B, "H": w.H, "T": w.T, "n": w.n, "n_txt": w.n_txt, "d": w.d_k,
+            "layout": LAYOUT_NAMES[layout],
             "parallelism": f"independent problems on {n} GPU(s), no collective",
             "l2": f"inputs larger than L2 ({input_bytes(w) / 1e9:.2f} GB read per step vs 126 MB); no flush"}
 
@@ -327,8 +334,11 @@ def run_b200(args, w):
     vda.load()
 
     peaks, peaks_kind = load_peaks()
+    layout = LAYOUTS[args.layout]
     d = synth.make_inputs_torch(w, seed=rank, device=dev)
-    prob = vda.make_problem(**w.problem())
+    if layout:
+        d = {k: synth.token_major(v) for k, v in d.items()}
+    prob = vda.make_problem(**w.problem(), layout=layout)
     wsb = vda.vda_workspace_size(prob)
     wsp = torch.empty(wsb, dtype=torch.uint8, device=dev)
     O = torch.empty_like(d["G"])
@@ -449,7 +459,7 @@ def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == 1 else "f32", "data": "synthetic",
-        "config": config_of(w, ws_n), "roofline": roof, "roofline_path": path, "e2e": e2e,
+        "config": config_of(w, ws_n, LAYOUTS[args.layout]), "roofline": roof, "roofline_path": path, "e2e": e2e,
         "clocks": clocks, "gpu_launches": vda.LAUNCHES_PER_FORWARD[w.dtype] * args.steps,
     }
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
@@ -492,9 +502,13 @@ def run_backward(args, w):
     _build.build()
     vda.load()
     peaks, peaks_kind = load_peaks()
+    layout = LAYOUTS[args.layout]
     d = synth.make_inputs_torch(w, seed=0, device=dev)
     dO = synth.grad_out_torch(w, seed=0, device=dev)
-    prob = vda.make_problem(**w.problem())
+    if layout:
+        d = {k: synth.token_major(v) for k, v in d.items()}
+        dO = synth.token_major(dO)
+    prob = vda.make_problem(**w.problem(), layout=layout)
     wsp = torch.empty(vda.vda_backward_workspace_size(prob), dtype=torch.uint8, device=dev)
     txt = w.n_txt > 0
     outs = [torch.empty_like(d[k]) for k in ("Q", "K", "V", "G")]
@@ -564,7 +578,7 @@ def run_backward(args, w):
         "metric": BWD_METRIC, "direction": "backward", "value": job_value(w.units, 1, ms_step), "unit": UNIT,
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == 1 else "f32", "data": "synthetic",
-        "config": config_of(w, 1),
+        "config": config_of(w, 1, LAYOUTS[args.layout]),
         "roofline": {"kernel": "whole vda_backward call", "bound": rf["bound"],
                      "achieved": rf["bytes"] / (ms_step / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json hbm_gbs)",

@@ -40,6 +40,10 @@ vda_status check_problem(const vda_problem* p) {
     return fail(VDA_ERR_INVALID_ARG, "lambda must be finite and > 0 (got %g)", (double)p->lambda);
   if (p->dtype != VDA_DTYPE_F32 && p->dtype != VDA_DTYPE_BF16)
     return fail(VDA_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
+  if (p->layout != VDA_LAYOUT_BHTND && p->layout != VDA_LAYOUT_BTNHD)
+    return fail(VDA_ERR_INVALID_ARG, "unknown layout %d", p->layout);
+  if (p->layout == VDA_LAYOUT_BTNHD && p->dtype != VDA_DTYPE_BF16)
+    return fail(VDA_ERR_UNSUPPORTED, "the token-major layout is supported for bfloat16 inputs only");
   if (p->dtype == VDA_DTYPE_F32) {
     if (p->d_k % 16 || p->d_v % 16 || p->d_k > 128 || p->d_v > 128)
       return fail(VDA_ERR_UNSUPPORTED,

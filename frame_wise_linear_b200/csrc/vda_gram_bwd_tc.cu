@@ -23,6 +23,7 @@
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
 #include "vda_internal.cuh"
+#include "vda_tok.cuh"
 
 namespace vda {
 namespace {
@@ -47,6 +48,7 @@ struct GramBwdParams {
   unsigned* err;
   int frames, heads, n, n_txt;
   int tpf, tpt;                   // tiles per frame, per text unit
+  TokGeom g;                      // the layout of K, V, dK, dV and the text's
 };
 
 struct Shared {
@@ -137,19 +139,24 @@ __global__ void __launch_bounds__(kThreads, 1) gram_bwd_tc_kernel(const __grid_c
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      int kv_issued = 0, w_issued = 0, cur = -1;
+      int kv_issued = 0, w_issued = 0, cur = -1, pos_unit = -1;
+      TokPos q{};
       for (int j = 0; j < J; ++j) {
         const TileRef r = tile_ref(p, t_begin + j);
+        if (r.unit != pos_unit) {
+          q = tok_pos(p.g, r.item, r.text);
+          pos_unit = r.unit;
+        }
         const int st = j & 1;
         if (!mbar_wait(&sh.kv_empty[st], ((j >> 1) & 1) ^ 1)) { set_abort(sh, p.err); break; }
         uint8_t* kv = kvbuf + st * 2 * kTile;
         const CUtensorMap* mk = r.text ? &p.mKt : &p.mK;
         const CUtensorMap* mv = r.text ? &p.mVt : &p.mV;
         mbar_expect_tx(&sh.kv_full[st], 2 * kTile);
-        tma_load_3d(kv, mk, &sh.kv_full[st], 0, r.y, r.item, pol);
-        tma_load_3d(kv + kBox, mk, &sh.kv_full[st], 64, r.y, r.item, pol);
-        tma_load_3d(kv + kTile, mv, &sh.kv_full[st], 0, r.y, r.item, pol);
-        tma_load_3d(kv + kTile + kBox, mv, &sh.kv_full[st], 64, r.y, r.item, pol);
+        tok_load(kv, mk, &sh.kv_full[st], p.g, q, 0, r.y, pol);
+        tok_load(kv + kBox, mk, &sh.kv_full[st], p.g, q, 64, r.y, pol);
+        tok_load(kv + kTile, mv, &sh.kv_full[st], p.g, q, 0, r.y, pol);
+        tok_load(kv + kTile + kBox, mv, &sh.kv_full[st], p.g, q, 64, r.y, pol);
         ++kv_issued;
         if (r.unit != cur) {
           // The unit's W1 | dB, once the previous unit's MMAs are done with the buffer.
@@ -235,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) gram_bwd_tc_kernel(const __grid_c
       if (named_bar_or(1 + half, 128, !ok)) break;   // one decision per half
       tc_fence_after();
       uint8_t* box = stg + half * kBox;
+      const TokPos q = et % 128 == 0 ? tok_pos(p.g, r.item, r.text) : TokPos{};   // the storing thread's
 #pragma unroll 1
       for (int m = 0; m < 2; ++m) {           // dK, then dV
         const uint32_t taddr = tmem + tb * 256 + m * 128 + half * 64 + lane_off;
@@ -258,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) gram_bwd_tc_kernel(const __grid_c
         named_bar_sync(1 + half, 128);
         if (et % 128 == 0) {   // rows past the unit's token count are clipped by the TMA
           const CUtensorMap* map = m == 0 ? (r.text ? &p.mdKt : &p.mdK) : (r.text ? &p.mdVt : &p.mdV);
-          tma_store_3d(map, box, 64 * half, r.y, r.item);
+          tok_store(map, box, p.g, q, 64 * half, r.y);
           bulk_commit();
         }
       }
@@ -283,17 +291,19 @@ cudaError_t launch_gram_bwd_tc(const vda_problem& p, const __nv_bfloat16* K, con
   GramBwdParams prm;
   memset(&prm, 0, sizeof(prm));
   const int heads = p.B * p.H, frames = heads * p.T;
-  if (!make_bf16_rows_map(&prm.mK, K, p.n, frames, kRows) || !make_bf16_rows_map(&prm.mV, V, p.n, frames, kRows) ||
+  if (!make_tok_map(&prm.mK, K, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mV, V, p.layout, p.B, p.H, p.T, p.n, kRows) ||
       !make_bf16_rows_map(&prm.mW, W, 256, frames, 128))
     return cudaErrorInvalidValue;
-  if (!make_bf16_rows_map(&prm.mdK, dK, p.n, frames, kRows) || !make_bf16_rows_map(&prm.mdV, dV, p.n, frames, kRows))
+  if (!make_tok_map(&prm.mdK, dK, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mdV, dV, p.layout, p.B, p.H, p.T, p.n, kRows))
     return cudaErrorInvalidValue;
   const bool text = p.n_txt > 0;
-  if (text && (!make_bf16_rows_map(&prm.mKt, Kt, p.n_txt, heads, kRows) ||
-               !make_bf16_rows_map(&prm.mVt, Vt, p.n_txt, heads, kRows) ||
+  if (text && (!make_tok_map(&prm.mKt, Kt, p.layout, p.B, p.H, 1, p.n_txt, kRows) ||
+               !make_tok_map(&prm.mVt, Vt, p.layout, p.B, p.H, 1, p.n_txt, kRows) ||
                !make_bf16_rows_map(&prm.mWt, Wt, 256, heads, 128) ||
-               !make_bf16_rows_map(&prm.mdKt, dKt, p.n_txt, heads, kRows) ||
-               !make_bf16_rows_map(&prm.mdVt, dVt, p.n_txt, heads, kRows)))
+               !make_tok_map(&prm.mdKt, dKt, p.layout, p.B, p.H, 1, p.n_txt, kRows) ||
+               !make_tok_map(&prm.mdVt, dVt, p.layout, p.B, p.H, 1, p.n_txt, kRows)))
     return cudaErrorInvalidValue;
   prm.W = W;
   prm.Wt = Wt;
@@ -304,6 +314,7 @@ cudaError_t launch_gram_bwd_tc(const vda_problem& p, const __nv_bfloat16* K, con
   prm.n_txt = p.n_txt;
   prm.tpf = (p.n + kRows - 1) / kRows;
   prm.tpt = text ? (p.n_txt + kRows - 1) / kRows : 0;
+  prm.g = TokGeom{p.layout, p.H, p.T};
   const size_t smem = 1024 + (3 + 2 * kStages) * kTile + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(gram_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

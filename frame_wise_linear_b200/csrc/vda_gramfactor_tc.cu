@@ -44,6 +44,7 @@
 // down (waiting, bounded, for its own copies and MMAs).
 #include "sm100.cuh"
 #include "vda_internal.cuh"
+#include "vda_tok.cuh"
 
 namespace vda {
 namespace {
@@ -73,6 +74,7 @@ struct GramFactorParams {
   unsigned* err;
   int BH, T, n, n_txt;
   float lam;
+  TokGeom g;            // the inputs' layout
 };
 
 struct Shared {
@@ -179,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         int rows, z;
         bool text;
         slot_info(p, s, rows, z, text);
+        const TokPos q = tok_pos(p.g, z, text);
         const CUtensorMap* mk = text ? &p.mKt : &p.mK;
         const CUtensorMap* mv = text ? &p.mVt : &p.mV;
         for (int r0 = 0; r0 < rows; r0 += kChunk) {
@@ -188,10 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           }
           uint8_t* st = stages + stage * kStageBytes;
           mbar_expect_tx(&sh.full[stage], kStageBytes);
-          tma_load_3d(st + 0 * kBox, mk, &sh.full[stage], 0, r0, z, pol);
-          tma_load_3d(st + 1 * kBox, mk, &sh.full[stage], 64, r0, z, pol);
-          tma_load_3d(st + 2 * kBox, mv, &sh.full[stage], 0, r0, z, pol);
-          tma_load_3d(st + 3 * kBox, mv, &sh.full[stage], 64, r0, z, pol);
+          tok_load(st + 0 * kBox, mk, &sh.full[stage], p.g, q, 0, r0, pol);
+          tok_load(st + 1 * kBox, mk, &sh.full[stage], p.g, q, 64, r0, pol);
+          tok_load(st + 2 * kBox, mv, &sh.full[stage], p.g, q, 0, r0, pol);
+          tok_load(st + 3 * kBox, mv, &sh.full[stage], p.g, q, 64, r0, pol);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -519,10 +522,13 @@ cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, c
   GramFactorParams prm;
   memset(&prm, 0, sizeof(prm));
   const int BH = p.B * p.H;
-  if (!make_bf16_rows_map(&prm.mK, K, p.n, BH * p.T, 64) || !make_bf16_rows_map(&prm.mV, V, p.n, BH * p.T, 64))
+  if (!make_tok_map(&prm.mK, K, p.layout, p.B, p.H, p.T, p.n, 64) ||
+      !make_tok_map(&prm.mV, V, p.layout, p.B, p.H, p.T, p.n, 64))
     return cudaErrorInvalidValue;
-  if (p.n_txt > 0 && (!make_bf16_rows_map(&prm.mKt, Kt, p.n_txt, BH, 64) || !make_bf16_rows_map(&prm.mVt, Vt, p.n_txt, BH, 64)))
+  if (p.n_txt > 0 && (!make_tok_map(&prm.mKt, Kt, p.layout, p.B, p.H, 1, p.n_txt, 64) ||
+                      !make_tok_map(&prm.mVt, Vt, p.layout, p.B, p.H, 1, p.n_txt, 64)))
     return cudaErrorInvalidValue;
+  prm.g = TokGeom{p.layout, p.H, p.T};
   const long long rows = (long long)BH * (p.T + 1) * 128;
   if (!make_f32_rows_map(&prm.mB, Bm, rows, 128)) return cudaErrorInvalidValue;
   prm.M = reinterpret_cast<uint8_t*>(M);

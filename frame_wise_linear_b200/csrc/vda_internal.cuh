@@ -114,6 +114,15 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
 // TMA descriptor of a [items][rows][128] bf16 tensor, boxes of 64 features x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
 bool make_bf16_rows_map(CUtensorMap* m, const void* ptr, int rows, int items, int box_rows);
+// TMA descriptor of a token tensor (bf16, 128 features) in either layout:
+// layout 0 [B][H][T][rows][128], layout 1 [B][T][rows][H][128] (T = 1 for
+// the text's [B][H][n_txt][128] / [B][n_txt][H][128]).  Layout 0 is the 3-D
+// map (c, r, unit) of make_bf16_rows_map; layout 1 has five dimensions in
+// increasing stride order, (c, h, r, t, b).  Boxes of 64 features x box_rows
+// tokens of one unit, 128-byte swizzle, so a box lands in shared memory as
+// 64 x box_rows in both layouts (vda_tma.cu).
+bool make_tok_map(CUtensorMap* m, const void* ptr, int layout, int B, int H, int T, int rows, int box_rows);
+
 // TMA descriptor of a [rows][128] float32 matrix, boxes of 32 columns x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
 bool make_f32_rows_map(CUtensorMap* m, const void* ptr, long long rows, int box_rows);

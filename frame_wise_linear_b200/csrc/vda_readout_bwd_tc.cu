@@ -28,6 +28,7 @@
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
 #include "vda_internal.cuh"
+#include "vda_tok.cuh"
 
 namespace vda {
 namespace {
@@ -56,6 +57,7 @@ struct ReadoutBwdParams {
   int frames;
   int n;
   int tiles_per_frame;
+  TokGeom g;                      // the layout of Q, G, dO, dQ and dG
 };
 
 struct Shared {
@@ -161,29 +163,33 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       int q_issued = 0, g_issued = 0, o_issued = 0, s_issued = 0;
-      auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int y, int u) {
+      TokPos q{};
+      auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int y) {
         mbar_expect_tx(bar, kTile);
-        tma_load_3d(dst, map, bar, 0, y, u, pol);
-        tma_load_3d(dst + kBox, map, bar, 64, y, u, pol);
+        tok_load(dst, map, bar, p.g, q, 0, y, pol);
+        tok_load(dst + kBox, map, bar, p.g, q, 64, y, pol);
       };
       for (int j = 0; j < J; ++j) {
         const int u = u_begin + j / tpf, y = (j % tpf) * kRows;
+        if (j % tpf == 0) q = tok_pos(p.g, u, false);
         const int st = j & 1;
         const uint32_t ph = ((j >> 1) & 1) ^ 1;
         if (!mbar_wait(&sh.q_empty[st], ph)) { set_abort(sh, p.err); break; }
-        load_tile(qbuf + st * kTile, &p.mQ, &sh.q_full[st], y, u);
+        load_tile(qbuf + st * kTile, &p.mQ, &sh.q_full[st], y);
         ++q_issued;
         if (!mbar_wait(&sh.g_empty[st], ph)) { set_abort(sh, p.err); break; }
-        load_tile(gbuf + st * kTile, &p.mG, &sh.g_full[st], y, u);
+        load_tile(gbuf + st * kTile, &p.mG, &sh.g_full[st], y);
         ++g_issued;
         if (!mbar_wait(&sh.o_empty[st], ph)) { set_abort(sh, p.err); break; }
-        load_tile(obuf + st * kTile, &p.mdO, &sh.o_full[st], y, u);
+        load_tile(obuf + st * kTile, &p.mdO, &sh.o_full[st], y);
         ++o_issued;
         if (j % tpf == 0) {
           // S_t of this frame, once the previous frame's last dQ MMAs are done with the buffer.
           const int fr = j / tpf;
           if (fr > 0 && !mbar_wait(&sh.s_empty, (fr - 1) & 1)) { set_abort(sh, p.err); break; }
-          load_tile(sbuf, &p.mS, &sh.s_full, 0, u);
+          mbar_expect_tx(&sh.s_full, kTile);
+          tma_load_3d(sbuf, &p.mS, &sh.s_full, 0, 0, u, pol);
+          tma_load_3d(sbuf + kBox, &p.mS, &sh.s_full, 64, 0, u, pol);
           ++s_issued;
           if (u + 1 < u_end) bulk_prefetch_l2(p.S + (size_t)(u + 1) * 128 * 128, 128 * 128 * 2);   // the next frame's
         }
@@ -317,17 +323,25 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
       mbar_arrive(&sh.dp_full[tb]);
       named_bar_sync(1 + half, 128);
       if (et % 128 == 0) {   // first thread of each half stores that half of dG
-        tma_store_3d(&p.mdG, grow, 64 * half, y, u);
+        tok_store(&p.mdG, grow, p.g, tok_pos(p.g, u, false), 64 * half, y);
         bulk_commit();
         bulk_wait_read<0>();
         mbar_arrive(&sh.g_empty[st]);
       }
       return true;
     };
-    // Tile i: dQ from TMEM, stored row by row (rows past n skipped).
+    // Tile i: dQ from TMEM, stored row by row (rows past n skipped).  The
+    // frame's first row and the row stride in dQ, decoded once per frame.
+    int dq_u = -1;
+    size_t dq_base = 0;
+    const size_t rstride = tok_row_stride(p.g);
     auto epi_dq = [&](int i) -> bool {
       const int tb = i % kTBufs;
       const int u = u_begin + i / tpf, y = (i % tpf) * kRows;
+      if (u != dq_u) {
+        dq_base = tok_base(p.g, tok_pos(p.g, u, false), p.n, false);
+        dq_u = u;
+      }
       bool ok = !aborted(sh) && mbar_wait(&sh.dq_full[tb], (i / kTBufs) & 1);
       if (!ok) set_abort(sh, p.err);
       if (named_bar_or(1 + half, 128, !ok)) return false;
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
       for (int k = 0; k < 8; ++k) {
         const int tr = y + r0 + k;             // token row; rows past n skipped
         if (tr < p.n)
-          *reinterpret_cast<uint4*>(p.dQ + ((size_t)u * p.n + tr) * 128 + half * 64 + (lane & 7) * 8) = ch[k];
+          *reinterpret_cast<uint4*>(p.dQ + dq_base + tr * rstride + half * 64 + (lane & 7) * 8) = ch[k];
       }
       tc_fence_before();
       mbar_arrive(&sh.t_empty[tb]);
@@ -408,9 +422,11 @@ cudaError_t launch_readout_bwd_tc(const vda_problem& p, const __nv_bfloat16* Q, 
   ReadoutBwdParams prm;
   memset(&prm, 0, sizeof(prm));
   const int frames = p.B * p.H * p.T;
-  if (!make_bf16_rows_map(&prm.mQ, Q, p.n, frames, kRows) || !make_bf16_rows_map(&prm.mG, G, p.n, frames, kRows) ||
-      !make_bf16_rows_map(&prm.mdO, dO, p.n, frames, kRows) ||
-      !make_bf16_rows_map(&prm.mdG, dG, p.n, frames, kRows) || !make_bf16_rows_map(&prm.mS, S, 128, frames, 128))
+  if (!make_tok_map(&prm.mQ, Q, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mG, G, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mdO, dO, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mdG, dG, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_bf16_rows_map(&prm.mS, S, 128, frames, 128))
     return cudaErrorInvalidValue;
   prm.S = S;
   prm.dQ = dQ;
@@ -419,6 +435,7 @@ cudaError_t launch_readout_bwd_tc(const vda_problem& p, const __nv_bfloat16* Q, 
   prm.frames = frames;
   prm.n = p.n;
   prm.tiles_per_frame = (p.n + kRows - 1) / kRows;
+  prm.g = TokGeom{p.layout, p.H, p.T};
   const size_t smem = 1024 + (1 + 3 * kStages) * kTile + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(readout_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

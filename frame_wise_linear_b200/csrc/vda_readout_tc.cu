@@ -27,6 +27,7 @@
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
 #include "vda_internal.cuh"
+#include "vda_tok.cuh"
 
 namespace vda {
 namespace {
@@ -55,6 +56,7 @@ struct ReadoutTcParams {
   unsigned* err;
   int units;       // B*H*T frames
   int tiles_per_unit;
+  TokGeom g;       // the layout of Q, G and O
 };
 
 struct Shared {
@@ -140,16 +142,22 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       int qs = 0, gs = 0;
       uint32_t qph = 0, gph = 0;
       int q_issued = 0, g_issued = 0;
+      int pos_u = -1;
+      TokPos q{};
       for (int tile = t_begin; tile < t_end && !aborted(sh); ++tile) {
         const int u = tile / p.tiles_per_unit;
         const int y = (tile % p.tiles_per_unit) * kRows;
+        if (u != pos_u) {
+          q = tok_pos(p.g, u, false);
+          pos_u = u;
+        }
         if (!mbar_wait(&sh.q_empty[qs], qph ^ 1)) {
           set_abort(sh, p.err);
           break;
         }
         mbar_expect_tx(&sh.q_full[qs], kTile);
-        tma_load_3d(qbuf + qs * kTile, &p.mQ, &sh.q_full[qs], 0, y, u, pol);
-        tma_load_3d(qbuf + qs * kTile + kBox, &p.mQ, &sh.q_full[qs], 64, y, u, pol);
+        tok_load(qbuf + qs * kTile, &p.mQ, &sh.q_full[qs], p.g, q, 0, y, pol);
+        tok_load(qbuf + qs * kTile + kBox, &p.mQ, &sh.q_full[qs], p.g, q, 64, y, pol);
         ++q_issued;
         if (++qs == kQStages) { qs = 0; qph ^= 1; }
         if (!mbar_wait(&sh.g_empty[gs], gph ^ 1)) {
@@ -157,8 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
           break;
         }
         mbar_expect_tx(&sh.g_full[gs], kTile);
-        tma_load_3d(gbuf + gs * kTile, &p.mG, &sh.g_full[gs], 0, y, u, pol);
-        tma_load_3d(gbuf + gs * kTile + kBox, &p.mG, &sh.g_full[gs], 64, y, u, pol);
+        tok_load(gbuf + gs * kTile, &p.mG, &sh.g_full[gs], p.g, q, 0, y, pol);
+        tok_load(gbuf + gs * kTile + kBox, &p.mG, &sh.g_full[gs], p.g, q, 64, y, pol);
         ++g_issued;
         if (++gs == kGStages) { gs = 0; gph ^= 1; }
       }
@@ -259,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       fence_proxy_async_smem();
       named_bar_sync(1 + half, 128);
       if (et % 128 == 0) {   // first thread of each half stores that half
-        tma_store_3d(&p.mO, rowp, 64 * half, y, u);
+        tok_store(&p.mO, rowp, p.g, tok_pos(p.g, u, false), 64 * half, y);
         bulk_commit();
         bulk_wait_read<0>();
         mbar_arrive(&sh.g_empty[gs]);
@@ -374,15 +382,17 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
   ReadoutTcParams prm;
   memset(&prm, 0, sizeof(prm));
   const int units = p.B * p.H * p.T;
-  if (!make_bf16_rows_map(&prm.mQ, Q, p.n, units, kRows) || !make_bf16_rows_map(&prm.mG, G, p.n, units, kRows) ||
-      !make_bf16_rows_map(&prm.mO, O, p.n, units, kRows) || !make_bf16_rows_map(&prm.mSF, SF, 128, units, 128) ||
-      !make_bf16_rows_map(&prm.mSB, SB, 128, units, 128))
+  if (!make_tok_map(&prm.mQ, Q, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mG, G, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mO, O, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_bf16_rows_map(&prm.mSF, SF, 128, units, 128) || !make_bf16_rows_map(&prm.mSB, SB, 128, units, 128))
     return cudaErrorInvalidValue;
   prm.SF = SF;
   prm.SB = SB;
   prm.err = err;
   prm.units = units;
   prm.tiles_per_unit = (p.n + kRows - 1) / kRows;
+  prm.g = TokGeom{p.layout, p.H, p.T};
   const size_t smem = 1024 + kSig + (kQStages + kGStages) * kTile + 2 * kPiece + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

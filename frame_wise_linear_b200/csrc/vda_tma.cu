@@ -33,6 +33,28 @@ bool make_bf16_rows_map(CUtensorMap* m, const void* ptr, int rows, int items, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tok_map(CUtensorMap* m, const void* ptr, int layout, int B, int H, int T, int rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn || B < 1 || H < 1 || T < 1 || rows < 1 || box_rows < 1 || box_rows > 256) return false;
+  const cuuint64_t row = 128 * 2;   // one token's 128 features, bytes
+  cuuint64_t dims[5], strides[4];
+  cuuint32_t box[5];
+  // [B][H][T][rows][128]: the 3-D map (c, r, unit).
+  if (layout == 0) return make_bf16_rows_map(m, ptr, rows, B * H * T, box_rows);
+  // [B][T][rows][H][128]: dims (c, h, r, t, b).
+  {
+    const cuuint64_t d[5] = {128, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t s[4] = {row, row * H, row * H * rows, row * H * rows * T};
+    const cuuint32_t b[5] = {64, 1, (cuuint32_t)box_rows, 1, 1};
+    for (int i = 0; i < 5; ++i) dims[i] = d[i], box[i] = b[i];
+    for (int i = 0; i < 4; ++i) strides[i] = s[i];
+  }
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_f32_rows_map(CUtensorMap* m, const void* ptr, long long rows, int box_rows) {
   auto fn = encode_fn();
   if (!fn || rows < 1 || box_rows < 1 || box_rows > 256) return false;

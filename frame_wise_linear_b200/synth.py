@@ -252,3 +252,14 @@ def grad_out_torch(w: Workload | str, seed: int = 0, device="cuda"):
                 t = t.view(torch.int16).view(torch.bfloat16)
             out[b, h].copy_(t)
     return out
+
+
+def token_major(x):
+    """A tensor of the [B, H, T, n, d] layout as [B, T*n, H, d] (text [B, H, n_txt, d] as
+    [B, n_txt, H, d]), contiguous: the inputs of the token-major layout, same values."""
+    if x is None:
+        return None
+    if x.dim() == 5:
+        B, H, T, n, d = x.shape
+        return x.permute(0, 2, 3, 1, 4).reshape(B, T * n, H, d).contiguous()
+    return x.permute(0, 2, 1, 3).contiguous()

@@ -30,6 +30,8 @@ VDA_ERR_TIMEOUT = 6
 
 VDA_DTYPE_F32 = 0
 VDA_DTYPE_BF16 = 1
+VDA_LAYOUT_BHTND = 0   # Q, K, V, G, O: [B, H, T, n, d]; text [B, H, n_txt, d]
+VDA_LAYOUT_BTNHD = 1   # Q, K, V, G, O: [B, T*n, H, d]; text [B, n_txt, H, d] (bf16 only)
 
 SYMBOLS = (
     "vda_workspace_size",
@@ -51,7 +53,8 @@ SYMBOLS = (
 class vda_problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32),
                 ("n", ctypes.c_int32), ("n_txt", ctypes.c_int32), ("d_k", ctypes.c_int32),
-                ("d_v", ctypes.c_int32), ("dtype", ctypes.c_int32), ("lambda_", ctypes.c_float)]
+                ("d_v", ctypes.c_int32), ("dtype", ctypes.c_int32), ("lambda_", ctypes.c_float),
+                ("layout", ctypes.c_int32)]
 
 
 class VdaError(RuntimeError):
@@ -120,9 +123,9 @@ def _check(status: int, where: str):
         raise VdaError(status, where, load().vda_last_error().decode())
 
 
-def make_problem(B, H, T, n, n_txt, d_k, d_v, dtype, lam) -> vda_problem:
+def make_problem(B, H, T, n, n_txt, d_k, d_v, dtype, lam, layout=0) -> vda_problem:
     return vda_problem(int(B), int(H), int(T), int(n), int(n_txt), int(d_k), int(d_v), int(dtype),
-                       float(lam))
+                       float(lam), int(layout))
 
 
 def _ptr(x) -> int | None:

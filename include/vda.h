@@ -20,9 +20,15 @@
  *     S^b_t = A_t^{-1} (lambda S^b_{t+1} + B_t),  S^b_{T+1} = S_0 (t = T..1)
  *     O_t   = sigmoid(G_t) * (Q_t S^f_t + Q_t S^b_t)            (element-wise)
  *
- * Layout.  Every tensor is dense, row-major, contiguous:
+ * Layout.  Every tensor is dense, row-major, contiguous.  With
+ * vda_problem.layout = VDA_LAYOUT_BHTND (0, the default):
  *     Q, K : [B, H, T, n, d_k]      V, G, O : [B, H, T, n, d_v]
  *     K_txt: [B, H, n_txt, d_k]     V_txt   : [B, H, n_txt, d_v]
+ * With VDA_LAYOUT_BTNHD (1; bfloat16 only), the token-major layout of a
+ * video transformer's attention, heads inside tokens:
+ *     Q, K : [B, T*n, H, d_k]       V, G, O : [B, T*n, H, d_v]
+ *     K_txt: [B, n_txt, H, d_k]     V_txt   : [B, n_txt, H, d_v]
+ * The gradients of vda_backward* take the layout of their inputs.  In both:
  *     S_fwd, S_bwd (states)          : [B, H, T, d_k, d_v], float32
  * Inputs and O share one element type, vda_problem.dtype: float32 or
  * bfloat16.  The state recurrence and every accumulation are float32; O is
@@ -70,6 +76,8 @@ typedef enum vda_status {
 
 typedef enum vda_dtype { VDA_DTYPE_F32 = 0, VDA_DTYPE_BF16 = 1 } vda_dtype;
 
+typedef enum vda_layout { VDA_LAYOUT_BHTND = 0, VDA_LAYOUT_BTNHD = 1 } vda_layout;
+
 /* Problem sizes.  B, H, T, n >= 1; n_txt >= 0.
  * float32: d_k, d_v multiples of 16 in [16, 128].
  * bfloat16: d_k = d_v = 128.
@@ -80,6 +88,7 @@ typedef struct vda_problem {
   int32_t B, H, T, n, n_txt, d_k, d_v;
   int32_t dtype; /* vda_dtype */
   float lambda;
+  int32_t layout; /* vda_layout; VDA_LAYOUT_BTNHD needs bfloat16 */
 } vda_problem;
 
 /* Bytes of device workspace vda_forward needs for `p` (written to *bytes).

@@ -167,3 +167,16 @@ def test_backward_entry_points_checked_and_fail_loudly(lib, entry):
     assert fn(p, *bad, ok, stream=0, workspace_bytes=need, check=False) == vda.VDA_ERR_INVALID_ARG
     assert fn(p, *args, ok, stream=0, workspace_bytes=need - 1, check=False) == vda.VDA_ERR_WORKSPACE
     assert fn(p, *args, ok, stream=0, workspace_bytes=need, check=False) == vda.VDA_ERR_CUDA
+
+
+def test_layout_checked(lib):
+    """An unknown layout is an argument error; the token-major layout needs bf16."""
+    import ctypes
+    size = ctypes.c_size_t(0)
+    bad = _p(layout=2)
+    assert lib.vda_workspace_size(ctypes.byref(bad), ctypes.byref(size)) == vda.VDA_ERR_INVALID_ARG
+    f32 = _p(dtype=vda.VDA_DTYPE_F32, layout=vda.VDA_LAYOUT_BTNHD)
+    assert lib.vda_workspace_size(ctypes.byref(f32), ctypes.byref(size)) == vda.VDA_ERR_UNSUPPORTED
+    ok = _p(layout=vda.VDA_LAYOUT_BTNHD)
+    assert vda.vda_workspace_size(ok) == vda.vda_workspace_size(_p())
+    assert vda.vda_backward_workspace_size(ok) == vda.vda_backward_workspace_size(_p())
