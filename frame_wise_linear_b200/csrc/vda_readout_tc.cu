@@ -231,10 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     for (int tile = t_begin; tile < t_end; ++tile) {
       const int u = tile / p.tiles_per_unit;
       const int y = (tile % p.tiles_per_unit) * kRows;
-      if (__any_sync(0xffffffffu, aborted(sh))) break;
-      bool ok = mbar_wait(&sh.t_full[tb], tph);
+      bool ok = !aborted(sh) && mbar_wait(&sh.t_full[tb], tph);
       ok = ok && mbar_wait(&sh.g_full[gs], gph);
-      if (!__all_sync(0xffffffffu, ok)) { set_abort(sh, p.err); break; }
+      if (!ok) set_abort(sh, p.err);
+      // One decision for the half's four warps, which meet at its named
+      // barrier below: a warp that left alone would strand the others.
+      if (named_bar_or(1 + half, 128, !ok)) break;
       tc_fence_after();
       uint8_t* gt = gbuf + gs * kTile;
       uint8_t* rowp = gt + half * kBox;
