@@ -180,3 +180,12 @@ def test_layout_checked(lib):
     ok = _p(layout=vda.VDA_LAYOUT_BTNHD)
     assert vda.vda_workspace_size(ok) == vda.vda_workspace_size(_p())
     assert vda.vda_backward_workspace_size(ok) == vda.vda_backward_workspace_size(_p())
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_backward_workspace_extends_the_forward_one(lib, layout):
+    """vda_backward_from_forward reads the forward's regions at the forward's offsets, so the backward
+    workspace is the forward's plus more (the forward's layout is its prefix)."""
+    for kw in (dict(), dict(n_txt=0), dict(T=1), dict(B=2, H=3, T=5, n=1008, n_txt=256)):
+        p = _p(layout=layout, **kw)
+        assert vda.vda_backward_workspace_size(p) > vda.vda_workspace_size(p)

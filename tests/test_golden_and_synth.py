@@ -81,3 +81,26 @@ def test_ill_conditioned_keys_are_nearly_low_rank():
     K = inp.widened("K")[0, 0, 0]
     s = np.linalg.svd(K, compute_uv=False)
     assert s[7] ** 2 > 50 and s[8] ** 2 < 0.05     # 8 dominant directions, the rest noise
+
+
+def test_token_major_permutation_is_the_documented_layout():
+    """synth.token_major: element (b, h, t, r, c) of [B, H, T, n, d] lands at (b, t*n + r, h, c); the
+    text's (b, h, r, c) at (b, r, h, c)."""
+    import torch
+    B, H, T, n, d, nt = 2, 3, 4, 5, 6, 7
+    x = torch.arange(B * H * T * n * d, dtype=torch.float32).reshape(B, H, T, n, d)
+    y = synth.token_major(x)
+    assert y.shape == (B, T * n, H, d) and y.is_contiguous()
+    for b in range(B):
+        for h in range(H):
+            for t in range(T):
+                for r in range(n):
+                    assert torch.equal(y[b, t * n + r, h], x[b, h, t, r])
+    xt = torch.arange(B * H * nt * d, dtype=torch.float32).reshape(B, H, nt, d)
+    yt = synth.token_major(xt)
+    assert yt.shape == (B, nt, H, d)
+    for b in range(B):
+        for h in range(H):
+            for r in range(nt):
+                assert torch.equal(yt[b, r, h], xt[b, h, r])
+    assert synth.token_major(None) is None
