@@ -484,7 +484,8 @@ def backward_roofline(w, peaks):
     bh = w.B * w.H
     frames = bh * w.T
     tok = frames * w.n
-    nbytes = tok * (3 * w.d_k + 6 * w.d_v) * es + bh * w.n_txt * 2 * (w.d_k + w.d_v) * es
+    # per token: Q, K, dQ, dK (d_k each); V, G, dO, dV, dG (d_v each); the text: K_txt, V_txt, dK_txt, dV_txt
+    nbytes = tok * (4 * w.d_k + 5 * w.d_v) * es + bh * w.n_txt * 2 * (w.d_k + w.d_v) * es
     flops = 2.0 * tok * w.d_k * (w.d_k + w.d_v) + 2.0 * tok * 3 * w.d_k * w.d_v + 2.0 * tok * w.d_k * (w.d_k + 2 * w.d_v)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)

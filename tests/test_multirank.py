@@ -65,3 +65,20 @@ def test_two_gloo_ranks():
     assert res[0][2] != res[1][2]                # independent problems per rank
     again = float(np.asarray(synth.make_inputs(w, seed=1).K).sum())
     assert again == res[1][2]                    # and each one reproducible
+
+
+def test_backward_roofline_bytes_are_the_tensors():
+    """The backward's algorithmic bytes: every input and gradient tensor once, summed from their shapes."""
+    import bench
+    from frame_wise_linear_b200 import synth
+    for name in ("768p", "768p_h8", "mid"):
+        w = synth.WORKLOADS[name]
+        es = 2 if w.dtype == synth.DTYPE_BF16 else 4
+        tok = (w.B, w.H, w.T, w.n)
+        txt = (w.B, w.H, w.n_txt)
+        shapes = [tok + (w.d_k,)] * 4 + [tok + (w.d_v,)] * 5 + [txt + (w.d_k,), txt + (w.d_v,)] * 2
+        want = sum(int(np.prod(s)) for s in shapes) * es
+        rf = bench.backward_roofline(w, {"hbm_gbs": 6549.1, "bf16_tflops": 1628.0})
+        assert rf["bytes"] == want, name
+    assert bench.backward_roofline(synth.WORKLOADS["768p"], {"hbm_gbs": 6549.1, "bf16_tflops": 1628.0})["bytes"] \
+        == 3352690688
