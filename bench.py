@@ -83,7 +83,7 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
-# Work counts (the design doc states them): algorithmic bytes / flops per launch.
+# Work counts: algorithmic bytes / flops per launch.
 # ---------------------------------------------------------------------------
 
 def stage_work(w):
@@ -196,6 +196,17 @@ class ClockSampler:
 # CPU oracle timing (bounded sample)
 # ---------------------------------------------------------------------------
 
+def cpu_threads():
+    """Threads the CPU legs give the oracle's BLAS: every host core."""
+    return os.cpu_count() or 1
+
+
+def blas_limits():
+    """Fixes the BLAS thread count for the oracle's timing (both CPU legs use the same)."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=cpu_threads(), user_api="blas")
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -204,34 +215,38 @@ def blas_threads():
             return max(n)
     except Exception:
         pass
-    return os.cpu_count() or 1
+    return cpu_threads()
 
 
-def cpu_oracle_sample(w, budget_s, max_frames=None):
-    """Times the float64 oracle on whole heads (all frames) until the budget is used.
-
-    Returns (frames*heads per second, units timed, description).  Input
-    generation and widening are outside the timed part.
-    """
+def cpu_sample_inputs(w, frames=None):
+    """The CPU legs' sample: head (0, 0) of the workload, its first `frames` frames (all by default)."""
     from frame_wise_linear_b200 import synth
+    x = synth.head_widened(w, 0, 0, seed=0)
+    T = w.T if frames is None else max(1, min(w.T, frames))
+    return [x["Q"][:T], x["K"][:T], x["V"][:T], x["G"][:T], x["K_txt"], x["V_txt"], w.lam], T
+
+
+def cpu_oracle_sample(w, budget_s):
+    """Times the float64 oracle on the CPU sample, repeated until the budget is used.
+
+    Returns (frames*heads per second, threads, description).  The same sample
+    and thread count as the reference arm's steps; input generation and
+    widening are outside the timed part.
+    """
     from oracle import vda_oracle as vo
-    spent, units, heads = 0.0, 0, 0
-    for b in range(w.B):
-        for h in range(w.H):
-            x = synth.head_widened(w, b, h, seed=0)
-            T = w.T if max_frames is None else min(w.T, max_frames)
-            args = [x["Q"][:T], x["K"][:T], x["V"][:T], x["G"][:T], x["K_txt"], x["V_txt"], w.lam]
+    args, T = cpu_sample_inputs(w)
+    with blas_limits():
+        vo.vda_head(*args)           # warm-up (BLAS thread pool start-up)
+        spent, reps = 0.0, 0
+        while spent < budget_s:
             t0 = time.perf_counter()
             vo.vda_head(*args)
             spent += time.perf_counter() - t0
-            units += T
-            heads += 1
-            if spent >= budget_s:
-                break
-        if spent >= budget_s:
-            break
-    desc = f"{heads} head(s) x {units // max(heads, 1)} frames of the {w.name} workload (float64 oracle)"
-    return units / spent, units, desc
+            reps += 1
+        threads = blas_threads()
+    desc = (f"head (0,0), frames 1..{T} of the {w.name} workload, repeated {reps} times "
+            f"(float64 oracle, {threads} BLAS threads)")
+    return reps * T / spent, threads, desc
 
 
 # ---------------------------------------------------------------------------
@@ -249,30 +264,33 @@ def run_reference(args, w):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    # Size each step so the whole run stays within about two minutes.
-    from frame_wise_linear_b200 import synth
     from oracle import vda_oracle as vo
-    x = synth.head_widened(w, 0, 0, seed=0)
-    t0 = time.perf_counter()
-    vo.vda_head(x["Q"][:2], x["K"][:2], x["V"][:2], x["G"][:2], x["K_txt"], x["V_txt"], w.lam)
-    per_frame = (time.perf_counter() - t0) / 2
-    budget = 120.0 / max(args.steps + args.warmup, 1)
-    frames = int(max(1, min(w.T, budget / max(per_frame, 1e-6))))
-    args_h = [x["Q"][:frames], x["K"][:frames], x["V"][:frames], x["G"][:frames], x["K_txt"], x["V_txt"], w.lam]
-    for _ in range(args.warmup):
-        vo.vda_head(*args_h)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        vo.vda_head(*args_h)
-    dt = time.perf_counter() - t0
+    # Each step is the CPU sample (head (0,0), all frames), cut to fewer
+    # frames only if the whole run would take more than about two minutes.
+    with blas_limits():
+        args2, _ = cpu_sample_inputs(w, 2)
+        vo.vda_head(*args2)
+        t0 = time.perf_counter()
+        vo.vda_head(*args2)
+        per_frame = (time.perf_counter() - t0) / 2
+        budget = 120.0 / max(args.steps + args.warmup, 1)
+        args_h, frames = cpu_sample_inputs(w, int(max(1, budget / max(per_frame, 1e-6))))
+        for _ in range(args.warmup):
+            vo.vda_head(*args_h)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            vo.vda_head(*args_h)
+        dt = time.perf_counter() - t0
+        threads = blas_threads()
     value = args.steps * frames / dt
-    sample = f"each step: head (0,0), frames 1..{frames} of the {w.name} workload (float64 oracle)"
+    sample = (f"each step: head (0,0), frames 1..{frames} of the {w.name} workload "
+              f"(float64 oracle, {threads} BLAS threads)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -280,6 +298,7 @@ def run_reference(args, w):
     return 0
 
 
+L2_BYTES = 126e6
 LAYOUTS = {"bhtnd": 0, "btnhd": 1}
 LAYOUT_NAMES = {0: "[B,H,T,n,d]", 1: "[B,T*n,H,d]"}
 
@@ -290,7 +309,10 @@ def config_of(w, n, layout=0):
             "B": w.B, "H": w.H, "T": w.T, "n": w.n, "n_txt": w.n_txt, "d": w.d_k,
             "layout": LAYOUT_NAMES[layout],
             "parallelism": f"independent problems on {n} GPU(s), no collective",
-            "l2": f"inputs larger than L2 ({input_bytes(w) / 1e9:.2f} GB read per step vs 126 MB); no flush"}
+            "l2": (f"inputs larger than L2 ({input_bytes(w) / 1e9:.2f} GB read per step vs 126 MB); no flush"
+                   if input_bytes(w) > L2_BYTES else
+                   f"inputs smaller than L2 ({input_bytes(w) / 1e6:.1f} MB vs 126 MB), not flushed: "
+                   "a latency-bound workload, not the headline")}
 
 
 def max_over_ranks(ms, dist, device):
@@ -463,8 +485,8 @@ def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
         "clocks": clocks, "gpu_launches": vda.LAUNCHES_PER_FORWARD[w.dtype] * args.steps,
     }
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
-        v, units, desc = cpu_oracle_sample(w, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        v, threads, desc = cpu_oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": desc}
     if pg:
         pg.barrier()

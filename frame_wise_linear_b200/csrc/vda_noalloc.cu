@@ -3,8 +3,16 @@
 //
 // The scratch is a file-scope __device__ array.  In host code its name is only
 // a host-side stand-in, not a device address, so the device address is looked
-// up with cudaGetSymbolAddress once per device (with that device current) and
-// cached; the workspace pointer handed to the kernels is that address.
+// up with cudaGetSymbolAddress (with the device current) and the workspace
+// pointer handed to the kernels is that address.
+//
+// That address belongs to a CUDA context, not to a device ordinal: the module
+// holding the array is loaded once per context.  The lookup is therefore
+// cached per context, keyed by the context's process-unique ID.  A device that
+// was reset (cudaDeviceReset) gets a new primary context with a new ID, and a
+// context a driver-API caller made current gets its own entry, so neither can
+// be handed the address of another context's scratch.
+#include <cudaTypedefs.h>
 #include <stdio.h>
 
 #include <mutex>
@@ -14,27 +22,73 @@
 namespace {
 
 constexpr size_t kScratchBytes = VDA_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 128;
+constexpr int kMaxContexts = 256;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
+struct CachedAddress {
+  unsigned long long ctx_id;
+  void* addr;
+};
 
-// Device address of g_scratch on the current device (looked up on first use).
+std::mutex g_mu;
+CachedAddress g_cache[kMaxContexts];
+int g_cached = 0;
+int g_next = 0;   // the entry a full cache replaces next
+
+PFN_cuCtxGetCurrent_v4000 g_get_current = nullptr;
+PFN_cuCtxGetId_v12000 g_get_id = nullptr;
+
+// Driver entry points through the runtime (the library does not link libcuda).
+bool driver_entry_points() {
+  if (g_get_current && g_get_id) return true;
+  void* a = nullptr;
+  void* b = nullptr;
+  cudaDriverEntryPointQueryResult qa, qb;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &a, 4000, cudaEnableDefault, &qa) != cudaSuccess ||
+      qa != cudaDriverEntryPointSuccess ||
+      cudaGetDriverEntryPointByVersion("cuCtxGetId", &b, 12000, cudaEnableDefault, &qb) != cudaSuccess ||
+      qb != cudaDriverEntryPointSuccess)
+    return false;
+  g_get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(a);
+  g_get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(b);
+  return true;
+}
+
+// ID of the context current on this thread (0 when none is).
+cudaError_t current_context_id(unsigned long long* id) {
+  *id = 0;
+  CUcontext ctx = nullptr;
+  if (g_get_current(&ctx) != CUDA_SUCCESS) return cudaErrorContextIsDestroyed;
+  if (!ctx) return cudaSuccess;
+  if (g_get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorContextIsDestroyed;
+  return cudaSuccess;
+}
+
+// Device address of g_scratch in the context current on this thread.  The
+// first call in a context makes the runtime's primary context current if no
+// context is, and looks the address up.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess) return e;
-    g_addr[dev] = p;
+  if (!driver_entry_points()) return cudaErrorNotSupported;
+  unsigned long long id = 0;
+  cudaError_t e = current_context_id(&id);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; id && i < g_cached; ++i)
+    if (g_cache[i].ctx_id == id) {
+      *out = g_cache[i].addr;
+      return cudaSuccess;
+    }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_scratch);   // initialises the primary context if none is current
+  if (e != cudaSuccess) return e;
+  if (!id && (e = current_context_id(&id)) != cudaSuccess) return e;
+  if (id) {
+    const int slot = g_cached < kMaxContexts ? g_cached++ : g_next;
+    g_next = (slot + 1) % kMaxContexts;
+    g_cache[slot] = CachedAddress{id, p};
   }
-  *out = g_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
@@ -59,7 +113,7 @@ extern "C" vda_status vda_forward_noalloc(const vda_problem* p, const void* Q, c
   cudaError_t e = scratch_address(&ws);
   if (e != cudaSuccess) {
     char msg[256];
-    snprintf(msg, sizeof(msg), "vda_forward_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    snprintf(msg, sizeof(msg), "vda_forward_noalloc: looking up the scratch address: %s", cudaGetErrorString(e));
     vda::set_error_message(msg);
     return VDA_ERR_CUDA;
   }

@@ -310,15 +310,30 @@ def problem_for(Q, K, V, G, K_txt, V_txt, lam) -> vda_problem:
     return make_problem(Bn, Hn, T, n, n_txt, d_k, d_v, dt, lam)
 
 
-def forward(Q, K, V, G, K_txt, V_txt, lam: float, stream=None, workspace=None, out=None):
-    """O = VDA(Q, K, V, G, K_txt, V_txt; lam) on the inputs' device."""
+def forward(Q, K, V, G, K_txt, V_txt, lam: float, stream=None, workspace=None, out=None, check=False):
+    """O = VDA(Q, K, V, G, K_txt, V_txt; lam) on the inputs' device.
+
+    The call is enqueued on `stream` (default: the current torch stream).  A
+    workspace allocated here is allocated on that stream and marked as used by
+    it, so torch's caching allocator does not hand its memory to another
+    stream while the kernels still run.  check=True synchronises the stream
+    and raises on a device-side condition (VDA_ERR_NOT_SPD, VDA_ERR_TIMEOUT).
+    """
     import torch
     prob = problem_for(Q, K, V, G, K_txt, V_txt, lam)
     ws_bytes = vda_workspace_size(prob)
-    if workspace is None or _nbytes(workspace) < ws_bytes:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
-    O = out if out is not None else torch.empty(G.shape, dtype=G.dtype, device=G.device)
+    s = torch.cuda.current_stream(Q.device) if stream is None else stream
+    if not isinstance(s, torch.cuda.Stream):
+        raise TypeError("stream must be a torch.cuda.Stream (or None for the current stream)")
+    with torch.cuda.stream(s):
+        if workspace is None or _nbytes(workspace) < ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+        O = out if out is not None else torch.empty(G.shape, dtype=G.dtype, device=G.device)
     txt = prob.n_txt > 0
     vda_forward(prob, Q, K, V, G, K_txt if txt else None, V_txt if txt else None, O, workspace,
-                stream=stream)
+                stream=s)
+    workspace.record_stream(s)
+    O.record_stream(s)
+    if check:
+        vda_sync_status(workspace, stream=s)
     return O

@@ -160,15 +160,21 @@ vda_status vda_forward_host(const vda_problem* p, const void* Q, const void* K, 
  *   - problems whose vda_workspace_size() exceeds the scratch are rejected
  *     with VDA_ERR_WORKSPACE before anything is enqueued (for example the
  *     mid workload, 8 heads x 16 frames, fits; 32 heads x 45 frames does not);
- *   - the first call on a device looks up the scratch's device address (with
- *     that device current); make that first call before any stream capture;
+ *   - the scratch's device address belongs to the CUDA context current on
+ *     the calling thread; the first call in each context (the device's
+ *     primary context, one a driver-API caller made current, or the new
+ *     primary context after a cudaDeviceReset) looks that address up and
+ *     caches it under the context's unique ID; make that first call before
+ *     any stream capture;
  *   - every call on a device shares the one scratch, which keeps the last
  *     call's contents (each call clears what must start at zero): calls that
  *     overlap on the GPU, on different streams or from different threads,
  *     race and give wrong results;
  *   - the device error word lives in the scratch, so device-side conditions
- *     (VDA_ERR_NOT_SPD, VDA_ERR_TIMEOUT) are not reported by this call; host
- *     side argument errors are, as for vda_forward.
+ *     (VDA_ERR_NOT_SPD, VDA_ERR_TIMEOUT) are not reported by this call: a
+ *     caller that needs them must validate O itself (for example, that it
+ *     is finite) or use vda_forward with vda_sync_status; host-side argument
+ *     errors are reported, as for vda_forward.
  * The pages describe no such entry point: it has no counterpart there. */
 #define VDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 vda_status vda_forward_noalloc(const vda_problem* p, const void* Q, const void* K, const void* V,

@@ -83,14 +83,16 @@ def test_768p_sampled_heads():
 
 @pytest.mark.slow
 def test_ill_conditioned_sampled_heads():
-    errs = _sampled("illcond", [(0, 0), (0, 31)])
+    errs = _sampled("illcond", [(0, 0), (0, 9), (0, 22), (0, 31)])
     assert max(errs) <= TOL[synth.DTYPE_BF16], errs
 
 
 @pytest.mark.slow
-def test_long_clip_180_frames_sampled_heads():
-    errs = _sampled("long180", [(0, 0), (1, 31)])
-    assert max(errs) <= TOL[synth.DTYPE_BF16], errs
+@pytest.mark.parametrize("name", ["long45", "long90", "long180"])
+def test_long_clip_sampled_heads(name):
+    """The long-clip sweep (B = 2): the first head of batch 0 and the last head of batch 1, every frame."""
+    errs = _sampled(name, [(0, 0), (1, 31)])
+    assert max(errs) <= TOL[synth.DTYPE_BF16], (name, errs)
 
 
 def test_repeat_is_bitwise_identical():

@@ -132,3 +132,53 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
 def test_unmutated_oracle_passes_every_pin():
     results = P.run_all()
     assert all(results.values()), results
+
+
+def _layout_case(seed, B=2, H=3, T=3, n=4, d_k=3, d_v=2, n_txt=2):
+    rng = np.random.default_rng(seed)
+    t = lambda *s: rng.standard_normal(s)  # noqa: E731
+    Q, K, V, G = t(B, H, T, n, d_k), t(B, H, T, n, d_k), t(B, H, T, n, d_v), t(B, H, T, n, d_v)
+    Kt, Vt = (t(B, H, n_txt, d_k), t(B, H, n_txt, d_v)) if n_txt else (None, None)
+    return Q, K, V, G, Kt, Vt
+
+
+def test_forward_layout_wrapper_matches_heads():
+    """The [B, H] wrapper is the per-head function applied to head (b, h) and put back at [b, h].
+
+    Heads and batch entries are independent problems ("VDN-MiniMax-H3", section 03:
+    the linear branch is per attention head).  Every head gets different data and a
+    non-square d_k x d_v, so a swapped (b, h) index, a transposed reshape or a
+    misordered head selection fails the element-wise equality.
+    """
+    Q, K, V, G, Kt, Vt = _layout_case(11)
+    B, H = Q.shape[:2]
+    O, states = vo.vda_forward(Q, K, V, G, Kt, Vt, 0.7, return_states=True)
+    assert O.shape == G.shape
+    assert len(states) == B * H
+    for b in range(B):
+        for h in range(H):
+            o1, s1 = vo.vda_head(Q[b, h], K[b, h], V[b, h], G[b, h], Kt[b, h], Vt[b, h], 0.7, return_states=True)
+            np.testing.assert_array_equal(O[b, h], o1)
+            for k in ("S0", "SF", "SB"):
+                np.testing.assert_array_equal(states[b * H + h][k], s1[k])
+    # distinct heads really differ, so the equality above can tell them apart
+    assert not np.allclose(O[0, 1], O[1, 0])
+    assert np.array_equal(vo.vda_forward(Q, K, V, G, Kt, Vt, 0.7), O)
+    # a selection returns exactly those heads, stacked in the order asked for
+    sel = [(1, 2), (0, 0), (1, 0)]
+    some, some_states = vo.vda_forward(Q, K, V, G, Kt, Vt, 0.7, heads=sel, return_states=True)
+    assert some.shape == (len(sel),) + G.shape[2:]
+    for i, (b, h) in enumerate(sel):
+        np.testing.assert_array_equal(some[i], O[b, h])
+        np.testing.assert_array_equal(some_states[i]["SF"], states[b * H + h]["SF"])
+
+
+def test_forward_layout_wrapper_without_text():
+    """n_txt = 0 (no text tensors) gives S_0 = 0 in every head ("VDN-MiniMax-H3", section 03, text injection)."""
+    Q, K, V, G, _, _ = _layout_case(12, n_txt=0)
+    B, H = Q.shape[:2]
+    O, states = vo.vda_forward(Q, K, V, G, None, None, 1.3, return_states=True)
+    for b in range(B):
+        for h in range(H):
+            np.testing.assert_array_equal(O[b, h], vo.vda_head(Q[b, h], K[b, h], V[b, h], G[b, h], None, None, 1.3))
+            assert not np.any(states[b * H + h]["S0"])
