@@ -49,6 +49,9 @@ STAGE_SOURCES = {
     1: {"gram+factor": "frame_wise_linear_b200/csrc/vda_gramfactor_tc.cu",
         "scan": "frame_wise_linear_b200/csrc/vda_scan_tc.cu",
         "readout": "frame_wise_linear_b200/csrc/vda_readout_tc.cu"},
+    2: {"gram+factor": "frame_wise_linear_b200/csrc/vda_gramfactor_tc.cu",
+        "scan": "frame_wise_linear_b200/csrc/vda_scan_tc.cu",
+        "readout": "frame_wise_linear_b200/csrc/vda_readout_tc.cu"},
     0: {"gram": "frame_wise_linear_b200/csrc/vda_simt.cu",
         "factor": "frame_wise_linear_b200/csrc/vda_factor.cu",
         "scan": "frame_wise_linear_b200/csrc/vda_simt.cu",
@@ -68,8 +71,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layout", choices=("bhtnd", "btnhd"), default="bhtnd",
                     help="token tensors as [B, H, T, n, d] (default) or token-major [B, T*n, H, d]")
-    ap.add_argument("--direction", choices=("forward", "backward"), default="forward",
-                    help="backward: time vda_backward (the gradients) instead; a separate line, not the headline")
+    ap.add_argument("--direction", choices=("forward", "backward", "merge"), default="forward",
+                    help="backward: time vda_backward (the gradients); merge: time vda_merge_project (both "
+                         "branches' output projections, summed); separate lines, not the headline")
     return ap.parse_args()
 
 
@@ -86,8 +90,16 @@ def load_peaks():
 # Work counts: algorithmic bytes / flops per launch.
 # ---------------------------------------------------------------------------
 
+def elem_bytes(w):
+    """Bytes of one input element and of one element of O (bf16 O for 8-bit inputs)."""
+    return {0: (4, 4), 1: (2, 2), 2: (1, 2)}[w.dtype]
+
+
+DTYPE_NAMES = {0: "f32", 1: "bf16", 2: "e4m3"}
+
+
 def stage_work(w):
-    es = 2 if w.dtype == 1 else 4
+    es, eo = elem_bytes(w)
     bh = w.B * w.H
     frames = bh * w.T
     slots = bh * (w.T + 1)
@@ -104,16 +116,16 @@ def stage_work(w):
         # two directions, one d_k x d_k by d_k x d_v product per frame
         "scan": dict(bound="alu", bytes=0, flops=2.0 * frames * 2.0 * d_k * d_k * d_v),
         # reads Q_t, G_t, writes O_t
-        "readout": dict(bound="hbm", bytes=frames * w.n * (d_k + 2 * d_v) * es,
+        "readout": dict(bound="hbm", bytes=frames * w.n * ((d_k + d_v) * es + d_v * eo),
                         flops=2.0 * frames * w.n * d_k * d_v),
     }
 
 
 def path_roofline(w, peaks):
-    es = 2 if w.dtype == 1 else 4
+    es, eo = elem_bytes(w)
     bh = w.B * w.H
     frames = bh * w.T
-    nbytes = frames * w.n * (2 * w.d_k + 3 * w.d_v) * es + bh * w.n_txt * (w.d_k + w.d_v) * es
+    nbytes = frames * w.n * ((2 * w.d_k + 2 * w.d_v) * es + w.d_v * eo) + bh * w.n_txt * (w.d_k + w.d_v) * es
     flops = 2.0 * frames * w.n * (w.d_k * (w.d_k + w.d_v) + w.d_k * w.d_v) \
         + 2.0 * bh * w.n_txt * w.d_k * (w.d_k + w.d_v)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
@@ -122,18 +134,19 @@ def path_roofline(w, peaks):
                 bound="hbm" if t_hbm >= t_tc else "tensor")
 
 
-def traffic_lookup(stage, dtype=1):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel's source is unchanged."""
+def traffic_lookup(stage, w):
+    """DRAM bytes per launch of a stage's kernel on workload `w`, from the committed ncu summary,
+    if the kernel's source is unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(path) or stage not in STAGE_SOURCES[dtype]:
+    if not os.path.exists(path) or stage not in STAGE_SOURCES[w.dtype]:
         return None
-    src = os.path.join(ROOT, STAGE_SOURCES[dtype][stage])
+    src = os.path.join(ROOT, STAGE_SOURCES[w.dtype][stage])
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     with open(path) as fh:
         for line in fh:
             p = line.split()
-            if len(p) >= 3 and not line.startswith("#") and p[0] == stage and p[1] == digest:
-                return float(p[2])
+            if len(p) >= 4 and not line.startswith("#") and p[0] == stage and p[1] == w.name and p[2] == digest:
+                return float(p[3])
     return None
 
 
@@ -305,7 +318,8 @@ LAYOUT_NAMES = {0: "[B,H,T,n,d]", 1: "[B,T*n,H,d]"}
 
 def config_of(w, n, layout=0):
     return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} n={w.n} d_k={w.d_k} d_v={w.d_v} "
-                        f"n_txt={w.n_txt} lambda={w.lam} {'bf16' if w.dtype == 1 else 'f32'}",
+                        f"n_txt={w.n_txt} lambda={w.lam} {DTYPE_NAMES[w.dtype]}"
+                        + (" (per-tensor scales, bf16 O)" if w.dtype == 2 else ""),
             "B": w.B, "H": w.H, "T": w.T, "n": w.n, "n_txt": w.n_txt, "d": w.d_k,
             "layout": LAYOUT_NAMES[layout],
             "parallelism": f"independent problems on {n} GPU(s), no collective",
@@ -331,7 +345,7 @@ def job_value(units_per_rank, n_ranks, ms_per_step):
 
 
 def input_bytes(w):
-    es = 2 if w.dtype == 1 else 4
+    es = elem_bytes(w)[0]
     return (w.B * w.H * (w.T * w.n * 2 * (w.d_k + w.d_v) + w.n_txt * (w.d_k + w.d_v))) * es
 
 
@@ -363,7 +377,7 @@ def run_b200(args, w):
     prob = vda.make_problem(**w.problem(), layout=layout)
     wsb = vda.vda_workspace_size(prob)
     wsp = torch.empty(wsb, dtype=torch.uint8, device=dev)
-    O = torch.empty_like(d["G"])
+    O = torch.empty(d["G"].shape, dtype=torch.float32 if w.dtype == 0 else torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
     kt = d["K_txt"] if w.n_txt else None
     vt = d["V_txt"] if w.n_txt else None
@@ -417,7 +431,7 @@ def run_b200(args, w):
     clocks = sampler.stop()
     vda.vda_sync_status(wsp, stream=stream)
     stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i, s in enumerate(vda.STAGES)}
-    if w.dtype == 1:   # one kernel for the Gram and the factor: report them as one stage
+    if w.dtype != 0:   # one kernel for the Gram and the factor: report them as one stage
         stage_ms = {"gram+factor": stage_ms["gram"] + stage_ms["factor"], "scan": stage_ms["scan"],
                     "readout": stage_ms["readout"]}
     ms = max_over_ranks(ms, pg, dev)
@@ -436,7 +450,7 @@ def run_b200(args, w):
         roof = {"kernel": dom, "bound": "alu", "achieved": wk["flops"] / t_s / 1e12, "peak": FP32_SIMT_TFLOPS,
                 "unit": "TFLOP/s", "peak_source": "derived: 148 SMs x 128 FP32 FMA/clk x 2 x 1.965 GHz"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    tr = traffic_lookup(dom, w.dtype)
+    tr = traffic_lookup(dom, w)
     roof["traffic"] = tr
     pr = path_roofline(w, peaks)
     path = {"t_roof_us": pr["t_roof_s"] * 1e6, "bound": pr["bound"], "bytes": pr["bytes"],
@@ -480,7 +494,7 @@ def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if w.dtype == 1 else "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": DTYPE_NAMES[w.dtype], "data": "synthetic",
         "config": config_of(w, ws_n, LAYOUTS[args.layout]), "roofline": roof, "roofline_path": path, "e2e": e2e,
         "clocks": clocks, "gpu_launches": vda.LAUNCHES_PER_FORWARD[w.dtype] * args.steps,
     }
@@ -618,6 +632,76 @@ def run_backward(args, w):
     return 0
 
 
+MERGE_METRIC = "branch merge (output projections of both branches, summed) tokens/sec at 768p shape; % of B200 bf16 peak"
+
+
+def run_merge(args, w):
+    """K timed vda_merge_project calls on one GPU: Y = O_lin W_lin + O_sm W_sm over the workload's tokens,
+    K = H * d_v features per branch, D = H * d_v outputs (the attention block's width)."""
+    import torch
+    from frame_wise_linear_b200 import build as _build
+    from frame_wise_linear_b200 import vda
+    if args.gpus != 1:
+        raise SystemExit("--direction merge runs on one GPU")
+    dev = torch.device("cuda", 0)
+    _build.build()
+    vda.load()
+    peaks, peaks_kind = load_peaks()
+    tokens, K = w.B * w.T * w.n, w.H * w.d_v
+    D = K
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    O = torch.randn(tokens, K, device=dev, generator=g).to(torch.bfloat16)
+    P = torch.randn(tokens, K, device=dev, generator=g).to(torch.bfloat16)
+    Wl = (torch.randn(K, D, device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
+    Ws = (torch.randn(K, D, device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
+    Y = torch.empty(tokens, D, device=dev, dtype=torch.bfloat16)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vda.vda_merge_project(tokens, K, D, O, Wl, P, Ws, Y, ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    vda.vda_sync_status(ws, stream=stream)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    vda.vda_sync_status(ws, stream=stream)
+    ms = a.elapsed_time(b) / args.steps
+    flops = 2.0 * tokens * (2 * K) * D
+    bytes_ = 2 * (2 * tokens * K + 2 * K * D + tokens * D)
+    tf = flops / (ms / 1e3) / 1e12
+    line = {
+        "metric": MERGE_METRIC, "direction": "merge", "value": tokens / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name} tokens ({w.B}x{w.T}x{w.n}), K = D = {K}, two branches, bf16",
+                   "tokens": tokens, "K": K, "D": D, "l2": "inputs larger than L2; no flush"},
+        "roofline": {"kernel": "merge_tc_kernel", "bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json bf16_tflops)", "traffic": None,
+                     "algorithmic_bytes": bytes_},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     from frame_wise_linear_b200 import synth
@@ -626,6 +710,8 @@ def main():
         return run_reference(args, w)
     if args.direction == "backward":
         return run_backward(args, w)
+    if args.direction == "merge":
+        return run_merge(args, w)
     return run_b200(args, w)
 
 

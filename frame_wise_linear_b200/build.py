@@ -6,7 +6,7 @@ Every .cu file under csrc/ is compiled with
 ``-gencode arch=compute_100a,code=sm_100a -lineinfo -O3`` and linked into one
 shared library next to this file.  The CUDA runtime is linked statically; the
 driver is reached through the runtime, so the library needs no link against
-libcuda.  cuBLAS (the backward's plain batched GEMMs) is linked dynamically.
+libcuda, and no other library is linked.  The link refuses undefined symbols.
 """
 from __future__ import annotations
 
@@ -74,7 +74,7 @@ def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -
     if failed:
         raise RuntimeError("nvcc failed building libvda.so")
     tmp = LIB + ".tmp"
-    cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs + ["-lcublas"]
+    cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-Xlinker", "--no-undefined", "-o", tmp] + objs
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

@@ -67,6 +67,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Testing hook: when `stall` is set the wait is made on `never`, an mbarrier
+// that nothing arrives on, so it runs out as a wait on a lost signal would;
+// otherwise this is mbar_wait(bar, parity).
+__device__ __forceinline__ bool mbar_wait_or_stall(uint64_t* bar, uint32_t parity, uint64_t* never, bool stall) {
+  return stall ? mbar_wait(never, 0) : mbar_wait(bar, parity);
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -184,6 +191,18 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem], kind::f8f6f4 (8-bit float inputs, f32
+// accumulate; 32 elements of K per instruction).
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem], kind::tf32 (float32 storage, tf32 inputs,
 // f32 accumulate).
 __device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -280,6 +299,18 @@ __device__ __forceinline__ float to_tf32(float x) {
   return __uint_as_float(r);
 }
 
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0), f32 D,
+// given majors (MN-major is allowed for 8-bit floats), M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                          // D format f32
+         | (0u << 7)                        // A format e4m3
+         | (0u << 10)                       // B format e4m3
+         | ((a_mn_major ? 1u : 0u) << 15)   // A major
+         | ((b_mn_major ? 1u : 0u) << 16)   // B major
+         | ((uint32_t)(N >> 3) << 17)       // N / 8
+         | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, f32 D, given majors, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                          // D format f32
@@ -363,6 +394,29 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
       : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
+}
+
+// 8 x 8 transpose of 16-byte chunks across the 8 lanes of a group (j = lane
+// % 8): chunk k of lane j becomes chunk j of lane k.  A lane holding one row's
+// eight chunks then holds chunk j of eight rows, so the group's eight lanes
+// store one whole 128-byte row segment per instruction (three butterfly
+// stages of shuffles).
+__device__ __forceinline__ void transpose8(uint4 (&x)[8], int j) {
+#pragma unroll
+  for (int s = 1; s < 8; s <<= 1) {
+    const bool hi = (j & s) != 0;
+#pragma unroll
+    for (int k0 = 0; k0 < 8; ++k0) {
+      if (k0 & s) continue;
+      const int k1 = k0 | s;
+      uint4 t = hi ? x[k0] : x[k1];
+      t.x = __shfl_xor_sync(0xffffffffu, t.x, s);
+      t.y = __shfl_xor_sync(0xffffffffu, t.y, s);
+      t.z = __shfl_xor_sync(0xffffffffu, t.z, s);
+      t.w = __shfl_xor_sync(0xffffffffu, t.w, s);
+      if (hi) x[k0] = t; else x[k1] = t;
+    }
+  }
 }
 
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a

@@ -38,12 +38,21 @@ vda_status check_problem(const vda_problem* p) {
     return fail(VDA_ERR_INVALID_ARG, "d_k, d_v must be >= 1 (got %d, %d)", p->d_k, p->d_v);
   if (!(p->lambda > 0.f) || !isfinite(p->lambda))
     return fail(VDA_ERR_INVALID_ARG, "lambda must be finite and > 0 (got %g)", (double)p->lambda);
-  if (p->dtype != VDA_DTYPE_F32 && p->dtype != VDA_DTYPE_BF16)
+  if (p->dtype != VDA_DTYPE_F32 && p->dtype != VDA_DTYPE_BF16 && p->dtype != VDA_DTYPE_E4M3)
     return fail(VDA_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
+  if (p->dtype == VDA_DTYPE_E4M3) {
+    const float sc[4] = {p->scale_q, p->scale_k, p->scale_v, p->scale_g};
+    for (float v : sc)
+      if (!(v > 0.f) || !isfinite(v))
+        return fail(VDA_ERR_INVALID_ARG, "e4m3 scales must be finite and > 0 (got %g, %g, %g, %g)",
+                    (double)sc[0], (double)sc[1], (double)sc[2], (double)sc[3]);
+  }
   if (p->layout != VDA_LAYOUT_BHTND && p->layout != VDA_LAYOUT_BTNHD)
     return fail(VDA_ERR_INVALID_ARG, "unknown layout %d", p->layout);
-  if (p->layout == VDA_LAYOUT_BTNHD && p->dtype != VDA_DTYPE_BF16)
-    return fail(VDA_ERR_UNSUPPORTED, "the token-major layout is supported for bfloat16 inputs only");
+  if (p->test_stall < 0 || p->test_stall > VDA_TEST_STALL_MAX)
+    return fail(VDA_ERR_INVALID_ARG, "unknown test_stall site %d", p->test_stall);
+  if (p->layout == VDA_LAYOUT_BTNHD && p->dtype == VDA_DTYPE_F32)
+    return fail(VDA_ERR_UNSUPPORTED, "the token-major layout is supported for bfloat16 and e4m3 inputs only");
   if (p->dtype == VDA_DTYPE_F32) {
     if (p->d_k % 16 || p->d_v % 16 || p->d_k > 128 || p->d_v > 128)
       return fail(VDA_ERR_UNSUPPORTED,
@@ -51,8 +60,8 @@ vda_status check_problem(const vda_problem* p) {
                   p->d_v);
   } else {
     if (p->d_k != 128 || p->d_v != 128)
-      return fail(VDA_ERR_UNSUPPORTED, "bfloat16 path supports d_k = d_v = 128 (got %d, %d)",
-                  p->d_k, p->d_v);
+      return fail(VDA_ERR_UNSUPPORTED, "%s path supports d_k = d_v = 128 (got %d, %d)",
+                  p->dtype == VDA_DTYPE_E4M3 ? "e4m3" : "bfloat16", p->d_k, p->d_v);
   }
   // Index arithmetic in the kernels: slots and frames fit 32 bits, element
   // offsets are 64-bit.
@@ -68,7 +77,11 @@ vda_status check_problem(const vda_problem* p) {
   return VDA_OK;
 }
 
-size_t elem_size(const vda_problem& p) { return p.dtype == VDA_DTYPE_BF16 ? 2 : 4; }
+// Bytes of one input element, and of one element of O (bfloat16 for e4m3 inputs).
+size_t elem_size(const vda_problem& p) {
+  return p.dtype == VDA_DTYPE_E4M3 ? 1 : p.dtype == VDA_DTYPE_BF16 ? 2 : 4;
+}
+size_t out_elem_size(const vda_problem& p) { return p.dtype == VDA_DTYPE_F32 ? 4 : 2; }
 
 struct Sizes {
   size_t q, k, v, g, kt, vt, o;
@@ -79,7 +92,7 @@ Sizes tensor_bytes(const vda_problem& p) {
   const size_t fr = (size_t)p.B * p.H * p.T * p.n;
   const size_t tx = (size_t)p.B * p.H * p.n_txt;
   return Sizes{fr * p.d_k * es, fr * p.d_k * es, fr * p.d_v * es, fr * p.d_v * es,
-               tx * p.d_k * es, tx * p.d_v * es, fr * p.d_v * es};
+               tx * p.d_k * es, tx * p.d_v * es, fr * p.d_v * out_elem_size(p)};
 }
 
 vda_status check_pointers(const vda_problem& p, const void* Q, const void* K, const void* V,
@@ -98,60 +111,62 @@ vda_status check_pointers(const vda_problem& p, const void* Q, const void* K, co
   return VDA_OK;
 }
 
-template <typename TIn>
-vda_status run_forward(const vda_problem& p, const void* Q, const void* K, const void* V,
-                       const void* G, const void* Kt, const void* Vt, void* O, char* ws,
-                       cudaStream_t st, float* S_fwd, float* S_bwd, cudaEvent_t const* ev) {
+// The float32 path: SIMT Gram, the register-blocked factor, SIMT scan and
+// readout; every state and product in float32.
+vda_status run_forward_f32(const vda_problem& p, const float* q, const float* k, const float* v, const float* g,
+                           const float* kt, const float* vt, float* O, char* ws, cudaStream_t st, float* S_fwd,
+                           float* S_bwd, cudaEvent_t const* ev) {
   const vda::Layout L = vda::make_layout(p);
   unsigned* err = reinterpret_cast<unsigned*>(ws + L.err);
   float* M = reinterpret_cast<float*>(ws + L.M);
   float* C = reinterpret_cast<float*>(ws + L.C);
-  // float32 path: the states live in the workspace unless the caller wants
-  // them.  bf16 path: the workspace holds bf16 states for the readout; the
-  // caller's float32 state buffers, if any, are written besides.
+  // The states live in the workspace unless the caller wants them.
   float* SF = S_fwd ? S_fwd : reinterpret_cast<float*>(ws + L.SF);
   float* SB = S_bwd ? S_bwd : reinterpret_cast<float*>(ws + L.SB);
+  cudaError_t e = cudaMemsetAsync(err, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
+  if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_gram_simt<float>(p, k, v, kt, vt, M, C, st)) != cudaSuccess) return cuda_fail(e, "gram launch");
+  if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_factor(p, M, err, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
+  if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_scan_simt(p, M, C, SF, SB, st)) != cudaSuccess) return cuda_fail(e, "scan launch");
+  if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = vda::launch_readout_simt<float>(p, q, g, SF, SB, O, st)) != cudaSuccess)
+    return cuda_fail(e, "readout launch");
+  if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "event record");
+  return VDA_OK;
+}
+
+// The tensor-core path (bfloat16 or e4m3 inputs, d = 128): the fused
+// Gram+factor kernel (A_t never leaves TMEM), the scan, the readout.  The
+// workspace holds bf16 states for the readout; the caller's float32 state
+// buffers, if any, are written besides.
+vda_status run_forward_tc(const vda_problem& p, const void* q, const void* k, const void* v, const void* g,
+                          const void* kt, const void* vt, void* O, char* ws, cudaStream_t st, float* S_fwd,
+                          float* S_bwd, cudaEvent_t const* ev) {
+  const vda::Layout L = vda::make_layout(p);
+  unsigned* err = reinterpret_cast<unsigned*>(ws + L.err);
+  float* M = reinterpret_cast<float*>(ws + L.M);
+  float* C = reinterpret_cast<float*>(ws + L.C);
   __nv_bfloat16* SFb = reinterpret_cast<__nv_bfloat16*>(ws + L.SF);
   __nv_bfloat16* SBb = reinterpret_cast<__nv_bfloat16*>(ws + L.SB);
   cudaError_t e = cudaMemsetAsync(err, 0, 256, st);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
-  const TIn* q = static_cast<const TIn*>(Q);
-  const TIn* k = static_cast<const TIn*>(K);
-  const TIn* v = static_cast<const TIn*>(V);
-  const TIn* g = static_cast<const TIn*>(G);
-  const TIn* kt = static_cast<const TIn*>(Kt);
-  const TIn* vt = static_cast<const TIn*>(Vt);
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
   if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "event record");
-  constexpr bool kBf16 = std::is_same<TIn, __nv_bfloat16>::value;
-  if constexpr (kBf16) {
-    // Gram and factor in one kernel: M_t and B_t, A_t never leaves TMEM.  The
-    // factor interval between events 1 and 2 is empty on this path.
-    if ((e = vda::launch_gramfactor_tc(p, k, v, kt, vt, M, C, err, st)) != cudaSuccess)
-      return cuda_fail(e, "gram+factor launch");
-  } else {
-    if ((e = vda::launch_gram_simt<TIn>(p, k, v, kt, vt, M, C, st)) != cudaSuccess)
-      return cuda_fail(e, "gram launch");
-  }
+  // Gram and factor in one kernel: the factor interval between events 1 and
+  // 2 is empty on this path.
+  if ((e = vda::launch_gramfactor_tc(p, k, v, kt, vt, M, C, err, st)) != cudaSuccess)
+    return cuda_fail(e, "gram+factor launch");
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "event record");
-  if constexpr (!kBf16) {
-    if ((e = vda::launch_factor(p, M, err, st)) != cudaSuccess) return cuda_fail(e, "factor launch");
-  }
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "event record");
-  if constexpr (kBf16) {
-    if ((e = vda::launch_scan_tc(p, M, C, SFb, SBb, S_fwd, S_bwd, err, st)) != cudaSuccess)
-      return cuda_fail(e, "scan launch");
-  } else {
-    if ((e = vda::launch_scan_simt(p, M, C, SF, SB, st)) != cudaSuccess) return cuda_fail(e, "scan launch");
-  }
+  if ((e = vda::launch_scan_tc(p, M, C, SFb, SBb, S_fwd, S_bwd, err, st)) != cudaSuccess)
+    return cuda_fail(e, "scan launch");
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "event record");
-  if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-    if ((e = vda::launch_readout_tc(p, q, g, SFb, SBb, static_cast<TIn*>(O), err, st)) != cudaSuccess)
-      return cuda_fail(e, "readout launch");
-  } else {
-    if ((e = vda::launch_readout_simt<TIn>(p, q, g, SF, SB, static_cast<TIn*>(O), st)) != cudaSuccess)
-      return cuda_fail(e, "readout launch");
-  }
+  if ((e = vda::launch_readout_tc(p, q, g, SFb, SBb, static_cast<__nv_bfloat16*>(O), err, st)) != cudaSuccess)
+    return cuda_fail(e, "readout launch");
   if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "event record");
   return VDA_OK;
 }
@@ -173,9 +188,9 @@ vda_status forward_impl(const vda_problem* p, const void* Q, const void* K, cons
     return fail(VDA_ERR_INVALID_ARG, "S_fwd / S_bwd not 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  if (p->dtype == VDA_DTYPE_BF16)
-    return run_forward<__nv_bfloat16>(*p, Q, K, V, G, Kt, Vt, O, ws, st, S_fwd, S_bwd, ev);
-  return run_forward<float>(*p, Q, K, V, G, Kt, Vt, O, ws, st, S_fwd, S_bwd, ev);
+  if (p->dtype != VDA_DTYPE_F32) return run_forward_tc(*p, Q, K, V, G, Kt, Vt, O, ws, st, S_fwd, S_bwd, ev);
+  auto f = [](const void* x) { return static_cast<const float*>(x); };
+  return run_forward_f32(*p, f(Q), f(K), f(V), f(G), f(Kt), f(Vt), static_cast<float*>(O), ws, st, S_fwd, S_bwd, ev);
 }
 
 }  // namespace
@@ -338,6 +353,38 @@ vda_status vda_backward_from_forward(const vda_problem* p, const void* Q, const 
                                      size_t workspace_bytes, void* stream) {
   return backward_impl(p, Q, K, V, G, K_txt, V_txt, dO, dQ, dK, dV, dG, dK_txt, dV_txt, workspace, workspace_bytes,
                        stream, true);
+}
+
+vda_status vda_merge_project(const vda_merge_problem* p, const void* O_lin, const void* W_lin, const void* O_sm,
+                             const void* W_sm, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  g_msg[0] = 0;
+  if (!p) return fail(VDA_ERR_INVALID_ARG, "problem is NULL");
+  if (p->tokens < 1 || p->tokens > (1LL << 31) - 256)
+    return fail(VDA_ERR_INVALID_ARG, "tokens must be in [1, 2^31 - 256] (got %lld)", (long long)p->tokens);
+  if (p->K < 64 || p->K % 64) return fail(VDA_ERR_UNSUPPORTED, "K must be a positive multiple of 64 (got %d)", p->K);
+  if (p->D < 8 || p->D % 8) return fail(VDA_ERR_UNSUPPORTED, "D must be a positive multiple of 8 (got %d)", p->D);
+  const void* req[3] = {O_lin, W_lin, Y};
+  const char* names[3] = {"O_lin", "W_lin", "Y"};
+  for (int i = 0; i < 3; ++i) {
+    if (!req[i]) return fail(VDA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(req[i])) return fail(VDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  if ((O_sm == nullptr) != (W_sm == nullptr))
+    return fail(VDA_ERR_INVALID_ARG, "O_sm and W_sm must both be given or both be NULL");
+  if (O_sm && (!aligned16(O_sm) || !aligned16(W_sm)))
+    return fail(VDA_ERR_INVALID_ARG, "O_sm / W_sm not 16-byte aligned");
+  if (!workspace) return fail(VDA_ERR_WORKSPACE, "workspace is NULL");
+  if ((uintptr_t)workspace & 255u) return fail(VDA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (workspace_bytes < 256) return fail(VDA_ERR_WORKSPACE, "workspace has %zu bytes, needs 256", workspace_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  using bf = __nv_bfloat16;
+  e = vda::launch_merge_tc(p->tokens, p->K, p->D, static_cast<const bf*>(O_lin), static_cast<const bf*>(W_lin),
+                           static_cast<const bf*>(O_sm), static_cast<const bf*>(W_sm), static_cast<bf*>(Y),
+                           static_cast<unsigned*>(workspace), st);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return VDA_OK;
 }
 
 vda_status vda_sync_status(void* workspace, void* stream) {

@@ -18,17 +18,13 @@
 //   dK = K (dA + dA^T) + V dB^T,  dV = K dB  (frames and text alike).
 //
 // Steps: the forward's Gram+factor and scan kernels (bf16 states), unless a
-// vda_forward call has just left them in the workspace; the
-// readout's backward in one tensor-core pass over the tokens (dQ, dG, E);
-// the scan kernel once more for both adjoints; the 128 x 128 products as
-// plain batched GEMMs in cuBLAS (one call per product over all frames: bf16
-// adjoints and states for dA, float32 data on TF32 tensor cores for the
-// text's) and element-wise kernels here; then the Gram
-// products' backward in one tensor-core pass over the tokens (dK, dV).
-#include <cublas_v2.h>
-
-#include <mutex>
-
+// vda_forward call has just left them in the workspace; the readout's
+// backward in one tensor-core pass over the tokens (dQ, dG, E); the scan
+// kernel once more for both adjoints (bf16); the 128 x 128 products per
+// frame and the text's small chain in one tensor-core kernel
+// (vda_bwd_operands_tc.cu); then the Gram products' backward in one
+// tensor-core pass over the tokens (dK, dV).  Six launches (four from the
+// forward's state), all on the caller's stream; no library calls.
 #include "sm100.cuh"
 #include "vda_internal.cuh"
 
@@ -57,111 +53,31 @@ __global__ void sum_states_kernel(const uint4* __restrict__ SF, const uint4* __r
   }
 }
 
-// The right-hand operands of the Gram backward, per matrix m: W1 = dA + dA^T
-// and dB = Gf + Gb (Gb null: dB = Gf), bf16, row-major, written to
-// W + m * 2 * 128^2 (W1) and the 128^2 elements after it (dB).  One CTA of
-// 32 x 8 threads per 32 x 32 tile: grid (16, matrices); the transposed tile
-// goes through shared memory so every global access is coalesced.
-__global__ void operands_kernel(const float* __restrict__ dA, const float* __restrict__ Gf,
-                                const float* __restrict__ Gb, __nv_bfloat16* __restrict__ W) {
-  __shared__ float tt[32][33];
-  const size_t m = blockIdx.y;
-  const int r0 = (blockIdx.x / 4) * 32, c0 = (blockIdx.x % 4) * 32;
-  const float* a = dA + m * kMat;
-  const int tx = threadIdx.x, ty = threadIdx.y;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) tt[ty + 8 * i][tx] = a[(size_t)(c0 + ty + 8 * i) * kD + r0 + tx];
-  __syncthreads();
-  __nv_bfloat16* w1 = W + m * 2 * kMat;
-  __nv_bfloat16* db = w1 + kMat;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + ty + 8 * i, c = c0 + tx;
-    const size_t e = (size_t)r * kD + c;
-    w1[e] = __float2bfloat16_rn(a[e] + tt[tx][ty + 8 * i]);
-    db[e] = __float2bfloat16_rn(Gb ? Gf[m * kMat + e] + Gb[m * kMat + e] : Gf[m * kMat + e]);
-  }
-}
-
-// M_0 (fp32, row-major) from the bf16 hi/lo operand image of each head's
-// text slot, and X_0 = Gf_1 + Gb_T.  One CTA per head.
-__global__ void text_inputs_kernel(const uint8_t* __restrict__ Mimg, const float* __restrict__ Gf,
-                                   const float* __restrict__ Gb, float* __restrict__ M0, float* __restrict__ X0,
-                                   int T) {
-  const int bh = blockIdx.x;
-  const uint8_t* img = Mimg + (size_t)bh * (T + 1) * 65536;   // the text slot
-  const float* gf1 = Gf + ((size_t)bh * T + 0) * kMat;
-  const float* gbT = Gb + ((size_t)bh * T + (T - 1)) * kMat;
-  for (int e = threadIdx.x; e < kD * kD; e += blockDim.x) {
-    const int r = e / kD, c = e % kD;
-    const int chunk = c / 8;
-    const uint32_t off = (chunk / 8) * 16384u + sm100::sw128(r, chunk % 8) + (c % 8) * 2;
-    const float hi = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(img + off));
-    const float lo = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(img + 32768 + off));
-    M0[(size_t)bh * kMat + e] = hi + lo;
-    X0[(size_t)bh * kMat + e] = gf1[e] + gbT[e];
-  }
-}
-
-// Per device, created on first use and kept until exit: the cuBLAS handle,
-// and the side stream (non-blocking) with the fork / join events of the
-// text's work.
-struct Blas {
-  std::mutex mu;
-  cublasHandle_t h = nullptr;
-  cudaStream_t side = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-constexpr int kMaxDevices = 64;
-Blas g_blas[kMaxDevices];
-
 int grid_for(size_t count) {
   size_t b = (count + 255) / 256;
   return (int)(b > 148 * 16 ? 148 * 16 : (b ? b : 1));
 }
 
-// Row-major C[m x n] = op(A) op(B) for a batch, through cuBLAS's column-major
-// convention (C^T = op(B)^T op(A)^T).  ta / tb: the row-major operand is used
-// transposed.  Types: bf16 operands with float32 accumulation (C bf16 or
-// float32), or float32 throughout.
-cublasStatus_t gemm_rm(cublasHandle_t h, bool ta, bool tb, int m, int n, int k, float alpha, const void* A,
-                       cudaDataType at, int lda, long long sa, const void* B, cudaDataType bt, int ldb,
-                       long long sb, float beta, void* C, cudaDataType ct, int ldc, long long sc, int batch,
-                       cublasComputeType_t ctype = CUBLAS_COMPUTE_32F) {
-  return cublasGemmStridedBatchedEx(h, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, n, m, k,
-                                    &alpha, B, bt, ldb, sb, A, at, lda, sa, &beta, C, ct, ldc, sc, batch, ctype,
-                                    CUBLAS_GEMM_DEFAULT);
-}
-
 struct BwdLayout {
   Layout fwd;
-  size_t Sb, E, Gf, Gb, GfB, GbB, dA, W, Wt, M0, X0, G0, S0, dA0, total;
+  size_t Sb, E, GfB, GbB, W, Wt, total;
 };
 
 // After the forward's regions (whose M_t, B_t and bf16 states a preceding
 // vda_forward leaves in place): frame-indexed blocks ([frames][128][128]),
-// so each product is one batched call; the text's per-head matrices in
-// blocks of their own.
+// and the text's operand image per head.
 BwdLayout make_bwd_layout(const vda_problem& p) {
   BwdLayout L;
   L.fwd = make_layout(p);
   const size_t bh = (size_t)p.B * p.H, frames = bh * p.T;
   size_t off = L.fwd.total;
   auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 256); return o; };
-  L.Sb = take(frames * kMat * 2);
-  L.E = take(frames * kMat * 4);
-  L.Gf = take(frames * kMat * 4);
-  L.Gb = take(frames * kMat * 4);
-  L.GfB = take(frames * kMat * 2);        // the adjoints as bf16, the dA products' operands
+  L.Sb = take(frames * kMat * 2);         // S = S^f + S^b, bf16
+  L.E = take(frames * kMat * 4);          // E_t = Q_t^T dP_t, float32
+  L.GfB = take(frames * kMat * 2);        // the adjoints, bf16
   L.GbB = take(frames * kMat * 2);
-  L.dA = take(frames * kMat * 4);
   L.W = take(frames * 2 * kMat * 2);      // per frame: W1 | dB, bf16
   L.Wt = take(bh * 2 * kMat * 2);         // per head, the text's
-  L.M0 = take(bh * kMat * 4);
-  L.X0 = take(bh * kMat * 4);
-  L.G0 = take(bh * kMat * 4);
-  L.S0 = take(bh * kMat * 4);
-  L.dA0 = take(bh * kMat * 4);
   L.total = off;
   return L;
 }
@@ -176,8 +92,7 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
                          __nv_bfloat16* dV, __nv_bfloat16* dG, __nv_bfloat16* dKt, __nv_bfloat16* dVt, char* ws,
                          cudaStream_t st, const char** where, bool from_forward) {
   const BwdLayout L = make_bwd_layout(p);
-  const int BH = p.B * p.H, T = p.T, n = p.n, frames = BH * T;
-  const size_t slot_stride = (size_t)(T + 1) * kMat;   // elements between a head's slot blocks
+  const int frames = p.B * p.H * p.T;
   unsigned* err = reinterpret_cast<unsigned*>(ws + L.fwd.err);
   float* M = reinterpret_cast<float*>(ws + L.fwd.M);
   float* Bm = reinterpret_cast<float*>(ws + L.fwd.C);
@@ -185,45 +100,16 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
   __nv_bfloat16* SBb = reinterpret_cast<__nv_bfloat16*>(ws + L.fwd.SB);
   __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(ws + L.Sb);
   float* E = reinterpret_cast<float*>(ws + L.E);
-  float* Gf = reinterpret_cast<float*>(ws + L.Gf);
-  float* Gb = reinterpret_cast<float*>(ws + L.Gb);
   __nv_bfloat16* GfB = reinterpret_cast<__nv_bfloat16*>(ws + L.GfB);
   __nv_bfloat16* GbB = reinterpret_cast<__nv_bfloat16*>(ws + L.GbB);
-  float* dA = reinterpret_cast<float*>(ws + L.dA);
   __nv_bfloat16* W = reinterpret_cast<__nv_bfloat16*>(ws + L.W);
   __nv_bfloat16* Wt = reinterpret_cast<__nv_bfloat16*>(ws + L.Wt);
-  float* M0 = reinterpret_cast<float*>(ws + L.M0);
-  float* X0 = reinterpret_cast<float*>(ws + L.X0);
-  float* G0 = reinterpret_cast<float*>(ws + L.G0);
-  float* S0 = reinterpret_cast<float*>(ws + L.S0);
-  float* dA0 = reinterpret_cast<float*>(ws + L.dA0);
-  const cudaDataType bf = CUDA_R_16BF, f32 = CUDA_R_32F;
   cudaError_t e;
 #define VDA_TRY(expr, what)                 \
   if ((e = (expr)) != cudaSuccess) {        \
     *where = what;                          \
     return e;                               \
   }
-#define VDA_BLAS(expr, what)                            \
-  if ((expr) != CUBLAS_STATUS_SUCCESS) {                \
-    *where = what;                                      \
-    return cudaErrorUnknown;                            \
-  }
-
-  int dev = 0;
-  VDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  Blas& bl = g_blas[dev];
-  std::lock_guard<std::mutex> lock(bl.mu);
-  if (!bl.h) VDA_BLAS(cublasCreate(&bl.h), "cublasCreate");
-  if (!bl.side) {
-    VDA_TRY(cudaStreamCreateWithFlags(&bl.side, cudaStreamNonBlocking), "side stream");
-    VDA_TRY(cudaEventCreateWithFlags(&bl.fork, cudaEventDisableTiming), "fork event");
-    VDA_TRY(cudaEventCreateWithFlags(&bl.join, cudaEventDisableTiming), "join event");
-  }
-  cublasHandle_t h = bl.h;
-  VDA_BLAS(cublasSetStream(h, st), "cublasSetStream");
-  VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
 
   // 1. The forward's M_t, B_t and bf16 states: recomputed, or left in the
   //    workspace by the vda_forward call that preceded this one (whose
@@ -245,49 +131,17 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
 
   // 3. The scans' adjoints: the scan kernel with E (frame-indexed, nothing
   //    at the text step) for B; direction 0 gives Gb (forward in time),
-  //    direction 1 gives Gf.
-  VDA_TRY(launch_scan_tc(p, M, E, GbB, GfB, Gb, Gf, err, st, /*b_frames=*/true), "adjoint scan launch");
+  //    direction 1 gives Gf; bf16, the next step's operands.
+  VDA_TRY(launch_scan_tc(p, M, E, GbB, GfB, nullptr, nullptr, err, st, /*b_frames=*/true), "adjoint scan launch");
 
-  // 4. The text's operands on the side stream (five small launches that
-  //    overlap the frames' work below): G_0 = M_0 (Gf_1 + Gb_T),
-  //    S_0 = M_0 B_0 / lambda, dA_0 = -G_0 S_0^T (TF32 tensor cores).
-  const bool text = p.n_txt > 0;
-  if (text) {
-    VDA_TRY(cudaEventRecord(bl.fork, st), "fork event");
-    VDA_TRY(cudaStreamWaitEvent(bl.side, bl.fork, 0), "fork wait");
-    VDA_BLAS(cublasSetStream(h, bl.side), "cublasSetStream");
-    VDA_BLAS(cublasSetMathMode(h, CUBLAS_TF32_TENSOR_OP_MATH), "cublasSetMathMode");
-    text_inputs_kernel<<<BH, 256, 0, bl.side>>>(reinterpret_cast<const uint8_t*>(M), Gf, Gb, M0, X0, T);
-    VDA_TRY(cudaGetLastError(), "text_inputs launch");
-    VDA_BLAS(gemm_rm(h, false, false, kD, kD, kD, 1.f, M0, f32, kD, kMat, X0, f32, kD, kMat, 0.f, G0, f32, kD, kMat,
-                     BH, CUBLAS_COMPUTE_32F_FAST_TF32), "G_0");
-    VDA_BLAS(gemm_rm(h, false, false, kD, kD, kD, 1.f / p.lambda, M0, f32, kD, kMat, Bm, f32, kD,
-                     (long long)slot_stride, 0.f, S0, f32, kD, kMat, BH, CUBLAS_COMPUTE_32F_FAST_TF32), "S_0");
-    VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, G0, f32, kD, kMat, S0, f32, kD, kMat, 0.f, dA0, f32, kD, kMat,
-                     BH, CUBLAS_COMPUTE_32F_FAST_TF32), "dA_0");
-    operands_kernel<<<dim3(16, BH), dim3(32, 8), 0, bl.side>>>(dA0, G0, nullptr, Wt);
-    VDA_TRY(cudaGetLastError(), "operands launch");
-    VDA_TRY(cudaEventRecord(bl.join, bl.side), "join event");
-    VDA_BLAS(cublasSetMathMode(h, CUBLAS_DEFAULT_MATH), "cublasSetMathMode");
-    VDA_BLAS(cublasSetStream(h, st), "cublasSetStream");
-  }
+  // 4. W1 = dA + dA^T and dB per frame, and the text's W1_0 | dB_0 per head
+  //    (vda_bwd_operands_tc.cu).
+  VDA_TRY(launch_bwd_operands_tc(p, GfB, GbB, SFb, SBb, M, Bm, W, Wt, err, st), "operands launch");
 
-  // 5. dA_t = -(Gf_t S^f_t^T + Gb_t S^b_t^T) from the bf16 adjoints and
-  //    states (float32 accumulation), then W1 = dA + dA^T and dB (from the
-  //    float32 adjoints).
-  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GfB, bf, kD, kMat, SFb, bf, kD, kMat, 0.f, dA, f32, kD, kMat,
-                   frames), "dA (forward part)");
-  VDA_BLAS(gemm_rm(h, false, true, kD, kD, kD, -1.f, GbB, bf, kD, kMat, SBb, bf, kD, kMat, 1.f, dA, f32, kD, kMat,
-                   frames), "dA (backward part)");
-  operands_kernel<<<dim3(16, frames), dim3(32, 8), 0, st>>>(dA, Gf, Gb, W);
-  VDA_TRY(cudaGetLastError(), "operands launch");
-  if (text) VDA_TRY(cudaStreamWaitEvent(st, bl.join, 0), "join wait");
-
-  // 6. dK = K W1 + V dB^T, dV = K dB, for the frames and the text, in one
+  // 5. dK = K W1 + V dB^T, dV = K dB, for the frames and the text, in one
   //    pass over the tokens (vda_gram_bwd_tc.cu).
   VDA_TRY(launch_gram_bwd_tc(p, K, V, W, Kt, Vt, Wt, dK, dV, dKt, dVt, err, st), "gram backward launch");
 #undef VDA_TRY
-#undef VDA_BLAS
   return cudaSuccess;
 }
 

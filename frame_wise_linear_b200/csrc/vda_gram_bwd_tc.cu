@@ -49,6 +49,7 @@ struct GramBwdParams {
   int frames, heads, n, n_txt;
   int tpf, tpt;                   // tiles per frame, per text unit
   TokGeom g;                      // the layout of K, V, dK, dV and the text's
+  int stall;                      // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
 };
 
 struct Shared {
@@ -56,6 +57,7 @@ struct Shared {
   uint64_t d_full[2], t_empty[2];
   uint64_t w_full, w_empty;
   uint64_t drain;
+  uint64_t never;                 // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int abort;
 };
@@ -113,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1) gram_bwd_tc_kernel(const __grid_c
     mbar_init(&sh.w_full, 1);
     mbar_init(&sh.w_empty, 1);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -196,7 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) gram_bwd_tc_kernel(const __grid_c
           cur = r.unit;
         }
         if (!(ok = mbar_wait(&sh.t_empty[tb], ((j >> 1) & 1) ^ 1))) break;
-        if (!(ok = mbar_wait(&sh.kv_full[st], (j >> 1) & 1))) break;
+        const bool stall = p.stall == VDA_TEST_STALL_GBWD_TILE && blockIdx.x == 0 && j == 0;
+        if (!(ok = mbar_wait_or_stall(&sh.kv_full[st], (j >> 1) & 1, &sh.never, stall))) break;
         tc_fence_after();
         const uint32_t ka = kvaddr + st * 2 * kTile, va = ka + kTile;
         const uint32_t dk = tmem + tb * 256, dv = dk + 128;
@@ -237,7 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1) gram_bwd_tc_kernel(const __grid_c
     for (int j = 0; j < J; ++j) {
       const TileRef r = tile_ref(p, t_begin + j);
       const int tb = j & 1;
-      bool ok = !aborted(sh) && mbar_wait(&sh.d_full[tb], (j >> 1) & 1);
+      const bool stall = p.stall == VDA_TEST_STALL_GBWD_STORE && blockIdx.x == 0 && j == 1;
+      bool ok = !aborted(sh) && mbar_wait_or_stall(&sh.d_full[tb], (j >> 1) & 1, &sh.never, stall);
       if (!ok) set_abort(sh, p.err);
       if (named_bar_or(1 + half, 128, !ok)) break;   // one decision per half
       tc_fence_after();
@@ -315,6 +320,7 @@ cudaError_t launch_gram_bwd_tc(const vda_problem& p, const __nv_bfloat16* K, con
   prm.tpf = (p.n + kRows - 1) / kRows;
   prm.tpt = text ? (p.n_txt + kRows - 1) / kRows : 0;
   prm.g = TokGeom{p.layout, p.H, p.T};
+  prm.stall = p.test_stall;
   const size_t smem = 1024 + (3 + 2 * kStages) * kTile + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(gram_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -1,5 +1,5 @@
 // Gram / cross products and the factor step in one kernel, on tcgen05 tensor
-// cores (bf16 inputs, d = 128).
+// cores (bf16 or e4m3 inputs, d = 128).
 //
 // For every slot (b, h, t) -- t = 0 is the text, t = 1..T the frames -- this
 // computes, after "VDN-MiniMax-H3" (aiezz.com), section 03, Video Delta
@@ -9,8 +9,12 @@
 //     M_t = lambda A_t^{-1}                                   (written as bf16 hi + lo)
 // The scan then runs S_t = M_t (S_{t-1} + B_t / lambda).
 //
-// Gram: per 16 tokens, two MMAs into TMEM: A += K^T K and B += K^T V (M = 128
-// features of K, N = 128, K-dim = tokens).
+// Gram: per 16 tokens (bf16, kind::f16) or 32 tokens (e4m3, kind::f8f6f4),
+// two MMAs into TMEM: A += K^T K and B += K^T V (M = 128 features of K, N =
+// 128, K-dim = tokens).  Products of 8-bit floats are exact in the float32
+// accumulator.  With e4m3 inputs (per-tensor scales s_k, s_v) the service
+// warps scale the chains to the values' units (A by s_k^2, B by s_k s_v)
+// before lambda is added and the sweep runs.
 // Factor: A_t stays where the chain left it, in TMEM (lane i = row i), and is
 // swept there: the sweep operator taken 8 pivots at a time in its Cholesky
 // form.  For a pivot block K with P = A_KK = L L^T and X = A[:, K],
@@ -52,9 +56,19 @@ namespace {
 using namespace sm100;
 
 constexpr int kStages = 5;
-constexpr int kChunk = 64;                    // tokens per stage
-constexpr int kBox = 64 * 64 * 2;             // one 64 x 64 bf16 box: 8 KB
-constexpr int kStageBytes = 4 * kBox;         // K lo/hi features, V lo/hi features
+constexpr int kHalfStage = 16384;             // K's part of a stage, then V's
+constexpr int kStageBytes = 2 * kHalfStage;
+// Per input type: tokens per stage and per MMA.  bf16: 64-token chunks, each
+// tensor as two 64-feature boxes (8 KB each), 16 tokens per MMA (kind::f16).
+// e4m3: 128-token chunks, each tensor as one 128-feature box (16 KB), 32
+// tokens per MMA (kind::f8f6f4).  Both fill a 128-byte-swizzled row per token.
+template <bool kF8>
+struct GramCfg {
+  static constexpr int kChunk = kF8 ? 128 : 64;
+  static constexpr int kKTok = kF8 ? 32 : 16;
+  static constexpr int kBoxes = kF8 ? 1 : 2;          // boxes per tensor and stage
+  static constexpr int kBox = kHalfStage / kBoxes;
+};
 constexpr int kFacGroups = 2;                 // factor groups, each sweeping its own slot
 constexpr int kThreads = 32 * (6 + 4 * kFacGroups);
 constexpr int kARegions = 3;                  // TMEM: three 128-column A regions, then B
@@ -65,6 +79,7 @@ constexpr int kEpiBar = 1;                    // named barrier of the B epilogue
 constexpr int kFacBar0 = 2;                   // named barriers of the factor groups: 2, 3
 constexpr int kOp = 128 * 8 * 4;              // factor operand: 128 rows x 8 tf32 (4 KB)
 constexpr uint32_t kIdescGram = idesc_bf16_f32(128, 128, /*a MN*/ true, /*b MN*/ true);
+constexpr uint32_t kIdescGram8 = idesc_e4m3_f32(128, 128, /*a MN*/ true, /*b MN*/ true);
 constexpr uint32_t kIdescUpd = idesc_tf32_f32(128, 128, /*negate A*/ true);
 
 struct GramFactorParams {
@@ -75,6 +90,9 @@ struct GramFactorParams {
   int BH, T, n, n_txt;
   float lam;
   TokGeom g;            // the inputs' layout
+  int stall;            // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
+  float a_scale;        // e4m3 inputs: A = a_scale K8^T K8 + lambda I, B = b_scale K8^T V8 (1 for bf16)
+  float b_scale;
 };
 
 struct Shared {
@@ -88,6 +106,7 @@ struct Shared {
   uint64_t upd[kFacGroups];     // per group, one phase per block step
   uint64_t fdone[kFacGroups];   // per group, one phase per slot: all its MMAs complete
   uint64_t drain;
+  uint64_t never;               // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int bad;
   int abort;
@@ -119,7 +138,10 @@ __device__ __forceinline__ void store_op(uint8_t* op, int i, const float (&v)[8]
   *reinterpret_cast<float4*>(op + 2048 + i * 16) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid_constant__ GramFactorParams p) {
+  using Cfg = GramCfg<kF8>;
+  constexpr int kChunk = Cfg::kChunk;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
@@ -147,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
       mbar_init(&sh.fdone[g], 1);
     }
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.bad = 0;
     sh.abort = 0;
     fence_barrier_init();
@@ -191,10 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
           }
           uint8_t* st = stages + stage * kStageBytes;
           mbar_expect_tx(&sh.full[stage], kStageBytes);
-          tok_load(st + 0 * kBox, mk, &sh.full[stage], p.g, q, 0, r0, pol);
-          tok_load(st + 1 * kBox, mk, &sh.full[stage], p.g, q, 64, r0, pol);
-          tok_load(st + 2 * kBox, mv, &sh.full[stage], p.g, q, 0, r0, pol);
-          tok_load(st + 3 * kBox, mv, &sh.full[stage], p.g, q, 64, r0, pol);
+#pragma unroll
+          for (int b = 0; b < Cfg::kBoxes; ++b) {   // features 64 b.. (bf16), or all 128 (e4m3)
+            tok_load(st + b * Cfg::kBox, mk, &sh.full[stage], p.g, q, 64 * b, r0, pol);
+            tok_load(st + kHalfStage + b * Cfg::kBox, mv, &sh.full[stage], p.g, q, 64 * b, r0, pol);
+          }
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -229,20 +253,27 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         const uint32_t da = tmem + reg * 128, db = tmem + kBCol;
         bool first = true;
         for (int r0 = 0; r0 < rows; r0 += kChunk) {
-          if (!mbar_wait(&sh.full[stage], phase)) {
+          const bool stall = p.stall == VDA_TEST_STALL_GRAM_STAGE && blockIdx.x == 0 && j == 0 && r0 == 0;
+          if (!mbar_wait_or_stall(&sh.full[stage], phase, &sh.never, stall)) {
             set_abort(sh, p.err);
             break;
           }
           tc_fence_after();
           const uint32_t sa = sbase + stage * kStageBytes;
 #pragma unroll
-          for (int k = 0; k < kChunk / 16; ++k) {
-            // 16 tokens = 16 rows of 128 bytes; MN blocks of 64 features 8 KB
-            // apart: K features in boxes 0-1, V features in boxes 2-3.
-            const uint64_t dk = smem_desc(sa + k * 16 * 128, kBox, 1024, kSwizzle128B);
-            const uint64_t dv = smem_desc(sa + 2 * kBox + k * 16 * 128, kBox, 1024, kSwizzle128B);
-            mma_bf16_ss(da, dk, dk, kIdescGram, first ? 0u : 1u);   // A = K^T K
-            mma_bf16_ss(db, dk, dv, kIdescGram, first ? 0u : 1u);   // B = K^T V
+          for (int k = 0; k < kChunk / Cfg::kKTok; ++k) {
+            // kKTok tokens = kKTok rows of 128 bytes, MN-major (features
+            // contiguous).  bf16: MN blocks of 64 features one box apart;
+            // e4m3: one 128-feature block.  K's rows first, then V's.
+            const uint64_t dk = smem_desc(sa + k * Cfg::kKTok * 128, Cfg::kBox, 1024, kSwizzle128B);
+            const uint64_t dv = smem_desc(sa + kHalfStage + k * Cfg::kKTok * 128, Cfg::kBox, 1024, kSwizzle128B);
+            if constexpr (kF8) {
+              mma_f8_ss(da, dk, dk, kIdescGram8, first ? 0u : 1u);   // A = K^T K
+              mma_f8_ss(db, dk, dv, kIdescGram8, first ? 0u : 1u);   // B = K^T V
+            } else {
+              mma_bf16_ss(da, dk, dk, kIdescGram, first ? 0u : 1u);
+              mma_bf16_ss(db, dk, dv, kIdescGram, first ? 0u : 1u);
+            }
             first = false;
           }
           mma_commit(&sh.empty[stage]);
@@ -316,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
       int rows, z;
       bool text;
       slot_info(p, s, rows, z, text);
-      bool ok = !aborted(sh) && mbar_wait(&sh.gdone, j & 1);
+      const bool stall = p.stall == VDA_TEST_STALL_SERVICE_GRAM && blockIdx.x == 0 && j == 0;
+      bool ok = !aborted(sh) && mbar_wait_or_stall(&sh.gdone, j & 1, &sh.never, stall);
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
       if (named_bar_or(kEpiBar, 128, !ok)) {
         live = false;
@@ -339,7 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
         named_bar_sync(kEpiBar, 128);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4*>(stg + sw128(row, q)) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+          *reinterpret_cast<uint4*>(stg + sw128(row, q)) =
+              make_uint4(__float_as_uint(p.b_scale * __uint_as_float(r[4 * q])),
+                         __float_as_uint(p.b_scale * __uint_as_float(r[4 * q + 1])),
+                         __float_as_uint(p.b_scale * __uint_as_float(r[4 * q + 2])),
+                         __float_as_uint(p.b_scale * __uint_as_float(r[4 * q + 3])));
         fence_proxy_async_smem();
         named_bar_sync(kEpiBar, 128);
         if (leader) {
@@ -367,6 +403,24 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             if (c * 32 != c0) tmem_st_32x32b_x32(trow + c * 32, zr);
+        }
+        if (kF8 && rows > 0) {
+          // e4m3: the chain holds K8^T K8 of the stored keys; A in the values'
+          // units is a_scale times that, so the sweep sees A at its true
+          // scale (its diagonal trick keeps 2 - (A^{-1})_ii, which needs A^{-1}
+          // of the true size to keep its digits).
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            if (c * 32 == c0) continue;
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(trow + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(p.a_scale * __uint_as_float(o[q]));
+            tmem_st_32x32b_x32(trow + c * 32, o);
+          }
+#pragma unroll
+          for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(p.a_scale * __uint_as_float(r[q]));
         }
 #pragma unroll
         for (int q = 0; q < 32; ++q)
@@ -410,7 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
 #pragma unroll 1
       for (int K = 0; K < 16; ++K) {
         if (K > 0) {
-          const bool okw = mbar_wait(&sh.upd[g], (K - 1) & 1);
+          const bool stall =
+              p.stall == VDA_TEST_STALL_FACTOR_UPDATE && blockIdx.x == 0 && g == 0 && nslot == 0 && K == 1;
+          const bool okw = mbar_wait_or_stall(&sh.upd[g], (K - 1) & 1, &sh.never, stall);
           if (!okw) set_abort(sh, p.err);
           if (named_bar_or(bar, 128, !okw)) break;   // the same for every thread
           tc_fence_after();
@@ -515,18 +571,20 @@ __global__ void __launch_bounds__(kThreads, 1) gramfactor_tc_kernel(const __grid
 
 }  // namespace
 
-cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                                 const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* M, float* Bm,
-                                 unsigned* err, cudaStream_t st) {
+cudaError_t launch_gramfactor_tc(const vda_problem& p, const void* K, const void* V, const void* Kt, const void* Vt,
+                                 float* M, float* Bm, unsigned* err, cudaStream_t st) {
   if (p.d_k != 128 || p.d_v != 128) return cudaErrorInvalidValue;
+  const bool f8 = p.dtype == VDA_DTYPE_E4M3;
+  const int esz = f8 ? 1 : 2;
+  const int chunk = f8 ? GramCfg<true>::kChunk : GramCfg<false>::kChunk;
   GramFactorParams prm;
   memset(&prm, 0, sizeof(prm));
   const int BH = p.B * p.H;
-  if (!make_tok_map(&prm.mK, K, p.layout, p.B, p.H, p.T, p.n, 64) ||
-      !make_tok_map(&prm.mV, V, p.layout, p.B, p.H, p.T, p.n, 64))
+  if (!make_tok_map(&prm.mK, K, p.layout, p.B, p.H, p.T, p.n, chunk, esz) ||
+      !make_tok_map(&prm.mV, V, p.layout, p.B, p.H, p.T, p.n, chunk, esz))
     return cudaErrorInvalidValue;
-  if (p.n_txt > 0 && (!make_tok_map(&prm.mKt, Kt, p.layout, p.B, p.H, 1, p.n_txt, 64) ||
-                      !make_tok_map(&prm.mVt, Vt, p.layout, p.B, p.H, 1, p.n_txt, 64)))
+  if (p.n_txt > 0 && (!make_tok_map(&prm.mKt, Kt, p.layout, p.B, p.H, 1, p.n_txt, chunk, esz) ||
+                      !make_tok_map(&prm.mVt, Vt, p.layout, p.B, p.H, 1, p.n_txt, chunk, esz)))
     return cudaErrorInvalidValue;
   prm.g = TokGeom{p.layout, p.H, p.T};
   const long long rows = (long long)BH * (p.T + 1) * 128;
@@ -537,16 +595,23 @@ cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, c
   prm.T = p.T;
   prm.n = p.n;
   prm.n_txt = p.n_txt;
+  // e4m3 inputs hold K / scale_k and V / scale_v: the chains accumulate the
+  // stored values' products, and the service warps scale them to the values'
+  // units (A by scale_k^2, B by scale_k scale_v) before anything else reads them.
   prm.lam = p.lambda;
+  prm.a_scale = f8 ? p.scale_k * p.scale_k : 1.f;
+  prm.b_scale = f8 ? p.scale_k * p.scale_v : 1.f;
+  prm.stall = p.test_stall;
   const size_t smem = 1024 + kStages * kStageBytes + 2 * kOutChunk + kFacGroups * (2 * kOp + 8 * 8 * 4) + sizeof(Shared);
-  cudaError_t e = cudaFuncSetAttribute(gramfactor_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = f8 ? gramfactor_tc_kernel<true> : gramfactor_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int slots = BH * (p.T + 1);
   const int grid = slots < sms ? slots : sms;
-  gramfactor_tc_kernel<<<grid, kThreads, smem, st>>>(prm);
+  kern<<<grid, kThreads, smem, st>>>(prm);
   return cudaGetLastError();
 }
 

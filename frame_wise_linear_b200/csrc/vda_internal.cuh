@@ -38,8 +38,8 @@ inline Layout make_layout(const vda_problem& p) {
   L.M = off;    off = align_up(off + slots * p.d_k * p.d_k * sizeof(float), 256);
   L.C = off;    off = align_up(off + slots * p.d_k * p.d_v * sizeof(float), 256);
   // The states for the readout: float32 on the float32 path; bfloat16 (the
-  // readout's MMA operand) on the bfloat16 path.
-  const size_t se = p.dtype == VDA_DTYPE_BF16 ? 2 : sizeof(float);
+  // readout's MMA operand) on the tensor-core paths (bfloat16 and e4m3 inputs).
+  const size_t se = p.dtype != VDA_DTYPE_F32 ? 2 : sizeof(float);
   L.SF = off;   off = align_up(off + frames * p.d_k * p.d_v * se, 256);
   L.SB = off;   off = align_up(off + frames * p.d_k * p.d_v * se, 256);
   L.total = off;
@@ -71,19 +71,17 @@ cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm
                            __nv_bfloat16* SBb, float* SF, float* SB, unsigned* err, cudaStream_t st,
                            bool b_frames = false);
 
-// Gram and factor in one kernel (vda_gramfactor_tc.cu): bf16 inputs,
-// d_k = d_v = 128.  Writes each slot's M_t into M as bf16 hi and lo halves
+// Gram and factor in one kernel (vda_gramfactor_tc.cu): bf16 or e4m3 inputs
+// (p.dtype), d_k = d_v = 128.  Writes each slot's M_t into M as bf16 hi and lo halves
 // (32 KB each) of the K-major, 128-byte-swizzled image of the scan's MMA A
 // operand, and B_t into Bm; A_t stays in TMEM.
-cudaError_t launch_gramfactor_tc(const vda_problem& p, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                                 const __nv_bfloat16* Kt, const __nv_bfloat16* Vt, float* M, float* Bm,
-                                 unsigned* err, cudaStream_t st);
+cudaError_t launch_gramfactor_tc(const vda_problem& p, const void* K, const void* V, const void* Kt, const void* Vt,
+                                 float* M, float* Bm, unsigned* err, cudaStream_t st);
 
-// Tensor-core readout (vda_readout_tc.cu): bf16 Q, G, O, d_k = d_v = 128.
-// SF, SB: the bfloat16 states written by launch_scan_tc.
-cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,
-                              const __nv_bfloat16* SF, const __nv_bfloat16* SB, __nv_bfloat16* O,
-                              unsigned* err, cudaStream_t st);
+// Tensor-core readout (vda_readout_tc.cu): bf16 or e4m3 Q, G (p.dtype), bf16
+// O, d_k = d_v = 128.  SF, SB: the bfloat16 states written by launch_scan_tc.
+cudaError_t launch_readout_tc(const vda_problem& p, const void* Q, const void* G, const __nv_bfloat16* SF,
+                              const __nv_bfloat16* SB, __nv_bfloat16* O, unsigned* err, cudaStream_t st);
 
 // Backward of the gated readout (vda_readout_bwd_tc.cu): bf16 Q, G, dO and
 // S = S^f + S^b ([frames][128][128]); writes dQ and dG (bf16, the tokens'
@@ -100,6 +98,16 @@ cudaError_t launch_gram_bwd_tc(const vda_problem& p, const __nv_bfloat16* K, con
                                const __nv_bfloat16* Wt, __nv_bfloat16* dK, __nv_bfloat16* dV, __nv_bfloat16* dKt,
                                __nv_bfloat16* dVt, unsigned* err, cudaStream_t st);
 
+// The backward's per-frame and per-text operands (vda_bwd_operands_tc.cu):
+// from the bf16 adjoints Gf, Gb and states S^f, S^b ([frames][128][128]),
+// W = [frames][256][128] bf16, W1 = -(Gf S^f^T + S^f Gf^T + Gb S^b^T + S^b
+// Gb^T) rows then dB = Gf + Gb rows; and, when n_txt > 0, Wt = [heads][256]
+// [128] bf16 for the text from M_0 (the M image of slot 0), B_0 and X_0 =
+// Gf_1 + Gb_T.
+cudaError_t launch_bwd_operands_tc(const vda_problem& p, const __nv_bfloat16* Gf, const __nv_bfloat16* Gb,
+                                   const __nv_bfloat16* SF, const __nv_bfloat16* SB, const float* M, const float* Bm,
+                                   __nv_bfloat16* W, __nv_bfloat16* Wt, unsigned* err, cudaStream_t st);
+
 // Backward (vda_backward.cu): bf16 inputs, d_k = d_v = 128.  Workspace bytes,
 // and the whole backward enqueued on `st` (on failure *where names the step);
 // from_forward: the workspace holds what a vda_forward call with the same
@@ -114,14 +122,33 @@ cudaError_t run_backward(const vda_problem& p, const __nv_bfloat16* Q, const __n
 // TMA descriptor of a [items][rows][128] bf16 tensor, boxes of 64 features x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.
 bool make_bf16_rows_map(CUtensorMap* m, const void* ptr, int rows, int items, int box_rows);
-// TMA descriptor of a token tensor (bf16, 128 features) in either layout:
-// layout 0 [B][H][T][rows][128], layout 1 [B][T][rows][H][128] (T = 1 for
-// the text's [B][H][n_txt][128] / [B][n_txt][H][128]).  Layout 0 is the 3-D
-// map (c, r, unit) of make_bf16_rows_map; layout 1 has five dimensions in
-// increasing stride order, (c, h, r, t, b).  Boxes of 64 features x box_rows
-// tokens of one unit, 128-byte swizzle, so a box lands in shared memory as
-// 64 x box_rows in both layouts (vda_tma.cu).
-bool make_tok_map(CUtensorMap* m, const void* ptr, int layout, int B, int H, int T, int rows, int box_rows);
+// The same [items][rows][128] bf16 tensor with boxes of box_cols features x
+// box_rows rows and the swizzle whose span is one box row (box_cols * 2 bytes:
+// 32, 64 or 128) (vda_tma.cu).  False on failure.
+bool make_bf16_box_map(CUtensorMap* m, const void* ptr, int rows, int items, int box_cols, int box_rows,
+                       int swizzle_bytes);
+
+// TMA descriptor of a [rows][cols] bf16 matrix (row stride cols * 2 bytes, a
+// multiple of 16), boxes of 64 columns x box_rows rows with the 128-byte
+// swizzle (vda_tma.cu).  False on failure.
+bool make_bf16_2d_map(CUtensorMap* m, const void* ptr, long long rows, long long cols, int box_cols, int box_rows);
+
+// The branch merge (vda_merge_tc.cu): Y = O_lin W_lin (+ O_sm W_sm when O_sm
+// is not null), bf16 [tokens][K] x [K][D] -> [tokens][D], K a multiple of 64.
+cudaError_t launch_merge_tc(long long tokens, int K, int D, const __nv_bfloat16* O_lin, const __nv_bfloat16* W_lin,
+                            const __nv_bfloat16* O_sm, const __nv_bfloat16* W_sm, __nv_bfloat16* Y, unsigned* err,
+                            cudaStream_t st);
+
+// TMA descriptor of a token tensor (128 features of elem_bytes each: 2 for
+// bf16, 1 for e4m3) in either layout: layout 0 [B][H][T][rows][128], layout
+// 1 [B][T][rows][H][128] (T = 1 for the text's [B][H][n_txt][128] /
+// [B][n_txt][H][128]).  Layout 0 is a 3-D map (c, r, unit); layout 1 has five
+// dimensions in increasing stride order, (c, h, r, t, b).  Boxes of one
+// 128-byte row per token (64 bf16 or 128 e4m3 features) x box_rows tokens of
+// one unit, 128-byte swizzle, so a box lands in shared memory the same way in
+// both layouts (vda_tma.cu).
+bool make_tok_map(CUtensorMap* m, const void* ptr, int layout, int B, int H, int T, int rows, int box_rows,
+                  int elem_bytes = 2);
 
 // TMA descriptor of a [rows][128] float32 matrix, boxes of 32 columns x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.

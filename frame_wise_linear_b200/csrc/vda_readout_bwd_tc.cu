@@ -58,6 +58,7 @@ struct ReadoutBwdParams {
   int n;
   int tiles_per_frame;
   TokGeom g;                      // the layout of Q, G, dO, dQ and dG
+  int stall;                      // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
 };
 
 struct Shared {
@@ -67,6 +68,7 @@ struct Shared {
   uint64_t p_full[kTBufs], dp_full[kTBufs], dq_full[kTBufs], t_empty[kTBufs];
   uint64_t s_full, s_empty, e_empty;
   uint64_t drain;
+  uint64_t never;                 // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int abort;
 };
@@ -80,28 +82,6 @@ __device__ __forceinline__ void set_abort(Shared& sh, unsigned* err) {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// 8 x 8 transpose of 16-byte chunks across the 8 lanes of a group (j = lane
-// % 8): chunk k of lane j becomes chunk j of lane k.  Then the group's 8
-// lanes hold one 128-byte row segment per chunk index, so a store writes
-// whole lines (three butterfly stages of shuffles).
-__device__ __forceinline__ void transpose8(uint4 (&x)[8], int j) {
-#pragma unroll
-  for (int s = 1; s < 8; s <<= 1) {
-    const bool hi = (j & s) != 0;
-#pragma unroll
-    for (int k0 = 0; k0 < 8; ++k0) {
-      if (k0 & s) continue;
-      const int k1 = k0 | s;
-      uint4 t = hi ? x[k0] : x[k1];
-      t.x = __shfl_xor_sync(0xffffffffu, t.x, s);
-      t.y = __shfl_xor_sync(0xffffffffu, t.y, s);
-      t.z = __shfl_xor_sync(0xffffffffu, t.z, s);
-      t.w = __shfl_xor_sync(0xffffffffu, t.w, s);
-      if (hi) x[k0] = t; else x[k1] = t;
-    }
-  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __grid_constant__ ReadoutBwdParams p) {
@@ -139,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
     mbar_init(&sh.s_empty, 1);
     mbar_init(&sh.e_empty, 256);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -214,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
       auto mma_p = [&](int j) -> bool {
         const int tb = j % kTBufs, st = j & 1;
         if (!mbar_wait(&sh.t_empty[tb], ((j / kTBufs) & 1) ^ 1)) return false;
-        if (!mbar_wait(&sh.q_full[st], (j >> 1) & 1)) return false;
+        const bool stall = p.stall == VDA_TEST_STALL_RBWD_TILE && blockIdx.x == 0 && j == 0;
+        if (!mbar_wait_or_stall(&sh.q_full[st], (j >> 1) & 1, &sh.never, stall)) return false;
         tc_fence_after();
         const uint32_t qa = qaddr + st * kTile;
 #pragma unroll
@@ -342,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_bwd_tc_kernel(const __gri
         dq_base = tok_base(p.g, tok_pos(p.g, u, false), p.n, false);
         dq_u = u;
       }
-      bool ok = !aborted(sh) && mbar_wait(&sh.dq_full[tb], (i / kTBufs) & 1);
+      const bool stall = p.stall == VDA_TEST_STALL_RBWD_DQ && blockIdx.x == 0 && i == 0;
+      bool ok = !aborted(sh) && mbar_wait_or_stall(&sh.dq_full[tb], (i / kTBufs) & 1, &sh.never, stall);
       if (!ok) set_abort(sh, p.err);
       if (named_bar_or(1 + half, 128, !ok)) return false;
       tc_fence_after();
@@ -436,6 +419,7 @@ cudaError_t launch_readout_bwd_tc(const vda_problem& p, const __nv_bfloat16* Q, 
   prm.n = p.n;
   prm.tiles_per_frame = (p.n + kRows - 1) / kRows;
   prm.g = TokGeom{p.layout, p.H, p.T};
+  prm.stall = p.test_stall;
   const size_t smem = 1024 + (1 + 3 * kStages) * kTile + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(readout_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -2,7 +2,10 @@
 //     O_t = sigmoid(G_t) * (Q_t (S^f_t + S^b_t))
 // ("VDN-MiniMax-H3" (aiezz.com), section 03, gate fusion item: a
 // content-dependent sigmoid gate on the branch output).  bfloat16 Q, G, O and
-// states, d = 128.
+// states, d = 128; or e4m3 Q and G with per-tensor scales (O and states
+// bfloat16): each Q tile is widened exactly to bfloat16 in shared memory for
+// the MMA (an MMA takes one element type for both operands, and the states
+// stay bfloat16), and G is widened in the epilogue.
 //
 // Precision: Q is exact in bf16; the scan hands over S^f and S^b as bf16,
 // and O = sigmoid(G) * (Q S^f + Q S^b) takes two MMA passes accumulated in
@@ -23,6 +26,9 @@
 //               through a 2-slot shared-memory ring into registers a frame
 //               ahead, then written into the MMA's B operand buffer as soon
 //               as the MMAs release it.
+//   warps 18..19 (e4m3 only) widen each Q tile into the bf16 A ring (freed
+//               by the tile's MMAs); the epilogue stores O from registers
+//               (whole 128-byte row segments after an 8-lane transpose).
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
@@ -45,6 +51,11 @@ constexpr int kPieces = 128 / kPieceRows;    // 8 pieces per frame
 constexpr int kPieceHalf = kPieceRows * 128 * 2;   // 4 KB of S^f (or S^b) per piece
 constexpr int kPiece = 2 * kPieceHalf;       // one staging slot: S^f piece | S^b piece
 constexpr int kThreads = 576;              // 2 control warps + 8 epilogue warps + 8 prep warps
+// e4m3 inputs: Q and G tiles are 16 KB (one 128-byte row per token); two
+// more warps widen each Q tile to the bf16 operand tile (A ring).
+constexpr int kTile8 = kRows * 128;          // 16 KB
+constexpr int kConvWarps = 2;
+constexpr int kThreads8 = kThreads + 32 * kConvWarps;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
 
@@ -53,20 +64,27 @@ struct ReadoutTcParams {
   CUtensorMap mSF, mSB;      // the same states as tiles: 64 columns x 128 rows, 128-byte swizzle
   const __nv_bfloat16* SF;   // [frames][128][128]
   const __nv_bfloat16* SB;
+  __nv_bfloat16* O;          // e4m3 inputs: O stored from registers
   unsigned* err;
   int units;       // B*H*T frames
+  int n;           // tokens per frame
   int tiles_per_unit;
   TokGeom g;       // the layout of Q, G and O
+  int stall;       // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
+  float q_scale;   // e4m3 inputs: the values Q and G stand for are q_scale Q and g_scale G (1 for bf16)
+  float g_scale;
 };
 
 struct Shared {
   uint64_t q_full[kQStages], q_empty[kQStages];
   uint64_t g_full[kGStages], g_empty[kGStages];
   uint64_t t_full[2], t_empty[2];
+  uint64_t a_full[2], a_empty[2];   // e4m3: the widened Q tiles (the MMA's A operand)
   uint64_t sig_full, sig_empty;
   uint64_t p_full[2];   // S staging slots
   uint64_t s0_full;     // the first frame's states, loaded straight into the operand buffer
   uint64_t drain;
+  uint64_t never;       // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int abort;
 };
@@ -82,13 +100,34 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_constant__ ReadoutTcParams p) {
+// Two e4m3 values (low byte first) to two f16 (exact: every e4m3 value is a
+// normal f16 or zero).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(x));
+  return r;
+}
+// Two f16 that came from e4m3 (normal or zero) to two bf16, exactly: the f16
+// exponent and top mantissa bits moved into bf16 position read as the value
+// times 2^-112 (a normal bf16), and the product with 2^112 is exact.
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2_exact(uint32_t h) {
+  const uint32_t bits = ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x77807780u));
+  return r;
+}
+
+template <bool kF8>
+__global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
+    readout_tc_kernel(const __grid_constant__ ReadoutTcParams p) {
+  constexpr int kQT = kF8 ? kTile8 : kTile;         // bytes of one Q (or G) input tile
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sig = base;                              // S^f | S^b
-  uint8_t* qbuf = base + kSig;                      // kQStages tiles
-  uint8_t* gbuf = qbuf + kQStages * kTile;          // kGStages tiles (G in, O out)
-  uint8_t* sstage = gbuf + kGStages * kTile;        // 2 S staging slots
+  uint8_t* qbuf = base + kSig;                      // kQStages input tiles
+  uint8_t* gbuf = qbuf + kQStages * kQT;            // kGStages tiles (bf16: G in, O out; e4m3: G in)
+  uint8_t* abuf = gbuf + kGStages * kQT;            // e4m3: 2 widened Q tiles (the MMA's A ring)
+  uint8_t* sstage = kF8 ? abuf + 2 * kTile : abuf;  // 2 S staging slots
   Shared& sh = *reinterpret_cast<Shared*>(sstage + 2 * kPiece);
 
   const int warp = threadIdx.x / 32;
@@ -100,11 +139,13 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&sh.q_full[i], 1);
-      mbar_init(&sh.q_empty[i], 1);
+      mbar_init(&sh.q_empty[i], kF8 ? 32 * kConvWarps : 1);   // e4m3: the widening threads
+      mbar_init(&sh.a_full[i], 32 * kConvWarps);
+      mbar_init(&sh.a_empty[i], 1);                           // the tile's MMAs are done with it
     }
     for (int i = 0; i < kGStages; ++i) {
       mbar_init(&sh.g_full[i], 1);
-      mbar_init(&sh.g_empty[i], 2);   // one arrival per stored half
+      mbar_init(&sh.g_empty[i], kF8 ? 256 : 2);   // bf16: one arrival per stored half; e4m3: per reader
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.t_full[i], 1);
@@ -116,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     mbar_init(&sh.p_full[1], 1);
     mbar_init(&sh.s0_full, 1);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -155,18 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
           set_abort(sh, p.err);
           break;
         }
-        mbar_expect_tx(&sh.q_full[qs], kTile);
-        tok_load(qbuf + qs * kTile, &p.mQ, &sh.q_full[qs], p.g, q, 0, y, pol);
-        tok_load(qbuf + qs * kTile + kBox, &p.mQ, &sh.q_full[qs], p.g, q, 64, y, pol);
+        mbar_expect_tx(&sh.q_full[qs], kQT);
+        tok_load(qbuf + qs * kQT, &p.mQ, &sh.q_full[qs], p.g, q, 0, y, pol);
+        if (!kF8) tok_load(qbuf + qs * kQT + kBox, &p.mQ, &sh.q_full[qs], p.g, q, 64, y, pol);
         ++q_issued;
         if (++qs == kQStages) { qs = 0; qph ^= 1; }
         if (!mbar_wait(&sh.g_empty[gs], gph ^ 1)) {
           set_abort(sh, p.err);
           break;
         }
-        mbar_expect_tx(&sh.g_full[gs], kTile);
-        tok_load(gbuf + gs * kTile, &p.mG, &sh.g_full[gs], p.g, q, 0, y, pol);
-        tok_load(gbuf + gs * kTile + kBox, &p.mG, &sh.g_full[gs], p.g, q, 64, y, pol);
+        mbar_expect_tx(&sh.g_full[gs], kQT);
+        tok_load(gbuf + gs * kQT, &p.mG, &sh.g_full[gs], p.g, q, 0, y, pol);
+        if (!kF8) tok_load(gbuf + gs * kQT + kBox, &p.mG, &sh.g_full[gs], p.g, q, 64, y, pol);
         ++g_issued;
         if (++gs == kGStages) { gs = 0; gph ^= 1; }
       }
@@ -183,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       int qs = 0, tb = 0;
       uint32_t qph = 0, tph = 0, sph = 0;
       int cur_u = -1;
-      const uint32_t qaddr = smem_u32(qbuf);
+      const uint32_t qaddr = smem_u32(kF8 ? abuf : qbuf);
       const uint32_t saddr = smem_u32(sig);
       for (int tile = t_begin; tile < t_end && !aborted(sh); ++tile) {
         const int u = tile / p.tiles_per_unit;
@@ -193,7 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
           cur_u = u;
         }
         if (!mbar_wait(&sh.t_empty[tb], tph ^ 1)) { set_abort(sh, p.err); break; }
-        if (!mbar_wait(&sh.q_full[qs], qph)) { set_abort(sh, p.err); break; }
+        // The A operand: the bf16 Q tile, or (e4m3) its widened copy.
+        const bool stall = p.stall == VDA_TEST_STALL_READOUT_TILE && blockIdx.x == 0 && tile == t_begin;
+        uint64_t* afull = kF8 ? &sh.a_full[qs] : &sh.q_full[qs];
+        if (!mbar_wait_or_stall(afull, qph, &sh.never, stall)) { set_abort(sh, p.err); break; }
         tc_fence_after();
         const uint32_t d = tmem + tb * 128;
         const uint32_t qa = qaddr + qs * kTile;
@@ -209,7 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
             mma_bf16_ss(d, a, b, kIdesc, (pass | k) ? 1u : 0u);
           }
         }
-        mma_commit(&sh.q_empty[qs]);
+        // bf16: the Q tile is free; e4m3: the widened tile is (the widening
+        // threads free the 8-bit input tile themselves).
+        mma_commit(kF8 ? &sh.a_empty[qs] : &sh.q_empty[qs]);
         mma_commit(&sh.t_full[tb]);
         const bool last_of_unit = (tile + 1 == t_end) || ((tile + 1) / p.tiles_per_unit != u);
         if (last_of_unit) mma_commit(&sh.sig_empty);
@@ -228,58 +275,109 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     const int row = quarter * 32 + lane;      // tile row this thread owns in TMEM
     int gs = 0, tb = 0;
     uint32_t gph = 0, tph = 0;
+    int o_u = -1;                             // e4m3: the unit whose first O row o_base is
+    size_t o_base = 0;
+    const size_t o_stride = tok_row_stride(p.g);
     for (int tile = t_begin; tile < t_end; ++tile) {
       const int u = tile / p.tiles_per_unit;
       const int y = (tile % p.tiles_per_unit) * kRows;
+      const bool stall = p.stall == VDA_TEST_STALL_READOUT_GATE && blockIdx.x == 0 && tile == t_begin + 1;
       bool ok = !aborted(sh) && mbar_wait(&sh.t_full[tb], tph);
-      ok = ok && mbar_wait(&sh.g_full[gs], gph);
+      ok = ok && mbar_wait_or_stall(&sh.g_full[gs], gph, &sh.never, stall);
       if (!ok) set_abort(sh, p.err);
       // One decision for the half's four warps, which meet at its named
       // barrier below: a warp that left alone would strand the others.
       if (named_bar_or(1 + half, 128, !ok)) break;
       tc_fence_after();
-      uint8_t* gt = gbuf + gs * kTile;
-      uint8_t* rowp = gt + half * kBox;
+      const float hq = 0.5f * p.q_scale, hg = 0.5f * p.g_scale;
       const uint32_t taddr = tmem + tb * 128 + half * 64 + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {           // 32 output columns per step
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, r);
-        tmem_ld_wait();
+      if constexpr (kF8) {
+        // G from its 16 KB tile (one 128-byte row per token); O straight from
+        // registers to global memory: the row's 64 columns as eight 16-byte
+        // chunks, transposed across 8-lane groups so that every store writes
+        // whole 128-byte row segments (rows past n skipped).
+        const uint8_t* g8row = gbuf + gs * kQT;
+        uint4 ch[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {          // 8 columns = one 16-byte chunk
-          const uint32_t off = sw128(row, c * 4 + q);
-          const uint4 gv = *reinterpret_cast<const uint4*>(rowp + off);
-          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-          uint32_t ow[4];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, r);
+          tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(&gw[e]);
-            const float g0 = __low2float(g2), g1 = __high2float(g2);
-            // sigmoid(g) d = (1 + tanh(g / 2)) d / 2: one special-function op.
-            const float h0 = 0.5f * __uint_as_float(r[q * 8 + 2 * e]);
-            const float h1 = 0.5f * __uint_as_float(r[q * 8 + 2 * e + 1]);
-            ow[e] = pack_bf16(fmaf(h0, tanh_approx(0.5f * g0), h0), fmaf(h1, tanh_approx(0.5f * g1), h1));
+          for (int q = 0; q < 4; ++q) {
+            const int f0 = half * 64 + c * 32 + q * 8;   // features f0 .. f0 + 7: half a 16-byte chunk
+            const uint2 gv = *reinterpret_cast<const uint2*>(g8row + sw128(row, f0 >> 4) + (f0 & 15));
+            const uint32_t gw[2] = {gv.x, gv.y};
+            uint32_t ow[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)(gw[e >> 1] >> (16 * (e & 1))));
+              const float2 gf = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+              const float h0 = hq * __uint_as_float(r[q * 8 + 2 * e]);
+              const float h1 = hq * __uint_as_float(r[q * 8 + 2 * e + 1]);
+              ow[e] = pack_bf16(fmaf(h0, tanh_approx(hg * gf.x), h0), fmaf(h1, tanh_approx(hg * gf.y), h1));
+            }
+            ch[c * 4 + q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
           }
-          *reinterpret_cast<uint4*>(rowp + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
-      }
-      tc_fence_before();
-      mbar_arrive(&sh.t_empty[tb]);
-      fence_proxy_async_smem();
-      named_bar_sync(1 + half, 128);
-      if (et % 128 == 0) {   // first thread of each half stores that half
-        tok_store(&p.mO, rowp, p.g, tok_pos(p.g, u, false), 64 * half, y);
-        bulk_commit();
-        bulk_wait_read<0>();
+        tc_fence_before();
+        mbar_arrive(&sh.t_empty[tb]);
         mbar_arrive(&sh.g_empty[gs]);
+        transpose8(ch, lane & 7);
+        if (u != o_u) {
+          o_base = tok_base(p.g, tok_pos(p.g, u, false), p.n, false);
+          o_u = u;
+        }
+        const int r0 = quarter * 32 + 8 * (lane >> 3);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int tr = y + r0 + k;
+          if (tr < p.n)
+            *reinterpret_cast<uint4*>(p.O + o_base + (size_t)tr * o_stride + half * 64 + (lane & 7) * 8) = ch[k];
+        }
+      } else {
+        // G is read from, and O written over, the G tile, then stored by TMA.
+        uint8_t* rowp = gbuf + gs * kTile + half * kBox;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {           // 32 output columns per step
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {          // 8 columns = one 16-byte chunk
+            const uint32_t off = sw128(row, c * 4 + q);
+            const uint4 gv = *reinterpret_cast<const uint4*>(rowp + off);
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t ow[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(&gw[e]);
+              // sigmoid(g) d = (1 + tanh(g / 2)) d / 2: one special-function op.
+              const float h0 = hq * __uint_as_float(r[q * 8 + 2 * e]);
+              const float h1 = hq * __uint_as_float(r[q * 8 + 2 * e + 1]);
+              ow[e] = pack_bf16(fmaf(h0, tanh_approx(hg * __low2float(g2)), h0),
+                                fmaf(h1, tanh_approx(hg * __high2float(g2)), h1));
+            }
+            *reinterpret_cast<uint4*>(rowp + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sh.t_empty[tb]);
+        fence_proxy_async_smem();
+        named_bar_sync(1 + half, 128);
+        if (et % 128 == 0) {   // first thread of each half stores that half
+          tok_store(&p.mO, rowp, p.g, tok_pos(p.g, u, false), 64 * half, y);
+          bulk_commit();
+          bulk_wait_read<0>();
+          mbar_arrive(&sh.g_empty[gs]);
+        }
       }
       if (++gs == kGStages) { gs = 0; gph ^= 1; }
       tb ^= 1;
       if (tb == 0) tph ^= 1;
     }
     if (et % 128 == 0) bulk_wait<0>();         // O stores complete before exit
-  } else {
+  } else if (warp < 18) {
     // ------------------------------------------------------------ S prep
     // S^f and S^b (bfloat16) of each frame of this CTA's range, in order.
     // The first frame's go straight into the operand buffer, which is free
@@ -321,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     }
     uint32_t seph = 0;
     int g = 0;                                 // pieces consumed
+    int landed = 0;                            // pieces whose copies are known to have landed
     bool s0_waited = false, stop = false;
     if (u_first <= u_last) {                   // the same for every prep thread
       // The first frame: hand the operand buffer to the MMAs once it has landed.
@@ -343,7 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       bool ok = true;
 #pragma unroll
       for (int j = 0; j < kPieces; ++j, ++g) {
-        ok = ok && mbar_wait(&sh.p_full[g & 1], (g >> 1) & 1);
+        const bool stall = p.stall == VDA_TEST_STALL_READOUT_STATE && blockIdx.x == 0 && g == 0;
+        ok = ok && mbar_wait_or_stall(&sh.p_full[g & 1], (g >> 1) & 1, &sh.never, stall);
+        if (ok) landed = g + 1;
         const uint8_t* f = sstage + (g & 1) * kPiece + prow * 256 + pchunk * 16;
         sf[j] = *reinterpret_cast<const uint4*>(f);
         sb[j] = *reinterpret_cast<const uint4*>(f + kPieceHalf);
@@ -366,7 +467,49 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     }
     if (pt == 0 && first_issued && !s0_waited) mbar_wait(&sh.s0_full, 0);
     if (pt == 0) {   // let the copies still in flight land before exit
-      for (int c = g; c < issued; ++c) mbar_wait(&sh.p_full[c & 1], (c >> 1) & 1);
+      for (int c = landed; c < issued; ++c) mbar_wait(&sh.p_full[c & 1], (c >> 1) & 1);
+    }
+  } else if constexpr (kF8) {
+    // ------------------------------------------------------------ widening (e4m3)
+    // Each thread widens two rows of every Q tile: 128 e4m3 features (one
+    // swizzled 128-byte row) into 128 bf16 (two 64-feature boxes, the MMA's
+    // K-major operand layout), once the tile has landed and the A buffer of
+    // its stage is free (its previous O store has read it).  No named
+    // barrier: each thread leaves on its own failed wait.
+    const int ct = threadIdx.x - kThreads;    // 0..63
+    int qs = 0;
+    uint32_t qph = 0;
+    for (int tile = t_begin; tile < t_end; ++tile) {
+      bool ok = !aborted(sh) && mbar_wait(&sh.q_full[qs], qph);
+      ok = ok && mbar_wait(&sh.a_empty[qs], qph ^ 1);
+      if (!ok) {
+        set_abort(sh, p.err);
+        break;
+      }
+      const uint8_t* src = qbuf + qs * kTile8;
+      uint8_t* dst = abuf + qs * kTile;
+#pragma unroll 1
+      for (int rr = 0; rr < 2; ++rr) {
+        const int row = ct + 64 * rr;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {          // features 16 c .. 16 c + 15
+          const uint4 v = *reinterpret_cast<const uint4*>(src + sw128(row, c));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o[2 * e] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(w[e] & 0xFFFFu)));
+            o[2 * e + 1] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(w[e] >> 16)));
+          }
+          uint8_t* box = dst + (c >> 2) * kBox;   // features 64 (c / 4) ..
+          *reinterpret_cast<uint4*>(box + sw128(row, 2 * (c & 3))) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(box + sw128(row, 2 * (c & 3) + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+      fence_proxy_async_smem();                // visible to the tensor core
+      mbar_arrive(&sh.q_empty[qs]);
+      mbar_arrive(&sh.a_full[qs]);
+      if (++qs == kQStages) { qs = 0; qph ^= 1; }
     }
   }
 
@@ -378,25 +521,33 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
 
 }  // namespace
 
-cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* G,
-                              const __nv_bfloat16* SF, const __nv_bfloat16* SB, __nv_bfloat16* O, unsigned* err,
-                              cudaStream_t st) {
+cudaError_t launch_readout_tc(const vda_problem& p, const void* Q, const void* G, const __nv_bfloat16* SF,
+                              const __nv_bfloat16* SB, __nv_bfloat16* O, unsigned* err, cudaStream_t st) {
+  const bool f8 = p.dtype == VDA_DTYPE_E4M3;
+  const int esz = f8 ? 1 : 2;
   ReadoutTcParams prm;
   memset(&prm, 0, sizeof(prm));
   const int units = p.B * p.H * p.T;
-  if (!make_tok_map(&prm.mQ, Q, p.layout, p.B, p.H, p.T, p.n, kRows) ||
-      !make_tok_map(&prm.mG, G, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+  if (!make_tok_map(&prm.mQ, Q, p.layout, p.B, p.H, p.T, p.n, kRows, esz) ||
+      !make_tok_map(&prm.mG, G, p.layout, p.B, p.H, p.T, p.n, kRows, esz) ||
       !make_tok_map(&prm.mO, O, p.layout, p.B, p.H, p.T, p.n, kRows) ||
       !make_bf16_rows_map(&prm.mSF, SF, 128, units, 128) || !make_bf16_rows_map(&prm.mSB, SB, 128, units, 128))
     return cudaErrorInvalidValue;
   prm.SF = SF;
   prm.SB = SB;
+  prm.O = O;
   prm.err = err;
   prm.units = units;
+  prm.n = p.n;
   prm.tiles_per_unit = (p.n + kRows - 1) / kRows;
   prm.g = TokGeom{p.layout, p.H, p.T};
-  const size_t smem = 1024 + kSig + (kQStages + kGStages) * kTile + 2 * kPiece + sizeof(Shared);
-  cudaError_t e = cudaFuncSetAttribute(readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  prm.stall = p.test_stall;
+  prm.q_scale = f8 ? p.scale_q : 1.f;
+  prm.g_scale = f8 ? p.scale_g : 1.f;
+  const size_t smem = 1024 + kSig + (kQStages + kGStages) * (f8 ? kTile8 : kTile) + (f8 ? 2 * kTile : 0) +
+                      2 * kPiece + sizeof(Shared);
+  auto kern = f8 ? readout_tc_kernel<true> : readout_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -408,7 +559,7 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
   // and G; only the state loads wait for the scan (griddep_wait).
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(f8 ? kThreads8 : kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -416,7 +567,7 @@ cudaError_t launch_readout_tc(const vda_problem& p, const __nv_bfloat16* Q, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, readout_tc_kernel, prm);
+  return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
 }  // namespace vda

@@ -61,12 +61,14 @@ struct ScanTcParams {
   int f32_out;             // also write the float32 states
   int b_frames;            // B is [frames * 128][128] with no text rows; the text step adds nothing
   float lam;
+  int stall;               // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
 };
 
 struct Shared {
   uint64_t m_full[2], m_empty[2];
   uint64_t x_full, d_full, b_full, b_empty;
   uint64_t drain;
+  uint64_t never;          // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int abort;
 };
@@ -98,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   const int bh = blockIdx.z;
   const int T = p.T;
   const size_t slot0 = (size_t)bh * (T + 1);
+  const bool first_cta = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
   auto slot_of = [&](int s) -> size_t { return slot0 + (s == 0 ? 0 : (dir == 0 ? s : T + 1 - s)); };
   // First row of B_s: its slot's, or, for frame-indexed B, its frame's (the
   // text step reads frame 1's rows and the row warps ignore them).
@@ -117,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     mbar_init(&sh.b_full, 1);
     mbar_init(&sh.b_empty, 32 * kRowWarps);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -172,13 +176,25 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       const uint32_t xaddr = smem_u32(xbuf);
       for (int s = 0; s <= T; ++s) {
         const int st = s & 1;
+        // After a timeout the row warps run on without waiting (to keep their
+        // named barrier balanced) and keep arriving on b_empty and x_full, so
+        // those barriers' phases no longer say anything: stop issuing.
+        if (aborted(sh)) break;
         // The row warps have copied B_s into registers: the buffer takes B_{s+1}.
         if (!mbar_wait(&sh.b_empty, s & 1)) {
           set_abort(sh, p.err);
           break;
         }
+        // B_s has landed (b_full's phases move only with this thread's own
+        // loads, so the wait is exact): B_{s+1}'s arrive.expect_tx can never
+        // meet a phase that still waits for B_s's bytes.
+        if (!mbar_wait(&sh.b_full, s & 1)) {
+          set_abort(sh, p.err);
+          break;
+        }
         if (s + 1 <= T) issue_b(s + 1);
-        if (!mbar_wait(&sh.m_full[st], (s >> 1) & 1) || !mbar_wait(&sh.x_full, s & 1)) {
+        const bool stall = p.stall == VDA_TEST_STALL_SCAN_OPERAND && first_cta && s == 1;
+        if (!mbar_wait(&sh.m_full[st], (s >> 1) & 1) || !mbar_wait_or_stall(&sh.x_full, s & 1, &sh.never, stall)) {
           set_abort(sh, p.err);
           break;
         }
@@ -299,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(&sh.x_full);
       if (s >= 2) store_state(s - 1);          // S_{s-1}, still in srow
-      const bool ok = !aborted(sh) && mbar_wait(&sh.d_full, s & 1);
+      const bool stall = p.stall == VDA_TEST_STALL_SCAN_PRODUCT && first_cta && s == 1;
+      const bool ok = !aborted(sh) && mbar_wait_or_stall(&sh.d_full, s & 1, &sh.never, stall);
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
       tc_fence_after();
       {
@@ -342,6 +359,7 @@ cudaError_t launch_scan_tc(const vda_problem& p, const float* M, const float* Bm
   prm.err = err;
   prm.T = p.T;
   prm.lam = p.lambda;
+  prm.stall = p.test_stall;
   const size_t smem = 1024 + 2 * kMBytes + 2 * kXHalf + kSStage + kBBuf + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -19,7 +19,12 @@ can be drawn alone):
   ill-conditioned keys: K_t = L2norm(U_t W + 0.05 E), U_t ~ N(0,1) (n x 8,
   fresh per frame), W ~ N(0,1) (8 x d_k, one per (b, h)), E ~ N(0,1).
 Values are drawn in float32, normalised in float32, then rounded to BF16
-(round to nearest even) for BF16 workloads.
+(round to nearest even) for BF16 workloads.  E4M3 workloads store each tensor
+x as the 8-bit float nearest to x / s (round to nearest even, saturating at
++-448), with one power-of-two scale s per tensor kind chosen from the
+distribution (2^-8 for the unit-norm Q, K rows, 2^-6 for the N(0, 1) V and
+G, 2^-5 for a G of larger spread): the values the device and the oracle see
+are s times the stored 8-bit floats.
 """
 
 from __future__ import annotations
@@ -35,6 +40,7 @@ _STREAM = {"Q": 0, "K": 1, "V": 2, "G": 3, "K_txt": 4, "V_txt": 5, "U": 6, "W": 
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
+DTYPE_E4M3 = 2
 
 
 @dataclasses.dataclass(frozen=True)
@@ -54,14 +60,26 @@ class Workload:
     rank: int = 8
     noise: float = 0.05
 
+    def scales(self) -> dict:
+        """Per-tensor scales of an E4M3 workload (1 for the other types); the text takes K's and V's."""
+        if self.dtype != DTYPE_E4M3:
+            return dict(Q=1.0, K=1.0, V=1.0, G=1.0, K_txt=1.0, V_txt=1.0)
+        qk, v = 2.0 ** -8, 2.0 ** -6
+        g = 2.0 ** -6 if self.g_std <= 1.0 else 2.0 ** -5
+        return dict(Q=qk, K=qk, V=v, G=g, K_txt=qk, V_txt=v)
+
     @property
     def units(self) -> int:
         """(frame, head) units, the metric's counting unit."""
         return self.B * self.H * self.T
 
     def problem(self) -> dict:
-        return dict(B=self.B, H=self.H, T=self.T, n=self.n, n_txt=self.n_txt,
-                    d_k=self.d_k, d_v=self.d_v, dtype=self.dtype, lam=self.lam)
+        d = dict(B=self.B, H=self.H, T=self.T, n=self.n, n_txt=self.n_txt,
+                 d_k=self.d_k, d_v=self.d_v, dtype=self.dtype, lam=self.lam)
+        if self.dtype == DTYPE_E4M3:
+            sc = self.scales()
+            d.update(scale_q=sc["Q"], scale_k=sc["K"], scale_v=sc["V"], scale_g=sc["G"])
+        return d
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -80,6 +98,11 @@ WORKLOADS = {
     "long90": Workload("long90", B=2, H=32, T=90, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16, lam=1.0),
     "long180": Workload("long180", B=2, H=32, T=180, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_BF16,
                         lam=1.0),
+    # The 768p clip with 8-bit (E4M3) Q, K, V, G and text, per-tensor scales, bf16 O.
+    "768p_fp8": Workload("768p_fp8", B=1, H=32, T=45, n=1008, n_txt=256, d_k=128, d_v=128, dtype=DTYPE_E4M3,
+                         lam=1.0),
+    "768p_fp8_h8": Workload("768p_fp8_h8", B=1, H=8, T=45, n=1008, n_txt=256, d_k=128, d_v=128,
+                            dtype=DTYPE_E4M3, lam=1.0),
 }
 
 
@@ -105,10 +128,48 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def widen(x: np.ndarray, dtype: int) -> np.ndarray:
-    """Exact float64 view of an input tensor as stored (BF16 bits or float32)."""
+E4M3_MAX = 448.0
+
+
+def e4m3_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """OCP E4M3 (1 sign, 4 exponent, 3 mantissa bits, bias 7; no infinities,
+    0x7F / 0xFF are NaN) bit patterns to their exact float64 values."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((b & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+# The 127 finite non-negative E4M3 values, increasing with their codes 0x00 .. 0x7E.
+_E4M3_POS = e4m3_bits_to_f64(np.arange(0x7F, dtype=np.uint8))
+
+
+def to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Values to the nearest E4M3 bit patterns (ties to the even code, which is
+    the even mantissa), saturating at +-448; NaN maps to 0x7F."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 0x7E)
+    lo = np.clip(hi - 1, 0, 0x7E)
+    d_hi = _E4M3_POS[hi] - a
+    d_lo = a - _E4M3_POS[lo]
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(np.signbit(x), code | np.uint8(0x80), code)
+    code = np.where(np.isnan(x), np.uint8(0x7F), code)
+    return code.astype(np.uint8)
+
+
+def widen(x: np.ndarray, dtype: int, scale: float = 1.0) -> np.ndarray:
+    """Exact float64 view of an input tensor as stored (BF16 bits, E4M3 bits
+    times the tensor's scale, or float32)."""
     if dtype == DTYPE_BF16:
         return bf16_bits_to_f32(x).astype(np.float64)
+    if dtype == DTYPE_E4M3:
+        return scale * e4m3_bits_to_f64(x)
     return np.asarray(x, dtype=np.float32).astype(np.float64)
 
 
@@ -130,7 +191,7 @@ class Inputs:
         a = getattr(self, name)
         if index is not None:
             a = a[index]
-        return widen(a, self.workload.dtype)
+        return widen(a, self.workload.dtype, self.workload.scales()[name])
 
     def nbytes_in(self) -> int:
         return sum(getattr(self, k).nbytes for k in ("Q", "K", "V", "G", "K_txt", "V_txt"))
@@ -166,12 +227,16 @@ def head_f32(w: Workload, b: int, h: int, seed: int = 0) -> dict:
 
 
 def head_inputs(w: Workload | str, b: int, h: int, seed: int = 0) -> dict:
-    """One (b, h)'s inputs in storage form (BF16 bits as uint16, or float32)."""
+    """One (b, h)'s inputs in storage form (BF16 bits as uint16, E4M3 bits as
+    uint8 of the values over their scale, or float32)."""
     if isinstance(w, str):
         w = WORKLOADS[w]
     f = head_f32(w, b, h, seed)
     if w.dtype == DTYPE_BF16:
         return {k: to_bf16_bits(v) for k, v in f.items()}
+    if w.dtype == DTYPE_E4M3:
+        sc = w.scales()
+        return {k: to_e4m3_bits(v.astype(np.float64) / sc[k]) for k, v in f.items()}
     return {k: np.ascontiguousarray(v, dtype=np.float32) for k, v in f.items()}
 
 
@@ -179,14 +244,15 @@ def head_widened(w: Workload | str, b: int, h: int, seed: int = 0) -> dict:
     """One (b, h)'s inputs as the exact float64 values the device sees."""
     if isinstance(w, str):
         w = WORKLOADS[w]
-    return {k: widen(v, w.dtype) for k, v in head_inputs(w, b, h, seed).items()}
+    sc = w.scales()
+    return {k: widen(v, w.dtype, sc[k]) for k, v in head_inputs(w, b, h, seed).items()}
 
 
 def make_inputs(w: Workload | str, seed: int = 0) -> Inputs:
     """All of a workload's inputs as host numpy arrays (storage dtype)."""
     if isinstance(w, str):
         w = WORKLOADS[w]
-    st = np.uint16 if w.dtype == DTYPE_BF16 else np.float32
+    st = {DTYPE_BF16: np.uint16, DTYPE_E4M3: np.uint8}.get(w.dtype, np.float32)
     shapes = dict(Q=(w.T, w.n, w.d_k), K=(w.T, w.n, w.d_k), V=(w.T, w.n, w.d_v), G=(w.T, w.n, w.d_v),
                   K_txt=(w.n_txt, w.d_k), V_txt=(w.n_txt, w.d_v))
     out = {k: np.empty((w.B, w.H) + s, dtype=st) for k, s in shapes.items()}
@@ -207,7 +273,7 @@ def make_inputs_torch(w: Workload | str, seed: int = 0, device="cuda", pin: bool
     import torch
     if isinstance(w, str):
         w = WORKLOADS[w]
-    tdt = torch.bfloat16 if w.dtype == DTYPE_BF16 else torch.float32
+    tdt = {DTYPE_BF16: torch.bfloat16, DTYPE_E4M3: torch.uint8}.get(w.dtype, torch.float32)
     shapes = dict(Q=(w.T, w.n, w.d_k), K=(w.T, w.n, w.d_k), V=(w.T, w.n, w.d_v), G=(w.T, w.n, w.d_v),
                   K_txt=(w.n_txt, w.d_k), V_txt=(w.n_txt, w.d_v))
     kw = dict(pin_memory=True) if (pin and str(device) == "cpu") else {}

@@ -30,8 +30,17 @@ VDA_ERR_TIMEOUT = 6
 
 VDA_DTYPE_F32 = 0
 VDA_DTYPE_BF16 = 1
+VDA_DTYPE_E4M3 = 2     # 8-bit float inputs with per-tensor scales (uint8 storage); O is bf16
 VDA_LAYOUT_BHTND = 0   # Q, K, V, G, O: [B, H, T, n, d]; text [B, H, n_txt, d]
 VDA_LAYOUT_BTNHD = 1   # Q, K, V, G, O: [B, T*n, H, d]; text [B, n_txt, H, d] (bf16 only)
+
+# Testing hook for the device timeout path (vda_problem.test_stall): the wait
+# named here runs out in the first CTA of its kernel (include/vda.h).
+TEST_STALL_SITES = {
+    "gram_stage": 1, "factor_update": 2, "service_gram": 3, "scan_operand": 4, "scan_product": 5,
+    "readout_tile": 6, "readout_gate": 7, "readout_state": 8, "rbwd_tile": 9, "rbwd_dq": 10,
+    "gbwd_tile": 11, "gbwd_store": 12,
+}
 
 SYMBOLS = (
     "vda_workspace_size",
@@ -44,6 +53,7 @@ SYMBOLS = (
     "vda_backward_workspace_size",
     "vda_backward",
     "vda_backward_from_forward",
+    "vda_merge_project",
     "vda_sync_status",
     "vda_status_string",
     "vda_last_error",
@@ -54,7 +64,13 @@ class vda_problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32),
                 ("n", ctypes.c_int32), ("n_txt", ctypes.c_int32), ("d_k", ctypes.c_int32),
                 ("d_v", ctypes.c_int32), ("dtype", ctypes.c_int32), ("lambda_", ctypes.c_float),
-                ("layout", ctypes.c_int32)]
+                ("layout", ctypes.c_int32), ("test_stall", ctypes.c_int32),
+                ("scale_q", ctypes.c_float), ("scale_k", ctypes.c_float), ("scale_v", ctypes.c_float),
+                ("scale_g", ctypes.c_float)]
+
+
+class vda_merge_problem(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_int64), ("K", ctypes.c_int32), ("D", ctypes.c_int32)]
 
 
 class VdaError(RuntimeError):
@@ -101,6 +117,9 @@ def load(path: str | None = None):
         lib.vda_backward.restype = st
         lib.vda_backward_from_forward.argtypes = [P] + [vp] * 13 + [vp, ctypes.c_size_t, vp]
         lib.vda_backward_from_forward.restype = st
+        lib.vda_merge_project.argtypes = [ctypes.POINTER(vda_merge_problem), vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                          vp]
+        lib.vda_merge_project.restype = st
         lib.vda_sync_status.argtypes = [vp, vp]
         lib.vda_sync_status.restype = st
         lib.vda_status_string.argtypes = [st]
@@ -123,9 +142,11 @@ def _check(status: int, where: str):
         raise VdaError(status, where, load().vda_last_error().decode())
 
 
-def make_problem(B, H, T, n, n_txt, d_k, d_v, dtype, lam, layout=0) -> vda_problem:
+def make_problem(B, H, T, n, n_txt, d_k, d_v, dtype, lam, layout=0, test_stall=0, scale_q=1.0, scale_k=1.0,
+                 scale_v=1.0, scale_g=1.0) -> vda_problem:
     return vda_problem(int(B), int(H), int(T), int(n), int(n_txt), int(d_k), int(d_v), int(dtype),
-                       float(lam), int(layout))
+                       float(lam), int(layout), int(test_stall), float(scale_q), float(scale_k), float(scale_v),
+                       float(scale_g))
 
 
 def _ptr(x) -> int | None:
@@ -220,7 +241,7 @@ VDA_TIMED_EVENTS = 5
 STAGES = ("gram", "factor", "scan", "readout")   # the intervals between the 5 events
 # Kernels one forward launches.  With bf16 inputs the Gram and the factor are
 # one kernel (the "factor" interval is then empty).
-LAUNCHES_PER_FORWARD = {VDA_DTYPE_F32: 4, VDA_DTYPE_BF16: 3}
+LAUNCHES_PER_FORWARD = {VDA_DTYPE_F32: 4, VDA_DTYPE_BF16: 3, VDA_DTYPE_E4M3: 3}
 
 
 def vda_forward_timed(problem, Q, K, V, G, K_txt, V_txt, O, workspace, events, stream=None,
@@ -266,6 +287,18 @@ def vda_forward_noalloc(problem, Q, K, V, G, K_txt, V_txt, O, stream=None, check
     return s
 
 
+def vda_merge_project(tokens, K, D, O_lin, W_lin, O_sm, W_sm, Y, workspace, stream=None, workspace_bytes=None,
+                      check=True) -> int:
+    """Y = O_lin W_lin + O_sm W_sm (bf16 device buffers; O_sm, W_sm may be None)."""
+    p = vda_merge_problem(int(tokens), int(K), int(D))
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    s = load().vda_merge_project(ctypes.byref(p), _ptr(O_lin), _ptr(W_lin), _ptr(O_sm), _ptr(W_sm), _ptr(Y),
+                                 _ptr(workspace), wb, _stream(stream))
+    if check:
+        _check(s, "vda_merge_project")
+    return s
+
+
 def vda_sync_status(workspace, stream=None, check=True) -> int:
     s = load().vda_sync_status(_ptr(workspace), _stream(stream))
     if check:
@@ -285,12 +318,21 @@ def vda_last_error() -> str:
 # Convenience layer (torch tensors in, torch tensor out)
 # ---------------------------------------------------------------------------
 
-def problem_for(Q, K, V, G, K_txt, V_txt, lam) -> vda_problem:
+def problem_for(Q, K, V, G, K_txt, V_txt, lam, scales=None) -> vda_problem:
+    """The problem of torch tensors in the [B, H, T, n, d] layout.  float32 and
+    bfloat16 tensors take their type; uint8 tensors are E4M3 bit patterns and
+    need `scales` = (scale_q, scale_k, scale_v, scale_g)."""
     import torch
+    sc = (1.0, 1.0, 1.0, 1.0)
     if Q.dtype == torch.bfloat16:
         dt = VDA_DTYPE_BF16
     elif Q.dtype == torch.float32:
         dt = VDA_DTYPE_F32
+    elif Q.dtype in (torch.uint8, torch.float8_e4m3fn):
+        dt = VDA_DTYPE_E4M3
+        if scales is None:
+            raise ValueError("E4M3 inputs need scales=(scale_q, scale_k, scale_v, scale_g)")
+        sc = tuple(float(x) for x in scales)
     else:
         raise TypeError(f"unsupported dtype {Q.dtype}")
     for name, x in (("K", K), ("V", V), ("G", G)):
@@ -307,10 +349,12 @@ def problem_for(Q, K, V, G, K_txt, V_txt, lam) -> vda_problem:
     for x in (Q, K, V, G) + ((K_txt, V_txt) if n_txt else ()):
         if not x.is_cuda or not x.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
-    return make_problem(Bn, Hn, T, n, n_txt, d_k, d_v, dt, lam)
+    return make_problem(Bn, Hn, T, n, n_txt, d_k, d_v, dt, lam, scale_q=sc[0], scale_k=sc[1], scale_v=sc[2],
+                        scale_g=sc[3])
 
 
-def forward(Q, K, V, G, K_txt, V_txt, lam: float, stream=None, workspace=None, out=None, check=False):
+def forward(Q, K, V, G, K_txt, V_txt, lam: float, stream=None, workspace=None, out=None, check=False,
+            scales=None):
     """O = VDA(Q, K, V, G, K_txt, V_txt; lam) on the inputs' device.
 
     The call is enqueued on `stream` (default: the current torch stream).  A
@@ -320,7 +364,7 @@ def forward(Q, K, V, G, K_txt, V_txt, lam: float, stream=None, workspace=None, o
     and raises on a device-side condition (VDA_ERR_NOT_SPD, VDA_ERR_TIMEOUT).
     """
     import torch
-    prob = problem_for(Q, K, V, G, K_txt, V_txt, lam)
+    prob = problem_for(Q, K, V, G, K_txt, V_txt, lam, scales)
     ws_bytes = vda_workspace_size(prob)
     s = torch.cuda.current_stream(Q.device) if stream is None else stream
     if not isinstance(s, torch.cuda.Stream):
@@ -328,7 +372,8 @@ def forward(Q, K, V, G, K_txt, V_txt, lam: float, stream=None, workspace=None, o
     with torch.cuda.stream(s):
         if workspace is None or _nbytes(workspace) < ws_bytes:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
-        O = out if out is not None else torch.empty(G.shape, dtype=G.dtype, device=G.device)
+        odt = torch.bfloat16 if prob.dtype == VDA_DTYPE_E4M3 else G.dtype
+        O = out if out is not None else torch.empty(G.shape, dtype=odt, device=G.device)
     txt = prob.n_txt > 0
     vda_forward(prob, Q, K, V, G, K_txt if txt else None, V_txt if txt else None, O, workspace,
                 stream=s)

@@ -31,8 +31,9 @@
  * The gradients of vda_backward* take the layout of their inputs.  In both:
  *     S_fwd, S_bwd (states)          : [B, H, T, d_k, d_v], float32
  * Inputs and O share one element type, vda_problem.dtype: float32 or
- * bfloat16.  The state recurrence and every accumulation are float32; O is
- * rounded to its type with round-to-nearest-even.  With bfloat16 inputs the
+ * bfloat16; with e4m3 inputs (per-tensor scales) O is bfloat16.  The state
+ * recurrence and every accumulation are float32; O is rounded to its type
+ * with round-to-nearest-even.  With bfloat16 inputs the
  * readout takes the two states as bfloat16 operands (O = sigmoid(G) *
  * (Q S^f + Q S^b) with S^f, S^b rounded to bfloat16, accumulated in
  * float32); the states returned by vda_forward_states are the float32 ones.
@@ -74,13 +75,17 @@ typedef enum vda_status {
   VDA_ERR_TIMEOUT = 6       /* device: a bounded wait gave up               */
 } vda_status;
 
-typedef enum vda_dtype { VDA_DTYPE_F32 = 0, VDA_DTYPE_BF16 = 1 } vda_dtype;
+/* Element type of the inputs.  VDA_DTYPE_E4M3: Q, K, V, G, K_txt and V_txt
+ * are 8-bit floats (OCP E4M3: 1 sign, 4 exponent, 3 mantissa bits, bias 7,
+ * largest finite 448, no infinities), each tensor with a per-tensor scale in
+ * vda_problem; O is bfloat16.  The forward only. */
+typedef enum vda_dtype { VDA_DTYPE_F32 = 0, VDA_DTYPE_BF16 = 1, VDA_DTYPE_E4M3 = 2 } vda_dtype;
 
 typedef enum vda_layout { VDA_LAYOUT_BHTND = 0, VDA_LAYOUT_BTNHD = 1 } vda_layout;
 
 /* Problem sizes.  B, H, T, n >= 1; n_txt >= 0.
  * float32: d_k, d_v multiples of 16 in [16, 128].
- * bfloat16: d_k = d_v = 128.
+ * bfloat16, e4m3: d_k = d_v = 128.
  * lambda: the ridge weight of every frame-wise solve, finite and > 0, one
  * value shared by all batches, heads, frames and the text (the pages name no
  * such parameter; one scalar per call is the plainest reading). */
@@ -89,7 +94,42 @@ typedef struct vda_problem {
   int32_t dtype; /* vda_dtype */
   float lambda;
   int32_t layout; /* vda_layout; VDA_LAYOUT_BTNHD needs bfloat16 */
+  int32_t test_stall; /* testing hook, VDA_TEST_STALL_*; 0 in normal use */
+  /* e4m3 inputs only (ignored otherwise): the value an element stands for is
+   * scale times its stored e4m3 value, one scale per tensor (K_txt takes
+   * scale_k, V_txt scale_v); each finite and > 0. */
+  float scale_q, scale_k, scale_v, scale_g;
 } vda_problem;
+
+/* Testing hook for the device timeout path (vda_problem.test_stall).  Every
+ * wait inside the tensor-core kernels is bounded (2 s of the GPU's global
+ * timer); a wait that runs out sets VDA_ERR_TIMEOUT in the error word and the
+ * kernel winds down: its other warps stop at their next decision point, the
+ * copies and MMAs it has issued complete, its tensor memory is released, and
+ * the kernels after it on the stream still end.  A nonzero test_stall names
+ * one wait below; in the first CTA of the kernel that holds it (and only
+ * there), that wait is made on a barrier nothing ever signals, so it runs out
+ * exactly as a wait on a lost signal would.  The call then returns VDA_OK
+ * (enqueued), vda_sync_status() reports VDA_ERR_TIMEOUT, and later calls run
+ * normally.  A site that the problem's sizes never reach (for example the
+ * text chunk when n_txt == 0) leaves the call unchanged.  The sites apply to
+ * the bfloat16 path (the float32 path has no bounded waits). */
+enum {
+  VDA_TEST_STALL_NONE = 0,
+  VDA_TEST_STALL_GRAM_STAGE = 1,     /* Gram+factor: the MMA thread's wait for its first token chunk   */
+  VDA_TEST_STALL_FACTOR_UPDATE = 2,  /* Gram+factor: factor group 0's wait for its first block update  */
+  VDA_TEST_STALL_SERVICE_GRAM = 3,   /* Gram+factor: the service warps' wait for the first Gram chain  */
+  VDA_TEST_STALL_SCAN_OPERAND = 4,   /* scan: the MMA thread's wait for the second step's operand      */
+  VDA_TEST_STALL_SCAN_PRODUCT = 5,   /* scan: the row warps' wait for the second step's product        */
+  VDA_TEST_STALL_READOUT_TILE = 6,   /* readout: the MMA thread's wait for the first Q tile            */
+  VDA_TEST_STALL_READOUT_GATE = 7,   /* readout: the epilogue's wait for the second G tile             */
+  VDA_TEST_STALL_READOUT_STATE = 8,  /* readout: the state warps' wait for the second frame's states   */
+  VDA_TEST_STALL_RBWD_TILE = 9,      /* readout backward: the MMA thread's wait for the first Q tile   */
+  VDA_TEST_STALL_RBWD_DQ = 10,       /* readout backward: the epilogue's wait for the first dQ         */
+  VDA_TEST_STALL_GBWD_TILE = 11,     /* Gram backward: the MMA thread's wait for the first K, V tile   */
+  VDA_TEST_STALL_GBWD_STORE = 12,    /* Gram backward: the epilogue's wait for the second dK, dV       */
+  VDA_TEST_STALL_MAX = 12
+};
 
 /* Bytes of device workspace vda_forward needs for `p` (written to *bytes).
  * Host only, enqueues nothing.  Errors: INVALID_ARG / UNSUPPORTED as for
@@ -192,10 +232,8 @@ vda_status vda_forward_noalloc(const vda_problem* p, const void* Q, const void* 
  * recomputes the forward's transitions and states in `workspace` (at least
  * vda_backward_workspace_size() bytes, 256-byte aligned); its device error
  * word is read by vda_sync_status() as for vda_forward.  Asynchronous on
- * `stream`; the plain batched GEMMs run in cuBLAS, whose handle the library
- * creates per device on first use and keeps until exit, as it does a
- * non-blocking side stream that the text's small steps fork onto and join
- * back from (events) within the call. */
+ * `stream`: every step is one of the library's kernels, enqueued on that
+ * stream only (no library calls, no other streams, no allocation). */
 vda_status vda_backward_workspace_size(const vda_problem* p, size_t* bytes);
 vda_status vda_backward(const vda_problem* p, const void* Q, const void* K, const void* V,
                         const void* G, const void* K_txt, const void* V_txt, const void* dO,
@@ -215,6 +253,28 @@ vda_status vda_backward_from_forward(const vda_problem* p, const void* Q, const 
                                      const void* G, const void* K_txt, const void* V_txt, const void* dO,
                                      void* dQ, void* dK, void* dV, void* dG, void* dK_txt, void* dV_txt,
                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* The merge of the hybrid attention's two branches ("VDN-MiniMax-H3"
+ * (aiezz.com), section 03, gate fusion item, restated in the laicaila.com
+ * page, section 技术原理): each branch has its own content-dependent sigmoid
+ * gate and its own output projection, and the projected branches are summed.
+ * With each gate applied by its branch (vda_forward applies the linear
+ * branch's), this computes
+ *     Y = O_lin W_lin + O_sm W_sm      (float32 accumulation, Y rounded to bf16)
+ * O_lin, O_sm: [tokens, K] bfloat16, row-major (a token's heads concatenated:
+ * the [B, T*n, H, d_v] output of the token-major layout is [B*T*n, H*d_v]);
+ * W_lin, W_sm: [K, D] bfloat16, row-major; Y: [tokens, D] bfloat16.  O_sm and
+ * W_sm are both NULL when there is no softmax branch (Y = O_lin W_lin).
+ * tokens >= 1; K a multiple of 64; D a multiple of 8 (>= 8).  Device
+ * pointers, 16-byte aligned.  workspace: at least 256 bytes of device memory
+ * (256-byte aligned) holding the device error word, which the call clears
+ * and vda_sync_status() reads.  Asynchronous on `stream`. */
+typedef struct vda_merge_problem {
+  int64_t tokens;
+  int32_t K, D;
+} vda_merge_problem;
+vda_status vda_merge_project(const vda_merge_problem* p, const void* O_lin, const void* W_lin, const void* O_sm,
+                             const void* W_sm, void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of
  * `workspace`: VDA_OK, VDA_ERR_NOT_SPD or VDA_ERR_TIMEOUT (first one set),

@@ -41,6 +41,19 @@ def test_every_declared_symbol_is_exported(lib):
         assert name in declared, f"binding exposes {name}, which include/ does not declare"
 
 
+def test_problem_struct_layout():
+    # the header's vda_problem: 15 int32 / float fields, no padding; in a
+    # zeroed struct the fields added after lambda (layout, test_stall, and
+    # the e4m3 scales, which only e4m3 problems read) mean the defaults
+    assert ctypes.sizeof(vda.vda_problem) == 60
+    assert vda.vda_problem.test_stall.offset == 40
+    assert vda.vda_problem.scale_q.offset == 44 and vda.vda_problem.scale_g.offset == 56
+    txt = open(os.path.join(ROOT, "include", "vda.h")).read()
+    assert "VDA_TEST_STALL_MAX = %d" % max(vda.TEST_STALL_SITES.values()) in txt
+    for name, v in vda.TEST_STALL_SITES.items():
+        assert "VDA_TEST_STALL_%s = %d" % (name.upper(), v) in txt
+
+
 def _p(**kw):
     base = dict(B=1, H=2, T=3, n=64, n_txt=8, d_k=128, d_v=128, dtype=vda.VDA_DTYPE_BF16, lam=1.0)
     base.update(kw)
@@ -73,6 +86,12 @@ def test_workspace_size_valid(lib, dtype, state_bytes):
     (dict(dtype=vda.VDA_DTYPE_F32, d_k=24), vda.VDA_ERR_UNSUPPORTED),
     (dict(dtype=vda.VDA_DTYPE_F32, d_k=256), vda.VDA_ERR_UNSUPPORTED),
     (dict(B=70000), vda.VDA_ERR_UNSUPPORTED),
+    (dict(test_stall=-1), vda.VDA_ERR_INVALID_ARG),
+    (dict(dtype=vda.VDA_DTYPE_E4M3, scale_q=0.0), vda.VDA_ERR_INVALID_ARG),
+    (dict(dtype=vda.VDA_DTYPE_E4M3, scale_v=float("inf")), vda.VDA_ERR_INVALID_ARG),
+    (dict(dtype=vda.VDA_DTYPE_E4M3, scale_k=-1.0), vda.VDA_ERR_INVALID_ARG),
+    (dict(dtype=vda.VDA_DTYPE_E4M3, d_k=64, d_v=64), vda.VDA_ERR_UNSUPPORTED),
+    (dict(test_stall=13), vda.VDA_ERR_INVALID_ARG),
 ])
 def test_bad_problem_rejected(lib, kw, status):
     p = _p(**kw)

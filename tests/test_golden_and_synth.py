@@ -104,3 +104,37 @@ def test_token_major_permutation_is_the_documented_layout():
             for r in range(nt):
                 assert torch.equal(yt[b, r, h], xt[b, h, r])
     assert synth.token_major(None) is None
+
+
+def test_e4m3_codec_against_an_independent_implementation():
+    """The 8-bit input format (OCP E4M3): every code decodes as torch's float8_e4m3fn does, and the
+    encoder rounds to nearest with ties to even (saturating at 448) as torch's conversion does."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    mine = synth.e4m3_bits_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    assert np.array_equal(mine[~np.isnan(ref)], ref[~np.isnan(ref)])
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(20000) * np.exp(rng.uniform(-14, 7, 20000))
+    mids = (synth._E4M3_POS[1:] + synth._E4M3_POS[:-1]) / 2          # exact ties
+    x = np.concatenate([x, synth._E4M3_POS, -synth._E4M3_POS, mids, -mids])
+    got = synth.to_e4m3_bits(x)
+    want = torch.from_numpy(np.clip(x, -448.0, 448.0)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, want)
+    assert list(synth.to_e4m3_bits(np.array([460.0, 1e9, -1e9]))) == [0x7E, 0x7E, 0xFE]   # saturation
+    # a few values by hand: 1 = 0 0111 000, 0.5 = 0 0110 000, -2.25 = 1 1000 001, 2^-9 = 0 0000 001
+    assert list(synth.to_e4m3_bits(np.array([1.0, 0.5, -2.25, 2.0 ** -9]))) == [0x38, 0x30, 0xC1, 0x01]
+
+
+def test_e4m3_workload_values_are_scale_times_codes():
+    w = synth.WORKLOADS["768p_fp8"].replace(H=1, T=1, n=16, n_txt=4)
+    raw = synth.head_inputs(w, 0, 0)
+    wide = synth.head_widened(w, 0, 0)
+    f = synth.head_f32(w, 0, 0)
+    for k, sc in w.scales().items():
+        assert raw[k].dtype == np.uint8
+        np.testing.assert_array_equal(wide[k], sc * synth.e4m3_bits_to_f64(raw[k]))
+        # the stored value is within half an 8-bit step (2^-4 relative) of the drawn one
+        big = np.abs(f[k]) > 2.0 ** -6 * sc
+        assert np.all(np.abs(wide[k] - f[k])[big] <= 2.0 ** -4 * np.abs(f[k])[big] + 1e-30)

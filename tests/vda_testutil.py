@@ -5,8 +5,11 @@ import numpy as np
 
 from frame_wise_linear_b200 import synth
 
-# Relative Frobenius tolerance on O (and on the states), by input dtype.
-TOL = {synth.DTYPE_F32: 1e-4, synth.DTYPE_BF16: 2e-2}
+# Relative Frobenius tolerance on O, by input dtype: 1e-4 for float32 inputs,
+# 2e-2 for bfloat16 inputs; E4M3 inputs produce a bfloat16 O through the same
+# bf16 state operands and bf16 output rounding, so they take the bfloat16 bar
+# (the comparison is against the oracle on the exact widened 8-bit inputs).
+TOL = {synth.DTYPE_F32: 1e-4, synth.DTYPE_BF16: 2e-2, synth.DTYPE_E4M3: 2e-2}
 
 
 def rel_fro(a, b) -> float:
@@ -17,7 +20,7 @@ def rel_fro(a, b) -> float:
 
 def to_device(inp: synth.Inputs):
     import torch
-    dt = torch.bfloat16 if inp.workload.dtype == synth.DTYPE_BF16 else torch.float32
+    dt = {synth.DTYPE_BF16: torch.bfloat16, synth.DTYPE_E4M3: torch.uint8}.get(inp.workload.dtype, torch.float32)
 
     def up(a):
         t = torch.from_numpy(np.ascontiguousarray(a))
@@ -36,15 +39,22 @@ def from_device(t) -> np.ndarray:
     return t.detach().cpu().numpy().astype(np.float64)
 
 
+def out_like(w: synth.Workload, G):
+    """An O buffer for the workload: G's shape, float32 or bfloat16 (bfloat16 for E4M3 inputs)."""
+    import torch
+    return torch.empty(G.shape, dtype=torch.float32 if w.dtype == synth.DTYPE_F32 else torch.bfloat16,
+                       device=G.device)
+
+
 def run_gpu(inp: synth.Inputs, states: bool = False):
     """Runs the library on a workload's inputs; returns O (float64) and optionally the states."""
     import torch
     from frame_wise_linear_b200 import vda
     w = inp.workload
     d = to_device(inp)
-    prob = vda.make_problem(w.B, w.H, w.T, w.n, w.n_txt, w.d_k, w.d_v, w.dtype, w.lam)
+    prob = vda.make_problem(**w.problem())
     ws = torch.empty(vda.vda_workspace_size(prob), dtype=torch.uint8, device="cuda")
-    O = torch.empty_like(d["G"])
+    O = out_like(w, d["G"])
     txt = w.n_txt > 0
     kt = d["K_txt"] if txt else None
     vt = d["V_txt"] if txt else None
