@@ -355,6 +355,33 @@ vda_status vda_backward_from_forward(const vda_problem* p, const void* Q, const 
                        stream, true);
 }
 
+vda_status vda_local_softmax(const vda_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                             const void* K_txt, const void* V_txt, void* O, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  g_msg[0] = 0;
+  if (!p) return fail(VDA_ERR_INVALID_ARG, "problem is NULL");
+  vda_problem q = *p;
+  q.lambda = 1.f;   // not read by this branch
+  vda_status s = check_problem(&q);
+  if (s != VDA_OK) return s;
+  if (q.dtype != VDA_DTYPE_BF16)
+    return fail(VDA_ERR_UNSUPPORTED, "the local softmax branch supports bfloat16 inputs only");
+  if ((s = check_pointers(q, Q, K, V, G, K_txt, V_txt, O)) != VDA_OK) return s;
+  if (!workspace) return fail(VDA_ERR_WORKSPACE, "workspace is NULL");
+  if ((uintptr_t)workspace & 255u) return fail(VDA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (workspace_bytes < 256) return fail(VDA_ERR_WORKSPACE, "workspace has %zu bytes, needs 256", workspace_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  using bf = __nv_bfloat16;
+  e = vda::launch_local_softmax_tc(q, static_cast<const bf*>(Q), static_cast<const bf*>(K), static_cast<const bf*>(V),
+                                   static_cast<const bf*>(G), static_cast<const bf*>(K_txt),
+                                   static_cast<const bf*>(V_txt), static_cast<bf*>(O),
+                                   static_cast<unsigned*>(workspace), st);
+  if (e != cudaSuccess) return cuda_fail(e, "local softmax launch");
+  return VDA_OK;
+}
+
 vda_status vda_merge_project(const vda_merge_problem* p, const void* O_lin, const void* W_lin, const void* O_sm,
                              const void* W_sm, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
   g_msg[0] = 0;

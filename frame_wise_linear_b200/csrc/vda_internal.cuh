@@ -139,6 +139,12 @@ cudaError_t launch_merge_tc(long long tokens, int K, int D, const __nv_bfloat16*
                             const __nv_bfloat16* O_sm, const __nv_bfloat16* W_sm, __nv_bfloat16* Y, unsigned* err,
                             cudaStream_t st);
 
+// The local softmax branch (vda_local_softmax_tc.cu): bf16 Q, K, V, G, O in
+// the problem's layout, the text's K_txt, V_txt (skipped when n_txt == 0).
+cudaError_t launch_local_softmax_tc(const vda_problem& p, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                                    const __nv_bfloat16* V, const __nv_bfloat16* G, const __nv_bfloat16* Kt,
+                                    const __nv_bfloat16* Vt, __nv_bfloat16* O, unsigned* err, cudaStream_t st);
+
 // TMA descriptor of a token tensor (128 features of elem_bytes each: 2 for
 // bf16, 1 for e4m3) in either layout: layout 0 [B][H][T][rows][128], layout
 // 1 [B][T][rows][H][128] (T = 1 for the text's [B][H][n_txt][128] /

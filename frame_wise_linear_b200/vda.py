@@ -53,6 +53,7 @@ SYMBOLS = (
     "vda_backward_workspace_size",
     "vda_backward",
     "vda_backward_from_forward",
+    "vda_local_softmax",
     "vda_merge_project",
     "vda_sync_status",
     "vda_status_string",
@@ -117,6 +118,8 @@ def load(path: str | None = None):
         lib.vda_backward.restype = st
         lib.vda_backward_from_forward.argtypes = [P] + [vp] * 13 + [vp, ctypes.c_size_t, vp]
         lib.vda_backward_from_forward.restype = st
+        lib.vda_local_softmax.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.vda_local_softmax.restype = st
         lib.vda_merge_project.argtypes = [ctypes.POINTER(vda_merge_problem), vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                                           vp]
         lib.vda_merge_project.restype = st
@@ -284,6 +287,17 @@ def vda_forward_noalloc(problem, Q, K, V, G, K_txt, V_txt, O, stream=None, check
                                    _ptr(K_txt), _ptr(V_txt), _ptr(O), _stream(stream))
     if check:
         _check(s, "vda_forward_noalloc")
+    return s
+
+
+def vda_local_softmax(problem, Q, K, V, G, K_txt, V_txt, O, workspace, stream=None, workspace_bytes=None,
+                      check=True) -> int:
+    """The local softmax branch: O = sigmoid(G) * windowed softmax attention (bf16 device buffers)."""
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    s = load().vda_local_softmax(ctypes.byref(problem), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(K_txt),
+                                 _ptr(V_txt), _ptr(O), _ptr(workspace), wb, _stream(stream))
+    if check:
+        _check(s, "vda_local_softmax")
     return s
 
 

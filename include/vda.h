@@ -254,6 +254,27 @@ vda_status vda_backward_from_forward(const vda_problem* p, const void* Q, const 
                                      void* dQ, void* dK, void* dV, void* dG, void* dK_txt, void* dV_txt,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* The local softmax branch of the hybrid attention, the linear branch's
+ * partner ("VDN-MiniMax-H3" (aiezz.com), section 03, local softmax branch
+ * item, restated in the laicaila.com page, section 技术原理; the "VDN-H3"
+ * page (comfyui-wiki.com) on the boundary anchors): frames form blocks of 5
+ * and a query token of frame t attends to every token of the frames of
+ * blocks t/5 - 1, t/5 and t/5 + 1 (those that exist), to every token of the
+ * first and last frames (the anchors, visible from every frame), and to every
+ * text token (text dual-branch injection item); the branch's own sigmoid gate
+ * (gate fusion item) is applied to its output:
+ *     O_t = sigmoid(G_t) * softmax(Q_t K_S^T / sqrt(d)) V_S     (per b, h, t)
+ * with S the tokens above.  The problem's sizes and layout as for vda_forward
+ * (bfloat16, d_k = d_v = 128; Q, K, V, G, O in the tokens' layout; K_txt,
+ * V_txt the text's keys and values, NULL when n_txt == 0); lambda is not
+ * read.  Scores, softmax and accumulation in float32; O rounded to bf16.
+ * workspace: at least 256 bytes of device memory (256-byte aligned) holding
+ * the device error word, which the call clears and vda_sync_status() reads.
+ * Asynchronous on `stream`. */
+vda_status vda_local_softmax(const vda_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                             const void* K_txt, const void* V_txt, void* O, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
 /* The merge of the hybrid attention's two branches ("VDN-MiniMax-H3"
  * (aiezz.com), section 03, gate fusion item, restated in the laicaila.com
  * page, section 技术原理): each branch has its own content-dependent sigmoid
