@@ -71,9 +71,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layout", choices=("bhtnd", "btnhd"), default="bhtnd",
                     help="token tensors as [B, H, T, n, d] (default) or token-major [B, T*n, H, d]")
-    ap.add_argument("--direction", choices=("forward", "backward", "merge"), default="forward",
+    ap.add_argument("--direction", choices=("forward", "backward", "merge", "softmax"), default="forward",
                     help="backward: time vda_backward (the gradients); merge: time vda_merge_project (both "
-                         "branches' output projections, summed); separate lines, not the headline")
+                         "branches' output projections, summed); softmax: time vda_local_softmax (the local "
+                         "softmax branch); separate lines, not the headline")
     return ap.parse_args()
 
 
@@ -702,6 +703,78 @@ def run_merge(args, w):
     return 0
 
 
+SOFTMAX_METRIC = "local softmax branch frames*heads/sec at 768p shape; % of B200 bf16 peak"
+
+
+def softmax_work(w):
+    """Tensor flops of the local softmax branch over the workload: per (b, h, t) query frame, Q K^T and P V over
+    its keys (the tokens of its key frames and the text): 4 n keys d."""
+    def key_frame_count(t, T, block=5):   # the window's frames and the anchors 0 and T - 1
+        b = t // block
+        lo, hi = max(0, (b - 1) * block), min(T, (b + 2) * block)
+        return (hi - lo) + (lo > 0) + (hi < T)
+    keys = sum(w.n * key_frame_count(t, w.T) + w.n_txt for t in range(w.T))
+    return 4.0 * w.B * w.H * w.n * keys * w.d_k
+
+
+def run_softmax(args, w):
+    """K timed vda_local_softmax calls on one GPU over the workload's shapes (the branch's own Q, K, V, G)."""
+    import torch
+    from frame_wise_linear_b200 import build as _build
+    from frame_wise_linear_b200 import synth, vda
+    if args.gpus != 1:
+        raise SystemExit("--direction softmax runs on one GPU")
+    dev = torch.device("cuda", 0)
+    _build.build()
+    vda.load()
+    peaks, peaks_kind = load_peaks()
+    d = synth.make_inputs_torch(w, seed=0, device=dev)
+    prob = vda.make_problem(**w.problem())
+    O = torch.empty_like(d["G"])
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kt, vt = (d["K_txt"], d["V_txt"]) if w.n_txt else (None, None)
+
+    def step():
+        vda.vda_local_softmax(prob, d["Q"], d["K"], d["V"], d["G"], kt, vt, O, ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    vda.vda_sync_status(ws, stream=stream)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    vda.vda_sync_status(ws, stream=stream)
+    ms = a.elapsed_time(b) / args.steps
+    tf = softmax_work(w) / (ms / 1e3) / 1e12
+    line = {
+        "metric": SOFTMAX_METRIC, "direction": "softmax", "value": job_value(w.units, 1, ms), "unit": UNIT,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, 1),
+        "roofline": {"kernel": "local_softmax_tc_kernel", "bound": "tensor", "achieved": tf,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json bf16_tflops)", "traffic": None,
+                     "flops": softmax_work(w)},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     from frame_wise_linear_b200 import synth
@@ -712,6 +785,8 @@ def main():
         return run_backward(args, w)
     if args.direction == "merge":
         return run_merge(args, w)
+    if args.direction == "softmax":
+        return run_softmax(args, w)
     return run_b200(args, w)
 
 

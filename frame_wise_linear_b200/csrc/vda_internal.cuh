@@ -150,11 +150,11 @@ cudaError_t launch_local_softmax_tc(const vda_problem& p, const __nv_bfloat16* Q
 // 1 [B][T][rows][H][128] (T = 1 for the text's [B][H][n_txt][128] /
 // [B][n_txt][H][128]).  Layout 0 is a 3-D map (c, r, unit); layout 1 has five
 // dimensions in increasing stride order, (c, h, r, t, b).  Boxes of one
-// 128-byte row per token (64 bf16 or 128 e4m3 features) x box_rows tokens of
-// one unit, 128-byte swizzle, so a box lands in shared memory the same way in
-// both layouts (vda_tma.cu).
+// box_bytes row per token (by default 128 bytes: 64 bf16 or 128 e4m3
+// features) x box_rows tokens of one unit, with the swizzle of that span, so
+// a box lands in shared memory the same way in both layouts (vda_tma.cu).
 bool make_tok_map(CUtensorMap* m, const void* ptr, int layout, int B, int H, int T, int rows, int box_rows,
-                  int elem_bytes = 2);
+                  int elem_bytes = 2, int box_bytes = 128);
 
 // TMA descriptor of a [rows][128] float32 matrix, boxes of 32 columns x
 // box_rows rows with the 128-byte swizzle (vda_tma.cu).  False on failure.

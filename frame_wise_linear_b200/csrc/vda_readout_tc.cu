@@ -27,8 +27,8 @@
 //               ahead, then written into the MMA's B operand buffer as soon
 //               as the MMAs release it.
 //   warps 18..19 (e4m3 only) widen each Q tile into the bf16 A ring (freed
-//               by the tile's MMAs); the epilogue stores O from registers
-//               (whole 128-byte row segments after an 8-lane transpose).
+//               by the tile's MMAs); the epilogue stores O through an 8 KB
+//               staging box per column half (32-column TMA stores).
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
@@ -54,6 +54,7 @@ constexpr int kThreads = 576;              // 2 control warps + 8 epilogue warps
 // e4m3 inputs: Q and G tiles are 16 KB (one 128-byte row per token); two
 // more warps widen each Q tile to the bf16 operand tile (A ring).
 constexpr int kTile8 = kRows * 128;          // 16 KB
+constexpr int kOStage = kRows * 32 * 2;      // 128 rows x 32 bf16 columns: 8 KB
 constexpr int kConvWarps = 2;
 constexpr int kThreads8 = kThreads + 32 * kConvWarps;
 constexpr uint32_t kTmemCols = 256;
@@ -64,7 +65,6 @@ struct ReadoutTcParams {
   CUtensorMap mSF, mSB;      // the same states as tiles: 64 columns x 128 rows, 128-byte swizzle
   const __nv_bfloat16* SF;   // [frames][128][128]
   const __nv_bfloat16* SB;
-  __nv_bfloat16* O;          // e4m3 inputs: O stored from registers
   unsigned* err;
   int units;       // B*H*T frames
   int n;           // tokens per frame
@@ -100,6 +100,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Byte offset of 16-byte chunk `chunk` (0..3) of row `row` in a 64-byte-
+// swizzled box (rows of 64 bytes, 512-byte atoms, 512-byte aligned).
+__device__ __forceinline__ uint32_t sw64(uint32_t row, uint32_t chunk) {
+  return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
+}
+
 // Two e4m3 values (low byte first) to two f16 (exact: every e4m3 value is a
 // normal f16 or zero).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
@@ -128,7 +134,8 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
   uint8_t* gbuf = qbuf + kQStages * kQT;            // kGStages tiles (bf16: G in, O out; e4m3: G in)
   uint8_t* abuf = gbuf + kGStages * kQT;            // e4m3: 2 widened Q tiles (the MMA's A ring)
   uint8_t* sstage = kF8 ? abuf + 2 * kTile : abuf;  // 2 S staging slots
-  Shared& sh = *reinterpret_cast<Shared*>(sstage + 2 * kPiece);
+  uint8_t* ostage = sstage + 2 * kPiece;            // e4m3: an 8 KB O staging box per column half
+  Shared& sh = *reinterpret_cast<Shared*>(ostage + (kF8 ? 2 * kOStage : 0));
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -275,9 +282,6 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
     const int row = quarter * 32 + lane;      // tile row this thread owns in TMEM
     int gs = 0, tb = 0;
     uint32_t gph = 0, tph = 0;
-    int o_u = -1;                             // e4m3: the unit whose first O row o_base is
-    size_t o_base = 0;
-    const size_t o_stride = tok_row_stride(p.g);
     for (int tile = t_begin; tile < t_end; ++tile) {
       const int u = tile / p.tiles_per_unit;
       const int y = (tile % p.tiles_per_unit) * kRows;
@@ -292,17 +296,18 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
       const float hq = 0.5f * p.q_scale, hg = 0.5f * p.g_scale;
       const uint32_t taddr = tmem + tb * 128 + half * 64 + ((uint32_t)(quarter * 32) << 16);
       if constexpr (kF8) {
-        // G from its 16 KB tile (one 128-byte row per token); O straight from
-        // registers to global memory: the row's 64 columns as eight 16-byte
-        // chunks, transposed across 8-lane groups so that every store writes
-        // whole 128-byte row segments (rows past n skipped).
+        // G from its 16 KB tile (one 128-byte row per token); O through the
+        // half's 8 KB staging box, 32 columns (64-byte rows) at a time, by
+        // TMA stores (rows past n clipped).
         const uint8_t* g8row = gbuf + gs * kQT;
-        uint4 ch[8];
-#pragma unroll
+        uint8_t* ostg = ostage + half * kOStage;
+        const bool leader = et % 128 == 0;
+#pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(taddr + c * 32, r);
           tmem_ld_wait();
+          uint4 ch[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int f0 = half * 64 + c * 32 + q * 8;   // features f0 .. f0 + 7: half a 16-byte chunk
@@ -317,23 +322,23 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
               const float h1 = hq * __uint_as_float(r[q * 8 + 2 * e + 1]);
               ow[e] = pack_bf16(fmaf(h0, tanh_approx(hg * gf.x), h0), fmaf(h1, tanh_approx(hg * gf.y), h1));
             }
-            ch[c * 4 + q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            ch[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
           }
-        }
-        tc_fence_before();
-        mbar_arrive(&sh.t_empty[tb]);
-        mbar_arrive(&sh.g_empty[gs]);
-        transpose8(ch, lane & 7);
-        if (u != o_u) {
-          o_base = tok_base(p.g, tok_pos(p.g, u, false), p.n, false);
-          o_u = u;
-        }
-        const int r0 = quarter * 32 + 8 * (lane >> 3);
+          if (c == 1) {
+            tc_fence_before();
+            mbar_arrive(&sh.t_empty[tb]);
+            mbar_arrive(&sh.g_empty[gs]);
+          }
+          if (leader) bulk_wait_read<0>();       // the half's previous store has read the box
+          named_bar_sync(1 + half, 128);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int tr = y + r0 + k;
-          if (tr < p.n)
-            *reinterpret_cast<uint4*>(p.O + o_base + (size_t)tr * o_stride + half * 64 + (lane & 7) * 8) = ch[k];
+          for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(ostg + sw64(row, q)) = ch[q];
+          fence_proxy_async_smem();
+          named_bar_sync(1 + half, 128);
+          if (leader) {
+            tok_store(&p.mO, ostg, p.g, tok_pos(p.g, u, false), 64 * half + 32 * c, y);
+            bulk_commit();
+          }
         }
       } else {
         // G is read from, and O written over, the G tile, then stored by TMA.
@@ -530,12 +535,11 @@ cudaError_t launch_readout_tc(const vda_problem& p, const void* Q, const void* G
   const int units = p.B * p.H * p.T;
   if (!make_tok_map(&prm.mQ, Q, p.layout, p.B, p.H, p.T, p.n, kRows, esz) ||
       !make_tok_map(&prm.mG, G, p.layout, p.B, p.H, p.T, p.n, kRows, esz) ||
-      !make_tok_map(&prm.mO, O, p.layout, p.B, p.H, p.T, p.n, kRows) ||
+      !make_tok_map(&prm.mO, O, p.layout, p.B, p.H, p.T, p.n, kRows, 2, f8 ? 64 : 128) ||
       !make_bf16_rows_map(&prm.mSF, SF, 128, units, 128) || !make_bf16_rows_map(&prm.mSB, SB, 128, units, 128))
     return cudaErrorInvalidValue;
   prm.SF = SF;
   prm.SB = SB;
-  prm.O = O;
   prm.err = err;
   prm.units = units;
   prm.n = p.n;
@@ -545,7 +549,7 @@ cudaError_t launch_readout_tc(const vda_problem& p, const void* Q, const void* G
   prm.q_scale = f8 ? p.scale_q : 1.f;
   prm.g_scale = f8 ? p.scale_g : 1.f;
   const size_t smem = 1024 + kSig + (kQStages + kGStages) * (f8 ? kTile8 : kTile) + (f8 ? 2 * kTile : 0) +
-                      2 * kPiece + sizeof(Shared);
+                      2 * kPiece + (f8 ? 2 * kOStage : 0) + sizeof(Shared);
   auto kern = f8 ? readout_tc_kernel<true> : readout_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -65,14 +65,19 @@ bool make_bf16_2d_map(CUtensorMap* m, const void* ptr, long long rows, long long
 }
 
 bool make_tok_map(CUtensorMap* m, const void* ptr, int layout, int B, int H, int T, int rows, int box_rows,
-                  int elem_bytes) {
+                  int elem_bytes, int box_bytes) {
   auto fn = encode_fn();
   if (!fn || B < 1 || H < 1 || T < 1 || rows < 1 || box_rows < 1 || box_rows > 256) return false;
   if (elem_bytes != 1 && elem_bytes != 2) return false;
-  // A box row is always 128 bytes: 64 bf16 features or 128 e4m3 features.
+  // A box row is box_bytes (128 by default: 64 bf16 or 128 e4m3 features),
+  // with the swizzle of that span.
+  if (box_bytes != 32 && box_bytes != 64 && box_bytes != 128) return false;
+  const CUtensorMapSwizzle sw = box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const cuuint64_t row = 128 * (cuuint64_t)elem_bytes;   // one token's 128 features, bytes
-  const cuuint32_t inner = 128 / elem_bytes;              // features per box row
+  const cuuint32_t inner = box_bytes / elem_bytes;        // features per box row
   cuuint64_t dims[5], strides[4];
   cuuint32_t box[5];
   int rank;
@@ -94,9 +99,8 @@ bool make_tok_map(CUtensorMap* m, const void* ptr, int layout, int B, int H, int
     for (int i = 0; i < 4; ++i) strides[i] = s[i];
   }
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return fn(m, dt, rank, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, rank, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_f32_rows_map(CUtensorMap* m, const void* ptr, long long rows, int box_rows) {
