@@ -459,6 +459,10 @@ def run_b200(args, w):
             "stage_timing": "a second timed region of K vda_forward_timed calls (CUDA events between the "
                             "kernels), %.4f ms per step" % (max_over_ranks(ms_instrumented, pg, dev) / args.steps)}
 
+    # The training direction beside the headline (bf16 only): the backward on the state one forward
+    # left in a backward-sized workspace, and forward + backward steps, K each, CUDA events on the stream.
+    path["backward"] = backward_extras(args, w, d, prob, kt, vt, stream, dev, pg) if w.dtype == 1 else None
+
     # end-to-end through host buffers (pinned), copies inside the timed region
     e2e_steps = args.e2e_steps if args.e2e_steps is not None else min(args.steps, 10)
     if e2e_steps <= 0:
@@ -490,6 +494,62 @@ def run_b200(args, w):
     return finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks)
 
 
+def backward_extras(args, w, d, prob, kt, vt, stream, dev, pg):
+    """ms per vda_backward_from_forward call after one vda_forward, and per training step (vda_forward +
+    vda_backward_from_forward), over K calls each (max over ranks); the backward's roofline fraction."""
+    import torch
+    from frame_wise_linear_b200 import synth, vda
+    rank = dist_env()[1]
+    dO = synth.grad_out_torch(w, seed=rank, device=dev)
+    if prob.layout:
+        dO = synth.token_major(dO)
+    wsb = torch.empty(vda.vda_backward_workspace_size(prob), dtype=torch.uint8, device=dev)
+    outs = [torch.empty_like(d[k]) for k in ("Q", "K", "V", "G")]
+    touts = [torch.empty_like(d["K_txt"]), torch.empty_like(d["V_txt"])] if w.n_txt else [None, None]
+    O2 = torch.empty_like(d["G"])
+    ins = (prob, d["Q"], d["K"], d["V"], d["G"], kt, vt)
+
+    def fwd():
+        vda.vda_forward(*ins, O2, wsb, stream=stream)
+
+    def bwd():
+        vda.vda_backward_from_forward(*ins, dO, *outs, *touts, wsb, stream=stream)
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(a.elapsed_time(b) / args.steps, pg, dev)
+
+    fwd()
+    ms_bwd = timed(bwd)
+
+    def train():
+        fwd()
+        bwd()
+
+    ms_train = timed(train)
+    vda.vda_sync_status(wsb, stream=stream)
+    peaks, _ = load_peaks()
+    rf = backward_roofline(w, peaks)
+    del wsb, outs, touts, dO, O2
+    torch.cuda.empty_cache()
+    return {"from_forward_ms": ms_bwd, "from_forward_frac": rf["t_roof_s"] / (ms_bwd / 1e3),
+            "train_step_ms": ms_train,
+            "train_step_value": job_value(w.units, dist_env()[0], ms_train),
+            "calls": "vda_backward_from_forward after one vda_forward; train step = vda_forward + "
+                     "vda_backward_from_forward; K calls each, CUDA events on the launching stream"}
+
+
 def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
     from frame_wise_linear_b200 import vda
     line = {
@@ -499,6 +559,9 @@ def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
         "config": config_of(w, ws_n, LAYOUTS[args.layout]), "roofline": roof, "roofline_path": path, "e2e": e2e,
         "clocks": clocks, "gpu_launches": vda.LAUNCHES_PER_FORWARD[w.dtype] * args.steps,
     }
+    bwd = path.pop("backward", None) if isinstance(path, dict) else None
+    if bwd is not None:
+        line["backward"] = bwd
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         v, threads, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",

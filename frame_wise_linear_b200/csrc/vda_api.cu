@@ -390,6 +390,9 @@ vda_status vda_merge_project(const vda_merge_problem* p, const void* O_lin, cons
     return fail(VDA_ERR_INVALID_ARG, "tokens must be in [1, 2^31 - 256] (got %lld)", (long long)p->tokens);
   if (p->K < 64 || p->K % 64) return fail(VDA_ERR_UNSUPPORTED, "K must be a positive multiple of 64 (got %d)", p->K);
   if (p->D < 8 || p->D % 8) return fail(VDA_ERR_UNSUPPORTED, "D must be a positive multiple of 8 (got %d)", p->D);
+  if (p->test_stall < 0 || p->test_stall > VDA_TEST_STALL_MAX)
+    return fail(VDA_ERR_INVALID_ARG, "unknown test_stall site %d", p->test_stall);
+  if (p->reserved != 0) return fail(VDA_ERR_INVALID_ARG, "reserved must be 0 (got %d)", p->reserved);
   const void* req[3] = {O_lin, W_lin, Y};
   const char* names[3] = {"O_lin", "W_lin", "Y"};
   for (int i = 0; i < 3; ++i) {
@@ -409,7 +412,7 @@ vda_status vda_merge_project(const vda_merge_problem* p, const void* O_lin, cons
   using bf = __nv_bfloat16;
   e = vda::launch_merge_tc(p->tokens, p->K, p->D, static_cast<const bf*>(O_lin), static_cast<const bf*>(W_lin),
                            static_cast<const bf*>(O_sm), static_cast<const bf*>(W_sm), static_cast<bf*>(Y),
-                           static_cast<unsigned*>(workspace), st);
+                           static_cast<unsigned*>(workspace), st, p->test_stall);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return VDA_OK;
 }

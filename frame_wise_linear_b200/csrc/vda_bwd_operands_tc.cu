@@ -65,6 +65,7 @@ struct BwdOperandsParams {
   unsigned* err;
   int frames, heads, T;
   float inv_lam;
+  int stall;                        // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
 };
 
 struct Shared {
@@ -72,6 +73,7 @@ struct Shared {
   uint64_t t_full[2], t_empty[2];
   uint64_t m_full, x_done, w_done;
   uint64_t drain;
+  uint64_t never;                   // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int abort;
 };
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_operands_tc_kernel(const __gr
     mbar_init(&sh.x_done, 1);
     mbar_init(&sh.w_done, 1);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -325,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_operands_tc_kernel(const __gr
 #pragma unroll 1
         for (int h = 0; h < 2 && ok; ++h) {   // (Gf, S^f), then (Gb, S^b)
           const int hj = 2 * j + h;
-          if (!(ok = mbar_wait(&sh.full[h], (hj >> 1) & 1))) break;
+          const bool stall = p.stall == VDA_TEST_STALL_OPERANDS && blockIdx.x == 0 && hj == 0;
+          if (!(ok = mbar_wait_or_stall(&sh.full[h], (hj >> 1) & 1, &sh.never, stall))) break;
           tc_fence_after();
           const uint32_t g = smem_u32(ring + h * kSlot), sv = g + kMat;
 #pragma unroll
@@ -430,6 +434,7 @@ cudaError_t launch_bwd_operands_tc(const vda_problem& p, const __nv_bfloat16* Gf
   prm.heads = heads;
   prm.T = p.T;
   prm.inv_lam = 1.f / p.lambda;
+  prm.stall = p.test_stall;
   const size_t smem = 1024 + kStage + 2 * kMat + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(bwd_operands_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -137,7 +137,7 @@ bool make_bf16_2d_map(CUtensorMap* m, const void* ptr, long long rows, long long
 // is not null), bf16 [tokens][K] x [K][D] -> [tokens][D], K a multiple of 64.
 cudaError_t launch_merge_tc(long long tokens, int K, int D, const __nv_bfloat16* O_lin, const __nv_bfloat16* W_lin,
                             const __nv_bfloat16* O_sm, const __nv_bfloat16* W_sm, __nv_bfloat16* Y, unsigned* err,
-                            cudaStream_t st);
+                            cudaStream_t st, int stall = 0);
 
 // The local softmax branch (vda_local_softmax_tc.cu): bf16 Q, K, V, G, O in
 // the problem's layout, the text's K_txt, V_txt (skipped when n_txt == 0).

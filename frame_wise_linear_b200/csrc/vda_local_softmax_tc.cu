@@ -62,6 +62,7 @@ struct LocalSoftmaxParams {
   int qtiles;                    // query tiles per frame
   float c;                       // log2(e) / sqrt(d)
   TokGeom g;
+  int stall;                     // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
 };
 
 struct Shared {
@@ -71,6 +72,7 @@ struct Shared {
   uint64_t p_full[2], pv_done[2];
   uint64_t o_free;
   uint64_t drain;
+  uint64_t never;                // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int abort;
 };
@@ -175,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
     }
     mbar_init(&sh.o_free, 128);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -305,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
       for (int j = 0; j < J; ++j) {
         const int pos = it + j, s = pos & 1;
         const KeyTile kt = key_tile(p, kf, j);
-        if (!(ok = !aborted(sh) && mbar_wait(&sh.s_full[s], (pos >> 1) & 1))) break;
+        const bool stall = p.stall == VDA_TEST_STALL_SOFTMAX && blockIdx.x == 0 && pos == 0;
+        if (!(ok = !aborted(sh) && mbar_wait_or_stall(&sh.s_full[s], (pos >> 1) & 1, &sh.never, stall))) break;
         tc_fence_after();
         float x[128];
 #pragma unroll
@@ -445,6 +449,7 @@ cudaError_t launch_local_softmax_tc(const vda_problem& p, const __nv_bfloat16* Q
   prm.qtiles = (p.n + kRows - 1) / kRows;
   prm.c = 1.4426950408889634f / sqrtf((float)p.d_k);
   prm.g = TokGeom{p.layout, p.H, p.T};
+  prm.stall = p.test_stall;
   const size_t smem = 1024 + 7 * kTile + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(local_softmax_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

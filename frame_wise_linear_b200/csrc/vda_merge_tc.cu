@@ -53,12 +53,14 @@ struct MergeParams {
   unsigned* err;
   int m_tiles, n_tiles;
   int kb0, kb;             // K blocks of the linear branch; of both
+  int stall;               // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
 };
 
 struct Shared {
   uint64_t full[kStages], empty[kStages];
   uint64_t t_full[2], t_empty[2];
   uint64_t drain;
+  uint64_t never;          // testing hook: nothing arrives on it
   uint32_t tmem_base;
   int abort;
 };
@@ -95,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1) merge_tc_kernel(const __grid_cons
       mbar_init(&sh.t_empty[i], 128);
     }
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.never, 1);
     sh.abort = 0;
     fence_barrier_init();
   }
@@ -156,7 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1) merge_tc_kernel(const __grid_cons
         const uint32_t d = tmem + tb * kBN;
         for (int kb = 0; kb < p.kb; ++kb, ++it) {
           const int s = it % kStages;
-          if (!(ok = mbar_wait(&sh.full[s], (it / kStages) & 1))) break;
+          const bool stall = p.stall == VDA_TEST_STALL_MERGE && blockIdx.x == 0 && it == 0;
+          if (!(ok = mbar_wait_or_stall(&sh.full[s], (it / kStages) & 1, &sh.never, stall))) break;
           tc_fence_after();
           const uint32_t so = s * kStageBytes;
 #pragma unroll
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) merge_tc_kernel(const __grid_cons
 
 cudaError_t launch_merge_tc(long long tokens, int K, int D, const __nv_bfloat16* O_lin, const __nv_bfloat16* W_lin,
                             const __nv_bfloat16* O_sm, const __nv_bfloat16* W_sm, __nv_bfloat16* Y, unsigned* err,
-                            cudaStream_t st) {
+                            cudaStream_t st, int stall) {
   MergeParams prm;
   memset(&prm, 0, sizeof(prm));
   if (!make_bf16_2d_map(&prm.mA0, O_lin, tokens, K, 64, kBM) || !make_bf16_2d_map(&prm.mW0, W_lin, K, D, 64, kBK) ||
@@ -242,6 +246,7 @@ cudaError_t launch_merge_tc(long long tokens, int K, int D, const __nv_bfloat16*
               !make_bf16_2d_map(&prm.mW1, W_sm, K, D, 64, kBK)))
     return cudaErrorInvalidValue;
   prm.err = err;
+  prm.stall = stall;
   prm.m_tiles = (int)((tokens + kBM - 1) / kBM);
   prm.n_tiles = (D + kBN - 1) / kBN;
   prm.kb0 = K / kBK;

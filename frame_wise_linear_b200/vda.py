@@ -39,7 +39,7 @@ VDA_LAYOUT_BTNHD = 1   # Q, K, V, G, O: [B, T*n, H, d]; text [B, n_txt, H, d] (b
 TEST_STALL_SITES = {
     "gram_stage": 1, "factor_update": 2, "service_gram": 3, "scan_operand": 4, "scan_product": 5,
     "readout_tile": 6, "readout_gate": 7, "readout_state": 8, "rbwd_tile": 9, "rbwd_dq": 10,
-    "gbwd_tile": 11, "gbwd_store": 12,
+    "gbwd_tile": 11, "gbwd_store": 12, "operands": 13, "merge": 14, "softmax": 15,
 }
 
 SYMBOLS = (
@@ -71,7 +71,8 @@ class vda_problem(ctypes.Structure):
 
 
 class vda_merge_problem(ctypes.Structure):
-    _fields_ = [("tokens", ctypes.c_int64), ("K", ctypes.c_int32), ("D", ctypes.c_int32)]
+    _fields_ = [("tokens", ctypes.c_int64), ("K", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("test_stall", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class VdaError(RuntimeError):
@@ -302,9 +303,9 @@ def vda_local_softmax(problem, Q, K, V, G, K_txt, V_txt, O, workspace, stream=No
 
 
 def vda_merge_project(tokens, K, D, O_lin, W_lin, O_sm, W_sm, Y, workspace, stream=None, workspace_bytes=None,
-                      check=True) -> int:
+                      check=True, test_stall=0) -> int:
     """Y = O_lin W_lin + O_sm W_sm (bf16 device buffers; O_sm, W_sm may be None)."""
-    p = vda_merge_problem(int(tokens), int(K), int(D))
+    p = vda_merge_problem(int(tokens), int(K), int(D), int(test_stall), 0)
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     s = load().vda_merge_project(ctypes.byref(p), _ptr(O_lin), _ptr(W_lin), _ptr(O_sm), _ptr(W_sm), _ptr(Y),
                                  _ptr(workspace), wb, _stream(stream))

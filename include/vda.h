@@ -128,7 +128,10 @@ enum {
   VDA_TEST_STALL_RBWD_DQ = 10,       /* readout backward: the epilogue's wait for the first dQ         */
   VDA_TEST_STALL_GBWD_TILE = 11,     /* Gram backward: the MMA thread's wait for the first K, V tile   */
   VDA_TEST_STALL_GBWD_STORE = 12,    /* Gram backward: the epilogue's wait for the second dK, dV       */
-  VDA_TEST_STALL_MAX = 12
+  VDA_TEST_STALL_OPERANDS = 13,      /* backward operands: the MMA thread's wait for its first frame   */
+  VDA_TEST_STALL_MERGE = 14,         /* vda_merge_project: the MMA thread's wait for its first K block */
+  VDA_TEST_STALL_SOFTMAX = 15,       /* vda_local_softmax: the softmax warps' wait for the first scores */
+  VDA_TEST_STALL_MAX = 15
 };
 
 /* Bytes of device workspace vda_forward needs for `p` (written to *bytes).
@@ -293,6 +296,8 @@ vda_status vda_local_softmax(const vda_problem* p, const void* Q, const void* K,
 typedef struct vda_merge_problem {
   int64_t tokens;
   int32_t K, D;
+  int32_t test_stall; /* testing hook as in vda_problem; 0 in normal use */
+  int32_t reserved;   /* 0 */
 } vda_merge_problem;
 vda_status vda_merge_project(const vda_merge_problem* p, const void* O_lin, const void* W_lin, const void* O_sm,
                              const void* W_sm, void* Y, void* workspace, size_t workspace_bytes, void* stream);

@@ -54,6 +54,20 @@ def test_problem_struct_layout():
         assert "VDA_TEST_STALL_%s = %d" % (name.upper(), v) in txt
 
 
+def test_merge_problem_struct_layout():
+    # the header's vda_merge_problem: int64 tokens, int32 K, D, test_stall, reserved
+    assert ctypes.sizeof(vda.vda_merge_problem) == 24
+    assert vda.vda_merge_problem.test_stall.offset == 16
+
+
+def test_merge_bad_problem_rejected(lib):
+    ok = 1 << 20
+    s = vda.vda_merge_project(128, 128, 64, ok, ok, None, None, ok, ok, stream=0, check=False, test_stall=99)
+    assert s == vda.VDA_ERR_INVALID_ARG, vda.vda_last_error()
+    s = vda.vda_merge_project(128, 128, 64, ok, ok, None, None, ok, ok, stream=0, check=False, test_stall=-1)
+    assert s == vda.VDA_ERR_INVALID_ARG, vda.vda_last_error()
+
+
 def _p(**kw):
     base = dict(B=1, H=2, T=3, n=64, n_txt=8, d_k=128, d_v=128, dtype=vda.VDA_DTYPE_BF16, lam=1.0)
     base.update(kw)
@@ -91,7 +105,7 @@ def test_workspace_size_valid(lib, dtype, state_bytes):
     (dict(dtype=vda.VDA_DTYPE_E4M3, scale_v=float("inf")), vda.VDA_ERR_INVALID_ARG),
     (dict(dtype=vda.VDA_DTYPE_E4M3, scale_k=-1.0), vda.VDA_ERR_INVALID_ARG),
     (dict(dtype=vda.VDA_DTYPE_E4M3, d_k=64, d_v=64), vda.VDA_ERR_UNSUPPORTED),
-    (dict(test_stall=13), vda.VDA_ERR_INVALID_ARG),
+    (dict(test_stall=16), vda.VDA_ERR_INVALID_ARG),
 ])
 def test_bad_problem_rejected(lib, kw, status):
     p = _p(**kw)

@@ -31,7 +31,8 @@ pytestmark = pytest.mark.gpu
 W = synth.Workload("stall", B=1, H=4, T=80, n=128, n_txt=16, d_k=128, d_v=128, dtype=synth.DTYPE_BF16, lam=1.0)
 FORWARD_SITES = ["gram_stage", "factor_update", "service_gram", "scan_operand", "scan_product",
                  "readout_tile", "readout_gate", "readout_state"]
-BACKWARD_SITES = ["rbwd_tile", "rbwd_dq", "gbwd_tile", "gbwd_store"]
+BACKWARD_SITES = ["rbwd_tile", "rbwd_dq", "operands", "gbwd_tile", "gbwd_store"]
+OTHER_SITES = ["merge", "softmax"]
 BOUND_S = 30.0   # a stalled call ends within a few 2 s wait limits
 
 
@@ -105,6 +106,50 @@ def test_backward_wait_that_runs_out_reports_timeout(site):
         assert np.array_equal(a, b), site
 
 
+def _merge(ws, stall=0):
+    """One merge of 4096 tokens (32 row tiles, so the first CTA has one), K = 128, D = 256, both branches."""
+    import torch
+    from frame_wise_linear_b200 import vda
+    g = torch.Generator(device="cuda").manual_seed(11)
+    O, P = (torch.randn(4096, 128, device="cuda", generator=g).to(torch.bfloat16) for _ in range(2))
+    Wl, Ws = (torch.randn(128, 256, device="cuda", generator=g).mul_(0.09).to(torch.bfloat16) for _ in range(2))
+    Y = torch.empty(4096, 256, dtype=torch.bfloat16, device="cuda")
+    vda.vda_merge_project(4096, 128, 256, O, Wl, P, Ws, Y, ws, test_stall=stall)
+    return Y
+
+
+def _softmax(d, prob, ws):
+    import torch
+    from frame_wise_linear_b200 import vda
+    O = torch.empty_like(d["G"])
+    vda.vda_local_softmax(prob, d["Q"], d["K"], d["V"], d["G"], d["K_txt"], d["V_txt"], O, ws)
+    return O
+
+
+@pytest.mark.parametrize("site", OTHER_SITES)
+def test_merge_and_local_softmax_wait_that_runs_out_reports_timeout(site):
+    import torch
+    from frame_wise_linear_b200 import vda
+    d, _, prob, _ = _setup()
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    if site == "merge":
+        run = lambda stall: _merge(ws, stall)
+    else:
+        run = lambda stall: _softmax(d, vda.make_problem(**W.problem(), test_stall=stall), ws)
+    ref = from_device(run(0))
+    assert vda.vda_sync_status(ws, check=False) == vda.VDA_OK
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    run(vda.TEST_STALL_SITES[site])
+    status = vda.vda_sync_status(ws, check=False)
+    dt = time.perf_counter() - t0
+    assert status == vda.VDA_ERR_TIMEOUT, (site, vda.vda_status_string(status), vda.vda_last_error())
+    assert dt < BOUND_S, (site, dt)
+    again = from_device(run(0))
+    assert vda.vda_sync_status(ws, check=False) == vda.VDA_OK
+    assert np.array_equal(again, ref), site
+
+
 def test_every_site_is_covered():
     from frame_wise_linear_b200 import vda
-    assert sorted(FORWARD_SITES + BACKWARD_SITES) == sorted(vda.TEST_STALL_SITES)
+    assert sorted(FORWARD_SITES + BACKWARD_SITES + OTHER_SITES) == sorted(vda.TEST_STALL_SITES)
