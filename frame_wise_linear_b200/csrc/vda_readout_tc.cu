@@ -26,8 +26,11 @@
 //               through a 2-slot shared-memory ring into registers a frame
 //               ahead, then written into the MMA's B operand buffer as soon
 //               as the MMAs release it.
-//   warps 18..19 (e4m3 only) widen each Q tile into the bf16 A ring (freed
-//               by the tile's MMAs); the epilogue stores O through an 8 KB
+//   e4m3 inputs: Q and G tiles are half the size, so their rings are 4
+//               deep (the same bytes in flight as bf16).  The epilogue warps
+//               also widen the next tile's Q to bf16, each thread its own row
+//               and column half, straight into tensor memory, where the MMAs
+//               read A from (two 64-column slots); O goes out through an 8 KB
 //               staging box per column half (32-column TMA stores).
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
@@ -40,8 +43,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kQStages = 2;
+constexpr int kQStages = 2;                  // bf16 input rings (32 KB tiles)
 constexpr int kGStages = 2;
+constexpr int kStages8 = 4;                  // e4m3 input rings (16 KB tiles)
 constexpr int kRows = 128;                   // tokens per tile
 constexpr int kBox = kRows * 64 * 2;         // 128 rows x 64 features bf16: 16 KB
 constexpr int kTile = 2 * kBox;              // 32 KB
@@ -51,13 +55,12 @@ constexpr int kPieces = 128 / kPieceRows;    // 8 pieces per frame
 constexpr int kPieceHalf = kPieceRows * 128 * 2;   // 4 KB of S^f (or S^b) per piece
 constexpr int kPiece = 2 * kPieceHalf;       // one staging slot: S^f piece | S^b piece
 constexpr int kThreads = 576;              // 2 control warps + 8 epilogue warps + 8 prep warps
-// e4m3 inputs: Q and G tiles are 16 KB (one 128-byte row per token); two
-// more warps widen each Q tile to the bf16 operand tile (A ring).
+// e4m3 inputs: Q and G tiles are 16 KB (one 128-byte row per token).
 constexpr int kTile8 = kRows * 128;          // 16 KB
 constexpr int kOStage = kRows * 32 * 2;      // 128 rows x 32 bf16 columns: 8 KB
-constexpr int kConvWarps = 2;
-constexpr int kThreads8 = kThreads + 32 * kConvWarps;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 256;          // two 128-column accumulators
+constexpr uint32_t kTmemCols8 = 512;         // e4m3: and two 64-column A slots (the widened Q)
+constexpr uint32_t kACol = 256;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);
 
 struct ReadoutTcParams {
@@ -76,10 +79,10 @@ struct ReadoutTcParams {
 };
 
 struct Shared {
-  uint64_t q_full[kQStages], q_empty[kQStages];
-  uint64_t g_full[kGStages], g_empty[kGStages];
+  uint64_t q_full[kStages8], q_empty[kStages8];
+  uint64_t g_full[kStages8], g_empty[kStages8];
   uint64_t t_full[2], t_empty[2];
-  uint64_t a_full[2], a_empty[2];   // e4m3: the widened Q tiles (the MMA's A operand)
+  uint64_t a_full[2];   // e4m3: the widened Q tiles in tensor memory (the MMA's A operand)
   uint64_t sig_full, sig_empty;
   uint64_t p_full[2];   // S staging slots
   uint64_t s0_full;     // the first frame's states, loaded straight into the operand buffer
@@ -124,16 +127,16 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2_exact(uint32_t h) {
 }
 
 template <bool kF8>
-__global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
-    readout_tc_kernel(const __grid_constant__ ReadoutTcParams p) {
+__global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_constant__ ReadoutTcParams p) {
   constexpr int kQT = kF8 ? kTile8 : kTile;         // bytes of one Q (or G) input tile
+  constexpr int kQS = kF8 ? kStages8 : kQStages;    // ring depths
+  constexpr int kGS = kF8 ? kStages8 : kGStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sig = base;                              // S^f | S^b
-  uint8_t* qbuf = base + kSig;                      // kQStages input tiles
-  uint8_t* gbuf = qbuf + kQStages * kQT;            // kGStages tiles (bf16: G in, O out; e4m3: G in)
-  uint8_t* abuf = gbuf + kGStages * kQT;            // e4m3: 2 widened Q tiles (the MMA's A ring)
-  uint8_t* sstage = kF8 ? abuf + 2 * kTile : abuf;  // 2 S staging slots
+  uint8_t* qbuf = base + kSig;                      // kQS input tiles
+  uint8_t* gbuf = qbuf + kQS * kQT;                 // kGS tiles (bf16: G in, O out; e4m3: G in)
+  uint8_t* sstage = gbuf + kGS * kQT;               // 2 S staging slots
   uint8_t* ostage = sstage + 2 * kPiece;            // e4m3: an 8 KB O staging box per column half
   Shared& sh = *reinterpret_cast<Shared*>(ostage + (kF8 ? 2 * kOStage : 0));
 
@@ -144,13 +147,12 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
   const int t_end = (int)(total * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kQStages; ++i) {
+    for (int i = 0; i < kQS; ++i) {
       mbar_init(&sh.q_full[i], 1);
-      mbar_init(&sh.q_empty[i], kF8 ? 32 * kConvWarps : 1);   // e4m3: the widening threads
-      mbar_init(&sh.a_full[i], 32 * kConvWarps);
-      mbar_init(&sh.a_empty[i], 1);                           // the tile's MMAs are done with it
+      mbar_init(&sh.q_empty[i], kF8 ? 256 : 1);   // bf16: the tile's MMAs; e4m3: the widening threads
     }
-    for (int i = 0; i < kGStages; ++i) {
+    for (int i = 0; i < 2; ++i) mbar_init(&sh.a_full[i], 256);
+    for (int i = 0; i < kGS; ++i) {
       mbar_init(&sh.g_full[i], 1);
       mbar_init(&sh.g_empty[i], kF8 ? 256 : 2);   // bf16: one arrival per stored half; e4m3: per reader
     }
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sh.tmem_base, kTmemCols);
+    tmem_alloc(&sh.tmem_base, kF8 ? kTmemCols8 : kTmemCols);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
         tok_load(qbuf + qs * kQT, &p.mQ, &sh.q_full[qs], p.g, q, 0, y, pol);
         if (!kF8) tok_load(qbuf + qs * kQT + kBox, &p.mQ, &sh.q_full[qs], p.g, q, 64, y, pol);
         ++q_issued;
-        if (++qs == kQStages) { qs = 0; qph ^= 1; }
+        if (++qs == kQS) { qs = 0; qph ^= 1; }
         if (!mbar_wait(&sh.g_empty[gs], gph ^ 1)) {
           set_abort(sh, p.err);
           break;
@@ -217,13 +219,13 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
         tok_load(gbuf + gs * kQT, &p.mG, &sh.g_full[gs], p.g, q, 0, y, pol);
         if (!kF8) tok_load(gbuf + gs * kQT + kBox, &p.mG, &sh.g_full[gs], p.g, q, 64, y, pol);
         ++g_issued;
-        if (++gs == kGStages) { gs = 0; gph ^= 1; }
+        if (++gs == kGS) { gs = 0; gph ^= 1; }
       }
       if (aborted(sh)) {  // let the loads still in flight land before exit
-        for (int c = q_issued > kQStages ? q_issued - kQStages : 0; c < q_issued; ++c)
-          mbar_wait(&sh.q_full[c % kQStages], (c / kQStages) & 1);
-        for (int c = g_issued > kGStages ? g_issued - kGStages : 0; c < g_issued; ++c)
-          mbar_wait(&sh.g_full[c % kGStages], (c / kGStages) & 1);
+        for (int c = q_issued > kQS ? q_issued - kQS : 0; c < q_issued; ++c)
+          mbar_wait(&sh.q_full[c % kQS], (c / kQS) & 1);
+        for (int c = g_issued > kGS ? g_issued - kGS : 0; c < g_issued; ++c)
+          mbar_wait(&sh.g_full[c % kGS], (c / kGS) & 1);
       }
     }
   } else if (warp == 1) {
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
       int qs = 0, tb = 0;
       uint32_t qph = 0, tph = 0, sph = 0;
       int cur_u = -1;
-      const uint32_t qaddr = smem_u32(kF8 ? abuf : qbuf);
+      const uint32_t qaddr = smem_u32(qbuf);
       const uint32_t saddr = smem_u32(sig);
       for (int tile = t_begin; tile < t_end && !aborted(sh); ++tile) {
         const int u = tile / p.tiles_per_unit;
@@ -242,10 +244,11 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
           cur_u = u;
         }
         if (!mbar_wait(&sh.t_empty[tb], tph ^ 1)) { set_abort(sh, p.err); break; }
-        // The A operand: the bf16 Q tile, or (e4m3) its widened copy.
+        // The A operand: the bf16 Q tile, or (e4m3) its widened copy in
+        // tensor memory (A slot = tile parity, as the accumulator).
         const bool stall = p.stall == VDA_TEST_STALL_READOUT_TILE && blockIdx.x == 0 && tile == t_begin;
-        uint64_t* afull = kF8 ? &sh.a_full[qs] : &sh.q_full[qs];
-        if (!mbar_wait_or_stall(afull, qph, &sh.never, stall)) { set_abort(sh, p.err); break; }
+        uint64_t* afull = kF8 ? &sh.a_full[tb] : &sh.q_full[qs];
+        if (!mbar_wait_or_stall(afull, kF8 ? tph : qph, &sh.never, stall)) { set_abort(sh, p.err); break; }
         tc_fence_after();
         const uint32_t d = tmem + tb * 128;
         const uint32_t qa = qaddr + qs * kTile;
@@ -253,17 +256,22 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
         for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            // A: Q tile, K-major; 16 features = 32 bytes inside a 128-byte row.
-            const uint64_t a = smem_desc(qa + (k / 4) * kBox + (k % 4) * 32, 16, 1024, kSwizzle128B);
             // B: S^f or S^b, MN-major; 16 rows of 128 bytes per k-step,
             // 64-column blocks 16 KB apart.
             const uint64_t b = smem_desc(saddr + pass * kTile + k * 16 * 128, kBox, 1024, kSwizzle128B);
-            mma_bf16_ss(d, a, b, kIdesc, (pass | k) ? 1u : 0u);
+            if constexpr (kF8) {
+              // A: 16 features = 8 columns of the tile's A slot.
+              mma_bf16_ts(d, tmem + kACol + tb * 64 + 8 * k, b, kIdesc, (pass | k) ? 1u : 0u);
+            } else {
+              // A: Q tile, K-major; 16 features = 32 bytes inside a 128-byte row.
+              const uint64_t a = smem_desc(qa + (k / 4) * kBox + (k % 4) * 32, 16, 1024, kSwizzle128B);
+              mma_bf16_ss(d, a, b, kIdesc, (pass | k) ? 1u : 0u);
+            }
           }
         }
-        // bf16: the Q tile is free; e4m3: the widened tile is (the widening
-        // threads free the 8-bit input tile themselves).
-        mma_commit(kF8 ? &sh.a_empty[qs] : &sh.q_empty[qs]);
+        // bf16: the Q tile is free.  e4m3: the widening threads free the
+        // 8-bit tile, and the A slot is free once t_full has arrived.
+        if (!kF8) mma_commit(&sh.q_empty[qs]);
         mma_commit(&sh.t_full[tb]);
         const bool last_of_unit = (tile + 1 == t_end) || ((tile + 1) / p.tiles_per_unit != u);
         if (last_of_unit) mma_commit(&sh.sig_empty);
@@ -282,11 +290,47 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
     const int row = quarter * 32 + lane;      // tile row this thread owns in TMEM
     int gs = 0, tb = 0;
     uint32_t gph = 0, tph = 0;
+    // e4m3: widen tile w's Q to bf16, this thread's row and column half, into
+    // the A slot of its parity (free: the MMAs of tile w - 2, which read it,
+    // were complete when this thread saw that tile's t_full).
+    int qs = 0;
+    uint32_t qph = 0;
+    auto widen = [&](int w) -> bool {
+      bool ok = !aborted(sh) && mbar_wait(&sh.q_full[qs], qph);
+      if (!__all_sync(0xffffffffu, ok)) return false;   // the TMEM store below is warp-wide
+      const uint8_t* src = qbuf + qs * kQT;
+      uint32_t o[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {           // features 64 half + 16 c .. + 15
+        const uint4 v = *reinterpret_cast<const uint4*>(src + sw128(row, 4 * half + c));
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          o[8 * c + 2 * e] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(wv[e] & 0xFFFFu)));
+          o[8 * c + 2 * e + 1] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(wv[e] >> 16)));
+        }
+      }
+      const int slot = (w - t_begin) & 1;
+      tmem_st_32x32b_x32(tmem + kACol + slot * 64 + half * 32 + ((uint32_t)(quarter * 32) << 16), o);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sh.q_empty[qs]);
+      mbar_arrive(&sh.a_full[slot]);
+      if (++qs == kQS) { qs = 0; qph ^= 1; }
+      return true;
+    };
+    bool wok = true;
+    if constexpr (kF8) {
+      if (t_begin < t_end) wok = widen(t_begin);
+    }
     for (int tile = t_begin; tile < t_end; ++tile) {
       const int u = tile / p.tiles_per_unit;
       const int y = (tile % p.tiles_per_unit) * kRows;
       const bool stall = p.stall == VDA_TEST_STALL_READOUT_GATE && blockIdx.x == 0 && tile == t_begin + 1;
-      bool ok = !aborted(sh) && mbar_wait(&sh.t_full[tb], tph);
+      if constexpr (kF8) {
+        if (wok && tile + 1 < t_end) wok = widen(tile + 1);   // the next tile's MMAs overlap this epilogue
+      }
+      bool ok = wok && !aborted(sh) && mbar_wait(&sh.t_full[tb], tph);
       ok = ok && mbar_wait_or_stall(&sh.g_full[gs], gph, &sh.never, stall);
       if (!ok) set_abort(sh, p.err);
       // One decision for the half's four warps, which meet at its named
@@ -377,7 +421,7 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
           mbar_arrive(&sh.g_empty[gs]);
         }
       }
-      if (++gs == kGStages) { gs = 0; gph ^= 1; }
+      if (++gs == kGS) { gs = 0; gph ^= 1; }
       tb ^= 1;
       if (tb == 0) tph ^= 1;
     }
@@ -474,54 +518,12 @@ __global__ void __launch_bounds__(kF8 ? kThreads8 : kThreads, 1)
     if (pt == 0) {   // let the copies still in flight land before exit
       for (int c = landed; c < issued; ++c) mbar_wait(&sh.p_full[c & 1], (c >> 1) & 1);
     }
-  } else if constexpr (kF8) {
-    // ------------------------------------------------------------ widening (e4m3)
-    // Each thread widens two rows of every Q tile: 128 e4m3 features (one
-    // swizzled 128-byte row) into 128 bf16 (two 64-feature boxes, the MMA's
-    // K-major operand layout), once the tile has landed and the A buffer of
-    // its stage is free (its previous O store has read it).  No named
-    // barrier: each thread leaves on its own failed wait.
-    const int ct = threadIdx.x - kThreads;    // 0..63
-    int qs = 0;
-    uint32_t qph = 0;
-    for (int tile = t_begin; tile < t_end; ++tile) {
-      bool ok = !aborted(sh) && mbar_wait(&sh.q_full[qs], qph);
-      ok = ok && mbar_wait(&sh.a_empty[qs], qph ^ 1);
-      if (!ok) {
-        set_abort(sh, p.err);
-        break;
-      }
-      const uint8_t* src = qbuf + qs * kTile8;
-      uint8_t* dst = abuf + qs * kTile;
-#pragma unroll 1
-      for (int rr = 0; rr < 2; ++rr) {
-        const int row = ct + 64 * rr;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {          // features 16 c .. 16 c + 15
-          const uint4 v = *reinterpret_cast<const uint4*>(src + sw128(row, c));
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o[8];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            o[2 * e] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(w[e] & 0xFFFFu)));
-            o[2 * e + 1] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(w[e] >> 16)));
-          }
-          uint8_t* box = dst + (c >> 2) * kBox;   // features 64 (c / 4) ..
-          *reinterpret_cast<uint4*>(box + sw128(row, 2 * (c & 3))) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(box + sw128(row, 2 * (c & 3) + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
-        }
-      }
-      fence_proxy_async_smem();                // visible to the tensor core
-      mbar_arrive(&sh.q_empty[qs]);
-      mbar_arrive(&sh.a_full[qs]);
-      if (++qs == kQStages) { qs = 0; qph ^= 1; }
-    }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 1) tmem_dealloc(tmem, kF8 ? kTmemCols8 : kTmemCols);
 }
 
 }  // namespace
@@ -548,8 +550,8 @@ cudaError_t launch_readout_tc(const vda_problem& p, const void* Q, const void* G
   prm.stall = p.test_stall;
   prm.q_scale = f8 ? p.scale_q : 1.f;
   prm.g_scale = f8 ? p.scale_g : 1.f;
-  const size_t smem = 1024 + kSig + (kQStages + kGStages) * (f8 ? kTile8 : kTile) + (f8 ? 2 * kTile : 0) +
-                      2 * kPiece + (f8 ? 2 * kOStage : 0) + sizeof(Shared);
+  const size_t smem = 1024 + kSig + (f8 ? 2 * kStages8 * kTile8 : (kQStages + kGStages) * kTile) + 2 * kPiece +
+                      (f8 ? 2 * kOStage : 0) + sizeof(Shared);
   auto kern = f8 ? readout_tc_kernel<true> : readout_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -563,7 +565,7 @@ cudaError_t launch_readout_tc(const vda_problem& p, const void* Q, const void* G
   // and G; only the state loads wait for the scan (griddep_wait).
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(f8 ? kThreads8 : kThreads);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
