@@ -26,12 +26,12 @@
 //               through a 2-slot shared-memory ring into registers a frame
 //               ahead, then written into the MMA's B operand buffer as soon
 //               as the MMAs release it.
-//   e4m3 inputs: Q and G tiles are half the size, so their rings are 4
-//               deep (the same bytes in flight as bf16).  The epilogue warps
+//   e4m3 inputs: Q and G tiles are half the size, so their rings are 3 and
+//               4 deep (about the bytes in flight of bf16).  The epilogue warps
 //               also widen the next tile's Q to bf16, each thread its own row
 //               and column half, straight into tensor memory, where the MMAs
-//               read A from (two 64-column slots); O goes out through an 8 KB
-//               staging box per column half (32-column TMA stores).
+//               read A from (two 64-column slots); O goes out through two
+//               8 KB staging boxes per column half (32-column TMA stores).
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
@@ -45,7 +45,8 @@ using namespace sm100;
 
 constexpr int kQStages = 2;                  // bf16 input rings (32 KB tiles)
 constexpr int kGStages = 2;
-constexpr int kStages8 = 4;                  // e4m3 input rings (16 KB tiles)
+constexpr int kQStages8 = 3;                 // e4m3 input rings (16 KB tiles)
+constexpr int kGStages8 = 4;
 constexpr int kRows = 128;                   // tokens per tile
 constexpr int kBox = kRows * 64 * 2;         // 128 rows x 64 features bf16: 16 KB
 constexpr int kTile = 2 * kBox;              // 32 KB
@@ -79,8 +80,8 @@ struct ReadoutTcParams {
 };
 
 struct Shared {
-  uint64_t q_full[kStages8], q_empty[kStages8];
-  uint64_t g_full[kStages8], g_empty[kStages8];
+  uint64_t q_full[kQStages8], q_empty[kQStages8];
+  uint64_t g_full[kGStages8], g_empty[kGStages8];
   uint64_t t_full[2], t_empty[2];
   uint64_t a_full[2];   // e4m3: the widened Q tiles in tensor memory (the MMA's A operand)
   uint64_t sig_full, sig_empty;
@@ -129,16 +130,16 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2_exact(uint32_t h) {
 template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_constant__ ReadoutTcParams p) {
   constexpr int kQT = kF8 ? kTile8 : kTile;         // bytes of one Q (or G) input tile
-  constexpr int kQS = kF8 ? kStages8 : kQStages;    // ring depths
-  constexpr int kGS = kF8 ? kStages8 : kGStages;
+  constexpr int kQS = kF8 ? kQStages8 : kQStages;   // ring depths
+  constexpr int kGS = kF8 ? kGStages8 : kGStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sig = base;                              // S^f | S^b
   uint8_t* qbuf = base + kSig;                      // kQS input tiles
   uint8_t* gbuf = qbuf + kQS * kQT;                 // kGS tiles (bf16: G in, O out; e4m3: G in)
   uint8_t* sstage = gbuf + kGS * kQT;               // 2 S staging slots
-  uint8_t* ostage = sstage + 2 * kPiece;            // e4m3: an 8 KB O staging box per column half
-  Shared& sh = *reinterpret_cast<Shared*>(ostage + (kF8 ? 2 * kOStage : 0));
+  uint8_t* ostage = sstage + 2 * kPiece;            // e4m3: two 8 KB O staging boxes per column half
+  Shared& sh = *reinterpret_cast<Shared*>(ostage + (kF8 ? 4 * kOStage : 0));
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -341,10 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
       const uint32_t taddr = tmem + tb * 128 + half * 64 + ((uint32_t)(quarter * 32) << 16);
       if constexpr (kF8) {
         // G from its 16 KB tile (one 128-byte row per token); O through the
-        // half's 8 KB staging box, 32 columns (64-byte rows) at a time, by
-        // TMA stores (rows past n clipped).
+        // half's two 8 KB staging boxes in turn, 32 columns (64-byte rows) at
+        // a time, by TMA stores (rows past n clipped).
         const uint8_t* g8row = gbuf + gs * kQT;
-        uint8_t* ostg = ostage + half * kOStage;
         const bool leader = et % 128 == 0;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
@@ -373,7 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
             mbar_arrive(&sh.t_empty[tb]);
             mbar_arrive(&sh.g_empty[gs]);
           }
-          if (leader) bulk_wait_read<0>();       // the half's previous store has read the box
+          uint8_t* ostg = ostage + (2 * half + c) * kOStage;
+          if (leader) bulk_wait_read<1>();       // the store two boxes back has read this one
           named_bar_sync(1 + half, 128);
 #pragma unroll
           for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(ostg + sw64(row, q)) = ch[q];
@@ -550,8 +551,8 @@ cudaError_t launch_readout_tc(const vda_problem& p, const void* Q, const void* G
   prm.stall = p.test_stall;
   prm.q_scale = f8 ? p.scale_q : 1.f;
   prm.g_scale = f8 ? p.scale_g : 1.f;
-  const size_t smem = 1024 + kSig + (f8 ? 2 * kStages8 * kTile8 : (kQStages + kGStages) * kTile) + 2 * kPiece +
-                      (f8 ? 2 * kOStage : 0) + sizeof(Shared);
+  const size_t smem = 1024 + kSig + (f8 ? (kQStages8 + kGStages8) * kTile8 : (kQStages + kGStages) * kTile) +
+                      2 * kPiece + (f8 ? 4 * kOStage : 0) + sizeof(Shared);
   auto kern = f8 ? readout_tc_kernel<true> : readout_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -9,9 +9,14 @@
 // 1..T (forward) or T..1 (backward).  S^f_t / S^b_t are written as float32.
 //
 // Precision: M_t arrives as bf16 hi + lo (written by the factor step in the
-// MMA operand layout); X is split the same way; the product takes three MMA
-// passes, M_hi X_hi + M_hi X_lo + M_lo X_hi, accumulated in float32 (the
-// dropped M_lo X_lo term is below 2^-16 relative).  ||M_t||_2 <= 1, so the
+// MMA operand layout); X is split the same way; the product is
+// M_hi X_hi + M_hi X_lo + M_lo X_hi in float32 (the dropped M_lo X_lo term is
+// below 2^-16 relative).  X_hi and X_lo sit side by side as one operand of
+// 2N columns, so M_hi [X_hi | X_lo] is one N = 2N pass, and M_lo X_hi
+// accumulates onto its first N columns; the row warps add the two halves.
+// (The step is bound by shared-memory bandwidth: the TMA writes of M_t and
+// B_t, X, the state staging and the MMAs' operand reads; this form reads
+// M_hi once instead of twice.)  ||M_t||_2 <= 1, so the
 // per-step error does not grow along the chain.  Each state goes out as
 // bfloat16 in the readout's operand layout (row-major, d_k x d_v); float32
 // states are written as well when the caller asks for them.
@@ -24,7 +29,7 @@
 //               while the step's MMAs run, then read S_t back from TMEM;
 //   warp 8      one thread: bulk-copies M_t (64 KB) into a 2-stage ring and
 //               B_t (this CTA's columns) by TMA as soon as the row warps have
-//               copied the previous one into registers, and issues the 24
+//               copied the previous one into registers, and issues the 16
 //               MMAs of each step.
 // Every wait is bounded; a timeout sets the error bit and the CTA winds down.
 #include "sm100.cuh"
@@ -49,6 +54,7 @@ constexpr int kBBuf = N * 128 * 4;           // B_t columns of this CTA, same la
 constexpr int kEpiBar = 1;                   // named barrier of the row warps
 constexpr int kAhead = 4;                    // steps of M_t and B_t prefetched into L2
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, N, /*a MN*/ false, /*b MN*/ true);
+constexpr uint32_t kIdesc2 = idesc_bf16_f32(128, 2 * N, /*a MN*/ false, /*b MN*/ true);
 
 struct ScanTcParams {
   CUtensorMap mSFb, mSBb;  // states for the readout: [frames][128][128] bfloat16, 64 x 128 boxes
@@ -125,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&sh.tmem_base, N);
+    tmem_alloc(&sh.tmem_base, 2 * N);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -201,15 +207,16 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
         tc_fence_after();
         prefetch(s + kAhead);
         const uint32_t ma = maddr + st * kMBytes;
+        // M_hi [X_hi | X_lo] into columns 0 .. 2N-1 (X_lo is the operand's
+        // second 64-column block), then M_lo X_hi onto columns 0 .. N-1.
 #pragma unroll
-        for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t a_off = pass == 2 ? kMBytes / 2 : 0;      // M lo on the last pass
-          const uint32_t b_off = pass == 1 ? kXHalf : 0;           // X lo on the second pass
+        for (int pass = 0; pass < 2; ++pass) {
+          const uint32_t a_off = pass == 1 ? kMBytes / 2 : 0;      // M lo on the second pass
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint64_t a = smem_desc(ma + a_off + (k / 4) * 16384 + (k % 4) * 32, 16, 1024, kSwizzle128B);
-            const uint64_t b = smem_desc(xaddr + b_off + k * 16 * 128, 16384, 1024, kSwizzle128B);
-            mma_bf16_ss(tmem, a, b, kIdesc, (pass | k) ? 1u : 0u);
+            const uint64_t b = smem_desc(xaddr + k * 16 * 128, kXHalf, 1024, kSwizzle128B);
+            mma_bf16_ss(tmem, a, b, pass == 0 ? kIdesc2 : kIdesc, (pass | k) ? 1u : 0u);
           }
         }
         mma_commit(&sh.d_full);
@@ -320,11 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
       if (!ok && !aborted(sh)) set_abort(sh, p.err);
       tc_fence_after();
       {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)((warp % 4) * 32) << 16) + kCols * hc, r);
+        // S_t = (M_hi X_hi + M_lo X_hi) + M_hi X_lo
+        uint32_t r[32], r2[32];
+        const uint32_t ta = tmem + ((uint32_t)((warp % 4) * 32) << 16) + kCols * hc;
+        tmem_ld_32x32b_x32(ta, r);
+        tmem_ld_32x32b_x32(ta + N, r2);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < kCols; ++j) srow[j] = __uint_as_float(r[j]);
+        for (int j = 0; j < kCols; ++j) srow[j] = __uint_as_float(r[j]) + __uint_as_float(r2[j]);
       }
     }
     if (T >= 1) store_state(T);
@@ -334,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, N);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 2 * N);
 }
 
 }  // namespace
