@@ -322,18 +322,12 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
         }
         tc_fence_before();
         mbar_arrive(&sh.s_free[s]);            // the MMAs may write the next scores here
-        // Scores in log2 units, keys past the tile's valid ones excluded; the
-        // row maximum over 8 interleaved partial maxima (short dependency
-        // chains instead of one of 128).
-        float mp[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mp[i] = -INFINITY;
+        float mt = -INFINITY;
 #pragma unroll
         for (int e = 0; e < 128; ++e) {
-          x[e] = e < kt.valid ? x[e] * p.c : -INFINITY;
-          mp[e & 7] = fmaxf(mp[e & 7], x[e]);
+          x[e] = e < kt.valid ? x[e] * p.c : -INFINITY;   // scores in log2 units; rows past the keys excluded
+          mt = fmaxf(mt, x[e]);
         }
-        const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         // P_j's buffer is free once PV_{j-2} is done, and a rescale of O needs PV_{j-1} done.
         const bool grow = j == 0 || mt > m + kRescale;
         if (j >= 2 && !(ok = mbar_wait(&sh.pv_done[s], ((pos - 2) >> 1) & 1))) break;
@@ -358,21 +352,17 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
           m = mn;
         }
         uint8_t* pt = pbuf + s * kTile;
-        float lp[8];                             // partial sums, as the maxima
-#pragma unroll
-        for (int i = 0; i < 8; ++i) lp[i] = 0.f;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {           // keys 8c .. 8c + 7
           float v[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             v[e] = ex2(x[8 * c + e] - m);
-            lp[e] += v[e];
+            l += v[e];
           }
           *reinterpret_cast<uint4*>(pt + (c >> 3) * kBox + sw128(row, c & 7)) =
               make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
         }
-        l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sh.p_full[s]);

@@ -150,16 +150,16 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQS; ++i) {
       mbar_init(&sh.q_full[i], 1);
-      mbar_init(&sh.q_empty[i], kF8 ? 256 : 1);   // bf16: the tile's MMAs; e4m3: the widening threads
+      mbar_init(&sh.q_empty[i], kF8 ? 128 : 1);   // bf16: the tile's MMAs; e4m3: the widening group
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&sh.a_full[i], 256);
+    for (int i = 0; i < 2; ++i) mbar_init(&sh.a_full[i], 128);
     for (int i = 0; i < kGS; ++i) {
       mbar_init(&sh.g_full[i], 1);
-      mbar_init(&sh.g_empty[i], kF8 ? 256 : 2);   // bf16: one arrival per stored half; e4m3: per reader
+      mbar_init(&sh.g_empty[i], kF8 ? 128 : 2);   // bf16: one arrival per stored half; e4m3: per reader
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.t_full[i], 1);
-      mbar_init(&sh.t_empty[i], 256);
+      mbar_init(&sh.t_empty[i], kF8 ? 128 : 256);   // e4m3: the tile's group; bf16: both halves
     }
     mbar_init(&sh.sig_full, 256);   // the 8 prep warps
     mbar_init(&sh.sig_empty, 1);
@@ -287,74 +287,82 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;          // 0..255
     const int quarter = warp % 4;             // TMEM lanes this warp may access
-    const int half = (warp - 2) / 4;          // column half 0..63 or 64..127
     const int row = quarter * 32 + lane;      // tile row this thread owns in TMEM
-    int gs = 0, tb = 0;
-    uint32_t gph = 0, tph = 0;
-    // e4m3: widen tile w's Q to bf16, this thread's row and column half, into
-    // the A slot of its parity (free: the MMAs of tile w - 2, which read it,
-    // were complete when this thread saw that tile's t_full).
-    int qs = 0;
-    uint32_t qph = 0;
-    auto widen = [&](int w) -> bool {
-      bool ok = !aborted(sh) && mbar_wait(&sh.q_full[qs], qph);
-      if (!__all_sync(0xffffffffu, ok)) return false;   // the TMEM store below is warp-wide
-      const uint8_t* src = qbuf + qs * kQT;
-      uint32_t o[32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {           // features 64 half + 16 c .. + 15
-        const uint4 v = *reinterpret_cast<const uint4*>(src + sw128(row, 4 * half + c));
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          o[8 * c + 2 * e] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(wv[e] & 0xFFFFu)));
-          o[8 * c + 2 * e + 1] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(wv[e] >> 16)));
-        }
-      }
-      const int slot = (w - t_begin) & 1;
-      tmem_st_32x32b_x32(tmem + kACol + slot * 64 + half * 32 + ((uint32_t)(quarter * 32) << 16), o);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sh.q_empty[qs]);
-      mbar_arrive(&sh.a_full[slot]);
-      if (++qs == kQS) { qs = 0; qph ^= 1; }
-      return true;
-    };
-    bool wok = true;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float hq = 0.5f * p.q_scale, hg = 0.5f * p.g_scale;
     if constexpr (kF8) {
-      if (t_begin < t_end) wok = widen(t_begin);
-    }
-    for (int tile = t_begin; tile < t_end; ++tile) {
-      const int u = tile / p.tiles_per_unit;
-      const int y = (tile % p.tiles_per_unit) * kRows;
-      const bool stall = p.stall == VDA_TEST_STALL_READOUT_GATE && blockIdx.x == 0 && tile == t_begin + 1;
-      if constexpr (kF8) {
-        if (wok && tile + 1 < t_end) wok = widen(tile + 1);   // the next tile's MMAs overlap this epilogue
-      }
-      bool ok = wok && !aborted(sh) && mbar_wait(&sh.t_full[tb], tph);
-      ok = ok && mbar_wait_or_stall(&sh.g_full[gs], gph, &sh.never, stall);
-      if (!ok) set_abort(sh, p.err);
-      // One decision for the half's four warps, which meet at its named
-      // barrier below: a warp that left alone would strand the others.
-      if (named_bar_or(1 + half, 128, !ok)) break;
-      tc_fence_after();
-      const float hq = 0.5f * p.q_scale, hg = 0.5f * p.g_scale;
-      const uint32_t taddr = tmem + tb * 128 + half * 64 + ((uint32_t)(quarter * 32) << 16);
-      if constexpr (kF8) {
-        // G from its 16 KB tile (one 128-byte row per token); O through the
-        // half's two 8 KB staging boxes in turn, 32 columns (64-byte rows) at
-        // a time, by TMA stores (rows past n clipped).
-        const uint8_t* g8row = gbuf + gs * kQT;
-        const bool leader = et % 128 == 0;
+      // e4m3: two groups of four warps take alternate tiles (the tile's
+      // parity: its accumulator and its A slot), all 128 columns each, so one
+      // group's gate and stores overlap the other's.  Per tile k of the group:
+      // the gate from TMEM and G, O through the group's two 8 KB staging
+      // boxes in turn (32 columns, 64-byte rows, TMA stores, rows past n
+      // clipped), and, before its last columns are read, the group's next
+      // tile's Q widened into its A slot (free: this tile's MMAs, which read
+      // it, are complete), so those MMAs overlap the rest of this tile.
+      const int grp = (warp - 2) / 4;
+      const bool leader = et % 128 == 0;
+      const uint32_t acc = tmem + grp * 128 + lane_off;
+      const uint32_t aslot = tmem + kACol + grp * 64 + lane_off;
+      const int K = t_end - t_begin;
+      auto widen = [&](int k) -> bool {       // tile t_begin + k's Q, this thread's row
+        const int qs = k % kQS;
+        bool ok = !aborted(sh) && mbar_wait(&sh.q_full[qs], (k / kQS) & 1);
+        if (!__all_sync(0xffffffffu, ok)) return false;   // the TMEM stores below are warp-wide
+        const uint8_t* src = qbuf + qs * kQT;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int h = 0; h < 2; ++h) {         // features 64 h .. 64 h + 63
+          uint32_t o[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {       // features 64 h + 16 c .. + 15
+            const uint4 v = *reinterpret_cast<const uint4*>(src + sw128(row, 4 * h + c));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              o[8 * c + 2 * e] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(wv[e] & 0xFFFFu)));
+              o[8 * c + 2 * e + 1] = f16x2_to_bf16x2_exact(e4m3x2_to_f16x2((uint16_t)(wv[e] >> 16)));
+            }
+          }
+          tmem_st_32x32b_x32(aslot + 32 * h, o);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sh.q_empty[qs]);
+        mbar_arrive(&sh.a_full[grp]);
+        return true;
+      };
+      bool ok = true;
+      if (grp < K) ok = widen(grp);
+      for (int k = grp; k < K; k += 2) {
+        const int tile = t_begin + k;
+        const int u = tile / p.tiles_per_unit;
+        const int y = (tile % p.tiles_per_unit) * kRows;
+        const int gs = k % kGS;
+        const bool stall = p.stall == VDA_TEST_STALL_READOUT_GATE && blockIdx.x == 0 && tile == t_begin + 1;
+        ok = ok && !aborted(sh) && mbar_wait(&sh.t_full[grp], (k >> 1) & 1);
+        ok = ok && mbar_wait_or_stall(&sh.g_full[gs], (k / kGS) & 1, &sh.never, stall);
+        if (!ok) set_abort(sh, p.err);
+        // One decision for the group's four warps, which meet at its named
+        // barrier below: a warp that left alone would strand the others.
+        if (named_bar_or(1 + grp, 128, !ok)) break;
+        tc_fence_after();
+        const uint8_t* g8row = gbuf + gs * kQT;
+        const TokPos opos = tok_pos(p.g, u, false);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {         // 32 columns at a time
+          // Before the last columns: the group's next tile into its A slot,
+          // then, with the accumulator read, that tile's MMAs may start.
+          if (c == 3 && k + 2 < K) ok = widen(k + 2);
           uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, r);
+          tmem_ld_32x32b_x32(acc + 32 * c, r);
           tmem_ld_wait();
+          if (c == 3) {
+            tc_fence_before();
+            mbar_arrive(&sh.t_empty[grp]);
+          }
           uint4 ch[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int f0 = half * 64 + c * 32 + q * 8;   // features f0 .. f0 + 7: half a 16-byte chunk
+            const int f0 = c * 32 + q * 8;    // features f0 .. f0 + 7: half a 16-byte chunk
             const uint2 gv = *reinterpret_cast<const uint2*>(g8row + sw128(row, f0 >> 4) + (f0 & 15));
             const uint32_t gw[2] = {gv.x, gv.y};
             uint32_t ow[4];
@@ -362,30 +370,46 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
             for (int e = 0; e < 4; ++e) {
               const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)(gw[e >> 1] >> (16 * (e & 1))));
               const float2 gf = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+              // sigmoid(g) d = (1 + tanh(g / 2)) d / 2: one special-function op.
               const float h0 = hq * __uint_as_float(r[q * 8 + 2 * e]);
               const float h1 = hq * __uint_as_float(r[q * 8 + 2 * e + 1]);
               ow[e] = pack_bf16(fmaf(h0, tanh_approx(hg * gf.x), h0), fmaf(h1, tanh_approx(hg * gf.y), h1));
             }
             ch[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
           }
-          if (c == 1) {
-            tc_fence_before();
-            mbar_arrive(&sh.t_empty[tb]);
-            mbar_arrive(&sh.g_empty[gs]);
-          }
-          uint8_t* ostg = ostage + (2 * half + c) * kOStage;
-          if (leader) bulk_wait_read<1>();       // the store two boxes back has read this one
-          named_bar_sync(1 + half, 128);
+          if (c == 3) mbar_arrive(&sh.g_empty[gs]);
+          uint8_t* ostg = ostage + (2 * grp + (c & 1)) * kOStage;
+          if (leader) bulk_wait_read<1>();     // the store two boxes back has read this one
+          named_bar_sync(1 + grp, 128);
 #pragma unroll
           for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(ostg + sw64(row, q)) = ch[q];
           fence_proxy_async_smem();
-          named_bar_sync(1 + half, 128);
+          named_bar_sync(1 + grp, 128);
           if (leader) {
-            tok_store(&p.mO, ostg, p.g, tok_pos(p.g, u, false), 64 * half + 32 * c, y);
+            tok_store(&p.mO, ostg, p.g, opos, 32 * c, y);
             bulk_commit();
           }
         }
-      } else {
+      }
+      if (leader) bulk_wait<0>();             // O stores complete before exit
+    } else {
+      // bf16: warps 2..5 take columns 0..63 and warps 6..9 columns 64..127
+      // of every tile (two warps per TMEM lane quarter).
+      const int half = (warp - 2) / 4;
+      int gs = 0, tb = 0;
+      uint32_t gph = 0, tph = 0;
+      for (int tile = t_begin; tile < t_end; ++tile) {
+        const int u = tile / p.tiles_per_unit;
+        const int y = (tile % p.tiles_per_unit) * kRows;
+        const bool stall = p.stall == VDA_TEST_STALL_READOUT_GATE && blockIdx.x == 0 && tile == t_begin + 1;
+        bool ok = !aborted(sh) && mbar_wait(&sh.t_full[tb], tph);
+        ok = ok && mbar_wait_or_stall(&sh.g_full[gs], gph, &sh.never, stall);
+        if (!ok) set_abort(sh, p.err);
+        // One decision for the half's four warps, which meet at its named
+        // barrier below: a warp that left alone would strand the others.
+        if (named_bar_or(1 + half, 128, !ok)) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem + tb * 128 + half * 64 + lane_off;
         // G is read from, and O written over, the G tile, then stored by TMA.
         uint8_t* rowp = gbuf + gs * kTile + half * kBox;
 #pragma unroll 1
@@ -421,12 +445,12 @@ __global__ void __launch_bounds__(kThreads, 1) readout_tc_kernel(const __grid_co
           bulk_wait_read<0>();
           mbar_arrive(&sh.g_empty[gs]);
         }
+        if (++gs == kGS) { gs = 0; gph ^= 1; }
+        tb ^= 1;
+        if (tb == 0) tph ^= 1;
       }
-      if (++gs == kGS) { gs = 0; gph ^= 1; }
-      tb ^= 1;
-      if (tb == 0) tph ^= 1;
+      if (et % 128 == 0) bulk_wait<0>();       // O stores complete before exit
     }
-    if (et % 128 == 0) bulk_wait<0>();         // O stores complete before exit
   } else if (warp < 18) {
     // ------------------------------------------------------------ S prep
     // S^f and S^b (bfloat16) of each frame of this CTA's range, in order.

@@ -106,6 +106,39 @@ def test_backward_wait_that_runs_out_reports_timeout(site):
         assert np.array_equal(a, b), site
 
 
+W8 = W.replace(name="stall_e4m3", dtype=synth.DTYPE_E4M3)
+
+
+@pytest.mark.parametrize("site", ["gram_stage", "factor_update", "service_gram", "readout_tile", "readout_gate",
+                                  "readout_state"])
+def test_e4m3_forward_wait_that_runs_out_reports_timeout(site):
+    """The e4m3 variants of the Gram+factor and readout kernels (their own loads, widening and epilogue)."""
+    import torch
+    from frame_wise_linear_b200 import vda
+    from vda_testutil import out_like
+    d = to_device(synth.make_inputs(W8, seed=5))
+    prob = vda.make_problem(**W8.problem())
+    ws = torch.empty(vda.vda_workspace_size(prob), dtype=torch.uint8, device="cuda")
+
+    def fwd(pr):
+        O = out_like(W8, d["G"])
+        vda.vda_forward(pr, d["Q"], d["K"], d["V"], d["G"], d["K_txt"], d["V_txt"], O, ws)
+        return O
+
+    ref = from_device(fwd(prob))
+    assert vda.vda_sync_status(ws, check=False) == vda.VDA_OK
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    fwd(vda.make_problem(**W8.problem(), test_stall=vda.TEST_STALL_SITES[site]))
+    status = vda.vda_sync_status(ws, check=False)
+    dt = time.perf_counter() - t0
+    assert status == vda.VDA_ERR_TIMEOUT, (site, vda.vda_status_string(status), vda.vda_last_error())
+    assert dt < BOUND_S, (site, dt)
+    again = from_device(fwd(prob))
+    assert vda.vda_sync_status(ws, check=False) == vda.VDA_OK
+    assert np.array_equal(again, ref), site
+
+
 def _merge(ws, stall=0):
     """One merge of 4096 tokens (32 row tiles, so the first CTA has one), K = 128, D = 256, both branches."""
     import torch
