@@ -14,21 +14,26 @@
 //     O_t = sigmoid(G_t) * softmax(Q_t K_S^T / sqrt(d)) V_S
 // bf16 Q, K, V, G, O; d = 128; float32 scores, softmax and accumulation.
 //
-// Design (persistent, one CTA per SM, 6 warps), work unit = 128 query tokens
+// Design (persistent, one CTA per SM, 10 warps), work unit = 128 query tokens
 // of one frame of one head; its key tiles are 128 tokens of one key frame (the
 // last tile of a frame partial) and then of the text:
-//   warp 0     TMA producer: the unit's Q tile, then K and V tiles through a
-//              2-stage ring (64 KB a stage).
+//   warp 0     TMA producer: the unit's Q tile, then K tiles through a
+//              3-stage ring and V tiles through a 2-stage ring (a K tile is
+//              free after its S MMAs, a V tile only after its P V).
 //   warp 1     TMEM and the MMAs: S_j = Q K_j^T into one of two 128-column
 //              score buffers, issued one tile ahead, and O += P_j V_j into a
-//              128-column accumulator once the softmax has written P_j.
-//   warps 2..5 softmax, one thread per query row: the row's scores from TMEM,
-//              the running maximum and sum (log2 domain), P_j = exp2 of the
-//              scaled scores as bf16 into shared memory; the accumulator is
-//              rescaled only when the maximum grows by more than 2^8 (the
-//              exponentials with a stale maximum stay below 2^8, and O and
-//              the sum share that maximum, so the quotient is exact).  After
-//              the last tile: O / sum, times sigmoid(G), stored from
+//              128-column accumulator once the softmax has written P_j, with
+//              P_j read from tensor memory (two 64-column slots).
+//   warps 2..9 softmax, two threads per query row (keys 0..63 and 64..127 of
+//              each tile, in the same TMEM lane quarter): the row's scores
+//              from TMEM, a tree for the half row's maximum, the partners'
+//              maxima swapped through shared memory, the running maximum and
+//              sum (log2 domain), P_j = exp2 of the scaled scores as bf16 into
+//              the P slot; the accumulator is rescaled only when the maximum
+//              grows by more than 2^8 (the exponentials with a stale maximum
+//              stay below 2^8, and O and the sum share that maximum, so the
+//              quotient is exact).  After the last tile: O / sum, times
+//              sigmoid(G), each thread its half of the columns, stored from
 //              registers as whole 128-byte row segments (8-lane transpose).
 // Every wait is bounded; a wait that runs out sets the timeout bit of the
 // error word and the CTA winds down.
@@ -41,14 +46,18 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 256;         // 8 warps: two threads per query row
+constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr int kKStages = 3;                  // K tiles in flight
+constexpr int kVStages = 2;                  // V tiles in flight (a V tile is held until its P V is done)
 constexpr int kRows = 128;                   // query and key tokens per tile
 constexpr int kBox = kRows * 64 * 2;         // 128 rows x 64 features bf16: 16 KB
 constexpr int kTile = 2 * kBox;              // 32 KB
 constexpr int kBlock = 5;                    // frames per block of the window
 constexpr float kRescale = 8.f;              // log2 growth of the maximum that forces a rescale
-constexpr uint32_t kTmemCols = 512;          // S0 | S1 | O
+constexpr uint32_t kTmemCols = 512;          // S0 | S1 | O | P0 | P1
 constexpr uint32_t kOCol = 256;
+constexpr uint32_t kPCol = 384;              // P slots: 64 columns (128 bf16 keys) each
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ false);   // Q K^T
 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, /*a MN*/ false, /*b MN*/ true);    // P V
 
@@ -67,7 +76,8 @@ struct LocalSoftmaxParams {
 
 struct Shared {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[2], kv_empty[2];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], pv_done[2];
   uint64_t o_free;
@@ -156,9 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qbuf = base;                      // Q tile, 32 KB
-  uint8_t* kvbuf = base + kTile;             // 2 stages: K tile | V tile
-  uint8_t* pbuf = kvbuf + 4 * kTile;         // 2 P tiles
-  Shared& sh = *reinterpret_cast<Shared*>(pbuf + 2 * kTile);
+  uint8_t* kbuf = qbuf + kTile;              // kKStages K tiles
+  uint8_t* vbuf = kbuf + kKStages * kTile;   // kVStages V tiles
+  float* xmax = reinterpret_cast<float*>(vbuf + kVStages * kTile);   // [2 parities][2 halves][128 rows]
+  float* xsum = xmax + 2 * 2 * kRows;                                 // [2 halves][128 rows]
+  Shared& sh = *reinterpret_cast<Shared*>(xsum + 2 * kRows);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -167,15 +179,21 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
   if (threadIdx.x == 0) {
     mbar_init(&sh.q_full, 1);
     mbar_init(&sh.q_empty, 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sh.k_full[i], 1);
+      mbar_init(&sh.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sh.v_full[i], 1);
+      mbar_init(&sh.v_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.kv_full[i], 1);
-      mbar_init(&sh.kv_empty[i], 1);
       mbar_init(&sh.s_full[i], 1);
-      mbar_init(&sh.s_free[i], 128);
-      mbar_init(&sh.p_full[i], 128);
+      mbar_init(&sh.s_free[i], kSoftmaxThreads);
+      mbar_init(&sh.p_full[i], kSoftmaxThreads);
       mbar_init(&sh.pv_done[i], 1);
     }
-    mbar_init(&sh.o_free, 128);
+    mbar_init(&sh.o_free, kSoftmaxThreads);
     mbar_init(&sh.drain, 1);
     mbar_init(&sh.never, 1);
     sh.abort = 0;
@@ -204,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
     if (lane == 0) {
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol_kv = policy_evict_last();   // a key frame serves 15 query frames
-      int kv_issued = 0, q_issued = 0, it = 0, ui = 0;
+      int k_issued = 0, v_issued = 0, q_issued = 0, it = 0, ui = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < units && ok; w += gridDim.x, ++ui) {
         const int qt = w % p.qtiles, t = (w / p.qtiles) % p.T, bh = w / (p.qtiles * p.T);
@@ -219,44 +237,46 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
         int cur = -2;
         TokPos kpos{};
         for (int j = 0; j < J; ++j, ++it) {
-          const int s = it & 1;
-          if (!(ok = mbar_wait(&sh.kv_empty[s], ((it >> 1) & 1) ^ 1))) break;
           const KeyTile kt = key_tile(p, kf, j);
           if (kt.frame != cur) {
             kpos = kt.text ? tok_pos(p.g, bh, true) : tok_pos(p.g, bh * p.T + kt.frame, false);
             cur = kt.frame;
           }
-          const CUtensorMap* mk = kt.text ? &p.mKt : &p.mK;
-          const CUtensorMap* mv = kt.text ? &p.mVt : &p.mV;
-          uint8_t* st = kvbuf + s * 2 * kTile;
-          mbar_expect_tx(&sh.kv_full[s], 2 * kTile);
-          tok_load(st, mk, &sh.kv_full[s], p.g, kpos, 0, kt.y, pol_kv);
-          tok_load(st + kBox, mk, &sh.kv_full[s], p.g, kpos, 64, kt.y, pol_kv);
-          tok_load(st + kTile, mv, &sh.kv_full[s], p.g, kpos, 0, kt.y, pol_kv);
-          tok_load(st + kTile + kBox, mv, &sh.kv_full[s], p.g, kpos, 64, kt.y, pol_kv);
-          ++kv_issued;
+          const int ks = it % kKStages, vs = it % kVStages;
+          if (!(ok = mbar_wait(&sh.k_empty[ks], ((it / kKStages) & 1) ^ 1))) break;
+          mbar_expect_tx(&sh.k_full[ks], kTile);
+          tok_load(kbuf + ks * kTile, kt.text ? &p.mKt : &p.mK, &sh.k_full[ks], p.g, kpos, 0, kt.y, pol_kv);
+          tok_load(kbuf + ks * kTile + kBox, kt.text ? &p.mKt : &p.mK, &sh.k_full[ks], p.g, kpos, 64, kt.y, pol_kv);
+          ++k_issued;
+          if (!(ok = mbar_wait(&sh.v_empty[vs], ((it / kVStages) & 1) ^ 1))) break;
+          mbar_expect_tx(&sh.v_full[vs], kTile);
+          tok_load(vbuf + vs * kTile, kt.text ? &p.mVt : &p.mV, &sh.v_full[vs], p.g, kpos, 0, kt.y, pol_kv);
+          tok_load(vbuf + vs * kTile + kBox, kt.text ? &p.mVt : &p.mV, &sh.v_full[vs], p.g, kpos, 64, kt.y, pol_kv);
+          ++v_issued;
         }
       }
       if (!ok) set_abort(sh, p.err);
       if (aborted(sh)) {   // the loads still in flight land before exit
-        for (int c = kv_issued > 2 ? kv_issued - 2 : 0; c < kv_issued; ++c)
-          mbar_wait(&sh.kv_full[c & 1], (c >> 1) & 1);
+        for (int c = k_issued > kKStages ? k_issued - kKStages : 0; c < k_issued; ++c)
+          mbar_wait(&sh.k_full[c % kKStages], (c / kKStages) & 1);
+        for (int c = v_issued > kVStages ? v_issued - kVStages : 0; c < v_issued; ++c)
+          mbar_wait(&sh.v_full[c % kVStages], (c / kVStages) & 1);
         if (q_issued > 0) mbar_wait(&sh.q_full, (q_issued - 1) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMAs
     if (lane == 0) {
-      const uint32_t qa = smem_u32(qbuf), kva = smem_u32(kvbuf), pa = smem_u32(pbuf);
-      int it = 0, ui = 0;   // global tile counter (ring and S / P buffers), unit counter
+      const uint32_t qa = smem_u32(qbuf), ka0 = smem_u32(kbuf), va0 = smem_u32(vbuf);
+      int it = 0, ui = 0;   // global tile counter (rings, S and P buffers), unit counter
       bool ok = true;
-      // S = Q K^T for the tile at ring position `pos` into S buffer pos & 1.
+      // S = Q K^T for the tile at position `pos` into S buffer pos & 1.
       auto issue_s = [&](int pos) -> bool {
-        const int s = pos & 1;
+        const int s = pos & 1, ks = pos % kKStages;
         if (!mbar_wait(&sh.s_free[s], ((pos >> 1) & 1) ^ 1)) return false;   // the softmax has read it
-        if (!mbar_wait(&sh.kv_full[s], (pos >> 1) & 1)) return false;
+        if (!mbar_wait(&sh.k_full[ks], (pos / kKStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t ka = kva + s * 2 * kTile;
+        const uint32_t ka = ka0 + ks * kTile;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k / 4) * kBox + (k % 4) * 32;
@@ -264,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
                       smem_desc(ka + off, 16, 1024, kSwizzle128B), kIdescS, k ? 1u : 0u);
         }
         mma_commit(&sh.s_full[s]);
+        mma_commit(&sh.k_empty[ks]);
         return true;
       };
       for (int w = blockIdx.x; w < units && ok; w += gridDim.x, ++ui) {
@@ -272,20 +293,22 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
         if (!(ok = mbar_wait(&sh.q_full, ui & 1))) break;
         if (!(ok = issue_s(it))) break;
         for (int j = 0; j < J && ok; ++j) {
-          const int pos = it + j, s = pos & 1;
+          const int pos = it + j, s = pos & 1, vs = pos % kVStages;
           if (j + 1 < J && !(ok = issue_s(pos + 1))) break;
           if (j + 1 == J) mma_commit(&sh.q_empty);   // the unit's last S MMAs read Q before anything after
           if (j == 0 && !(ok = mbar_wait(&sh.o_free, (ui & 1) ^ 1))) break;   // the previous unit's O is read
           if (!(ok = mbar_wait(&sh.p_full[s], (pos >> 1) & 1))) break;
+          if (!(ok = mbar_wait(&sh.v_full[vs], (pos / kVStages) & 1))) break;
           tc_fence_after();
-          const uint32_t va = kva + s * 2 * kTile + kTile, pb = pa + s * kTile;
+          // O += P V: P (K-major, 16 keys = 8 columns a step) from tensor
+          // memory, V (MN-major) from shared memory.
+          const uint32_t va = va0 + vs * kTile;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            mma_bf16_ss(tmem + kOCol, smem_desc(pb + (k / 4) * kBox + (k % 4) * 32, 16, 1024, kSwizzle128B),
+          for (int k = 0; k < 8; ++k)
+            mma_bf16_ts(tmem + kOCol, tmem + kPCol + s * 64 + 8 * k,
                         smem_desc(va + k * 16 * 128, kBox, 1024, kSwizzle128B), kIdescO, (j | k) ? 1u : 0u);
-          }
           mma_commit(&sh.pv_done[s]);
-          mma_commit(&sh.kv_empty[s]);
+          mma_commit(&sh.v_empty[vs]);
         }
         it += J;
       }
@@ -295,8 +318,16 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int row = (warp % 4) * 32 + lane;   // query row = TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    // Two threads per query row: warps 2..5 take keys (and O columns) 0..63,
+    // warps 6..9 keys 64..127, in the same TMEM lane quarter.  The partners
+    // swap their partial row maxima (and at the end their partial sums)
+    // through shared memory at a named barrier of the quarter's two warps,
+    // which is also where they decide together to stop after a timeout.
+    const int quarter = warp % 4;
+    const int half = (warp - 2) / 4;
+    const int row = quarter * 32 + lane;       // query row = TMEM lane
+    const int bar = 1 + quarter;               // named barrier of the row's two threads (64 threads)
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const size_t rstride = tok_row_stride(p.g);
     int it = 0, ui = 0;
     bool ok = true;
@@ -309,110 +340,139 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
         const int pos = it + j, s = pos & 1;
         const KeyTile kt = key_tile(p, kf, j);
         const bool stall = p.stall == VDA_TEST_STALL_SOFTMAX && blockIdx.x == 0 && pos == 0;
-        if (!(ok = !aborted(sh) && mbar_wait_or_stall(&sh.s_full[s], (pos >> 1) & 1, &sh.never, stall))) break;
-        tc_fence_after();
-        float x[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + s * 128 + lane_off + c * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
-        }
-        tc_fence_before();
-        mbar_arrive(&sh.s_free[s]);            // the MMAs may write the next scores here
+        ok = !aborted(sh) && mbar_wait_or_stall(&sh.s_full[s], (pos >> 1) & 1, &sh.never, stall);
+        // P_j's slot is free once PV_{j-2} is done.
+        ok = ok && (j < 2 || mbar_wait(&sh.pv_done[s], ((pos - 2) >> 1) & 1));
+        ok = __all_sync(0xffffffffu, ok);    // the TMEM loads below are warp-wide
+        float x[64];
         float mt = -INFINITY;
+        if (ok) {
+          tc_fence_after();
+          uint32_t xr[64];
+          const uint32_t sa = tmem + s * 128 + lane_off + half * 64;
+          tmem_ld_32x32b_x32(sa, *reinterpret_cast<uint32_t(*)[32]>(&xr[0]));
+          tmem_ld_32x32b_x32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32]));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&sh.s_free[s]);          // the MMAs may write the next scores here
+          // scores in log2 units; keys past the tile's valid ones excluded
+          const int valid = kt.valid - half * 64;
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          x[e] = e < kt.valid ? x[e] * p.c : -INFINITY;   // scores in log2 units; rows past the keys excluded
-          mt = fmaxf(mt, x[e]);
+          for (int e = 0; e < 64; ++e) x[e] = e < valid ? __uint_as_float(xr[e]) * p.c : -INFINITY;
+          // the half row's maximum by a pairwise tree (depth 6, not a chain of 64)
+          float tm[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) tm[i] = fmaxf(x[2 * i], x[2 * i + 1]);
+#pragma unroll
+          for (int w2 = 16; w2 >= 1; w2 >>= 1) {
+#pragma unroll
+            for (int i = 0; i < w2; ++i) tm[i] = fmaxf(tm[2 * i], tm[2 * i + 1]);
+          }
+          mt = tm[0];
         }
-        // P_j's buffer is free once PV_{j-2} is done, and a rescale of O needs PV_{j-1} done.
+        if (!ok) set_abort(sh, p.err);
+        xmax[(s * 2 + half) * kRows + row] = mt;
+        if (named_bar_or(bar, 64, !ok)) {       // one decision for the row's two threads
+          ok = false;                          // (both leave every loop: no barrier left unmet)
+          break;
+        }
+        mt = fmaxf(mt, xmax[(s * 2 + (half ^ 1)) * kRows + row]);
+        // A rescale of O needs PV_{j-1} done; the row's two threads take the
+        // same decision (the same m and mt), each for its half of O.
         const bool grow = j == 0 || mt > m + kRescale;
-        if (j >= 2 && !(ok = mbar_wait(&sh.pv_done[s], ((pos - 2) >> 1) & 1))) break;
         if (grow) {
           const float mn = fmaxf(m, mt);
           if (j >= 1) {
-            if (!(ok = mbar_wait(&sh.pv_done[s ^ 1], ((pos - 1) >> 1) & 1))) break;
+            ok = mbar_wait(&sh.pv_done[s ^ 1], ((pos - 1) >> 1) & 1);
+            if (!ok) set_abort(sh, p.err);
+            if (named_bar_or(bar, 64, !ok)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const float a = ex2(m - mn);
             l *= a;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
               uint32_t r[32];
-              tmem_ld_32x32b_x32(tmem + kOCol + lane_off + c * 32, r);
+              const uint32_t oa = tmem + kOCol + lane_off + half * 64 + c * 32;
+              tmem_ld_32x32b_x32(oa, r);
               tmem_ld_wait();
 #pragma unroll
               for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(a * __uint_as_float(r[e]));
-              tmem_st_32x32b_x32(tmem + kOCol + lane_off + c * 32, r);
+              tmem_st_32x32b_x32(oa, r);
             }
             tmem_st_wait();
           }
           m = mn;
         }
-        uint8_t* pt = pbuf + s * kTile;
+        // P = 2^(x - m) as bf16 pairs into the tile's P slot (keys 64 half ..
+        // 64 half + 63 are columns 32 half .. 32 half + 31).
+        {
+          uint32_t pw[32];
+          float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {           // keys 8c .. 8c + 7
-          float v[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            v[e] = ex2(x[8 * c + e] - m);
-            l += v[e];
+          for (int e = 0; e < 32; ++e) {
+            const float v0 = ex2(x[2 * e] - m), v1 = ex2(x[2 * e + 1] - m);
+            lp[e & 3] += v0 + v1;
+            pw[e] = pack_bf16(v0, v1);
           }
-          *reinterpret_cast<uint4*>(pt + (c >> 3) * kBox + sw128(row, c & 7)) =
-              make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+          l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+          tmem_st_32x32b_x32(tmem + kPCol + s * 64 + lane_off + half * 32, pw);
+          tmem_st_wait();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sh.p_full[s]);
       }
       if (!ok) break;
-      // ---- epilogue: O / l times sigmoid(G), rows past n skipped
+      // ---- epilogue: O / l times sigmoid(G), this thread's half of the
+      // columns; rows past n skipped.
       const int last = it + J - 1;
-      if (!(ok = !aborted(sh) && mbar_wait(&sh.pv_done[last & 1], (last >> 1) & 1))) break;
+      ok = !aborted(sh) && mbar_wait(&sh.pv_done[last & 1], (last >> 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) set_abort(sh, p.err);
+      xsum[half * kRows + row] = l;
+      if (named_bar_or(bar, 64, !ok)) {
+        ok = false;
+        break;
+      }
+      const float inv = 1.f / (l + xsum[(half ^ 1) * kRows + row]);
       tc_fence_after();
       const TokPos qpos = tok_pos(p.g, bh * p.T + t, false);
       const size_t obase = tok_base(p.g, qpos, p.n, false);
       const int tok = qt * kRows + row;
-      const float inv = 1.f / l;
-      const int r0 = (warp % 4) * 32 + 8 * (lane >> 3);
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {          // 64 columns at a time
-        uint4 ch[8];
+      const int r0 = quarter * 32 + 8 * (lane >> 3);
+      uint4 ch[8];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + kOCol + lane_off + hf * 64 + c * 32, r);
-          tmem_ld_wait();
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + kOCol + lane_off + half * 64 + c * 32, r);
+        tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = hf * 64 + c * 32 + q * 8;
-            uint4 gv = make_uint4(0, 0, 0, 0);
-            if (tok < p.n) gv = *reinterpret_cast<const uint4*>(p.G + obase + (size_t)tok * rstride + col);
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
-            uint32_t ow[4];
+        for (int q = 0; q < 4; ++q) {
+          const int col = half * 64 + c * 32 + q * 8;
+          uint4 gv = make_uint4(0, 0, 0, 0);
+          if (tok < p.n) gv = *reinterpret_cast<const uint4*>(p.G + obase + (size_t)tok * rstride + col);
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+          uint32_t ow[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 gf = __bfloat1622float2(g2[e]);
-              // sigmoid(g) x = (1 + tanh(g / 2)) x / 2
-              const float h0 = 0.5f * inv * __uint_as_float(r[q * 8 + 2 * e]);
-              const float h1 = 0.5f * inv * __uint_as_float(r[q * 8 + 2 * e + 1]);
-              ow[e] = pack_bf16(fmaf(h0, tanh_approx(0.5f * gf.x), h0), fmaf(h1, tanh_approx(0.5f * gf.y), h1));
-            }
-            ch[c * 4 + q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+          for (int e = 0; e < 4; ++e) {
+            const float2 gf = __bfloat1622float2(g2[e]);
+            // sigmoid(g) x = (1 + tanh(g / 2)) x / 2
+            const float h0 = 0.5f * inv * __uint_as_float(r[q * 8 + 2 * e]);
+            const float h1 = 0.5f * inv * __uint_as_float(r[q * 8 + 2 * e + 1]);
+            ow[e] = pack_bf16(fmaf(h0, tanh_approx(0.5f * gf.x), h0), fmaf(h1, tanh_approx(0.5f * gf.y), h1));
           }
+          ch[c * 4 + q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
-        if (hf == 1) {
-          tc_fence_before();
-          mbar_arrive(&sh.o_free);               // the next unit's first PV may overwrite O
-        }
-        transpose8(ch, lane & 7);
+      }
+      tc_fence_before();
+      mbar_arrive(&sh.o_free);                 // the next unit's first PV may overwrite O
+      transpose8(ch, lane & 7);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int tr = qt * kRows + r0 + k;
-          if (tr < p.n) *reinterpret_cast<uint4*>(p.O + obase + (size_t)tr * rstride + hf * 64 + (lane & 7) * 8) = ch[k];
-        }
+      for (int k = 0; k < 8; ++k) {
+        const int tr = qt * kRows + r0 + k;
+        if (tr < p.n) *reinterpret_cast<uint4*>(p.O + obase + (size_t)tr * rstride + half * 64 + (lane & 7) * 8) = ch[k];
       }
       it += J;
     }
@@ -450,7 +510,7 @@ cudaError_t launch_local_softmax_tc(const vda_problem& p, const __nv_bfloat16* Q
   prm.c = 1.4426950408889634f / sqrtf((float)p.d_k);
   prm.g = TokGeom{p.layout, p.H, p.T};
   prm.stall = p.test_stall;
-  const size_t smem = 1024 + 7 * kTile + sizeof(Shared);
+  const size_t smem = 1024 + (1 + kKStages + kVStages) * kTile + 3 * 2 * kRows * sizeof(float) + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(local_softmax_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
