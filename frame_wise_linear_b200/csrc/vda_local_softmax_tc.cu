@@ -14,14 +14,14 @@
 //     O_t = sigmoid(G_t) * softmax(Q_t K_S^T / sqrt(d)) V_S
 // bf16 Q, K, V, G, O; d = 128; float32 scores, softmax and accumulation.
 //
-// Design (persistent, one CTA per SM, 10 warps), work unit = 128 query tokens
+// Design (persistent, one CTA per SM, 11 warps), work unit = 128 query tokens
 // of one frame of one head; its key tiles are 128 tokens of one key frame (the
 // last tile of a frame partial) and then of the text:
-//   warp 0     TMA producer: the unit's Q tile, then K tiles through a
-//              3-stage ring and V tiles through a 2-stage ring (a K tile is
-//              free after its S MMAs, a V tile only after its P V).
+//   warps 0, 10 TMA producers: warp 0 the unit's Q tile and K tiles through a
+//              3-stage ring, warp 10 V tiles through a 2-stage ring (a K tile
+//              is free after its S MMAs, a V tile only after its P V).
 //   warp 1     TMEM and the MMAs: S_j = Q K_j^T into one of two 128-column
-//              score buffers, issued one tile ahead, and O += P_j V_j into a
+//              score buffers, issued two tiles ahead, and O += P_j V_j into a
 //              128-column accumulator once the softmax has written P_j, with
 //              P_j read from tensor memory (two 64-column slots).
 //   warps 2..9 softmax, two threads per query row (keys 0..63 and 64..127 of
@@ -47,7 +47,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kSoftmaxThreads = 256;         // 8 warps: two threads per query row
-constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr int kVWarp = 2 + kSoftmaxThreads / 32;   // the V producer, after the softmax warps
+constexpr int kThreads = 32 * (kVWarp + 1);
 constexpr int kKStages = 3;                  // K tiles in flight
 constexpr int kVStages = 2;                  // V tiles in flight (a V tile is held until its P V is done)
 constexpr int kRows = 128;                   // query and key tokens per tile
@@ -217,21 +218,30 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == kVWarp) {
+    // ------------------------------------------------------------ producers
+    // Warp 0 loads Q and the K tiles, the last warp the V tiles: a V stage is
+    // freed only by its P V, late, and K loads must not queue behind it.
     if (lane == 0) {
+      const bool kl = warp == 0;
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol_kv = policy_evict_last();   // a key frame serves 15 query frames
-      int k_issued = 0, v_issued = 0, q_issued = 0, it = 0, ui = 0;
+      const int stages = kl ? kKStages : kVStages;
+      uint64_t* full = kl ? sh.k_full : sh.v_full;
+      uint64_t* empty = kl ? sh.k_empty : sh.v_empty;
+      uint8_t* ring = kl ? kbuf : vbuf;
+      int issued = 0, q_issued = 0, it = 0, ui = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < units && ok; w += gridDim.x, ++ui) {
         const int qt = w % p.qtiles, t = (w / p.qtiles) % p.T, bh = w / (p.qtiles * p.T);
-        const TokPos qpos = tok_pos(p.g, bh * p.T + t, false);
-        if (!(ok = mbar_wait(&sh.q_empty, (ui & 1) ^ 1))) break;   // the previous unit's S MMAs are done
-        mbar_expect_tx(&sh.q_full, kTile);
-        tok_load(qbuf, &p.mQ, &sh.q_full, p.g, qpos, 0, qt * kRows, pol_q);
-        tok_load(qbuf + kBox, &p.mQ, &sh.q_full, p.g, qpos, 64, qt * kRows, pol_q);
-        ++q_issued;
+        if (kl) {
+          const TokPos qpos = tok_pos(p.g, bh * p.T + t, false);
+          if (!(ok = mbar_wait(&sh.q_empty, (ui & 1) ^ 1))) break;   // the previous unit's S MMAs are done
+          mbar_expect_tx(&sh.q_full, kTile);
+          tok_load(qbuf, &p.mQ, &sh.q_full, p.g, qpos, 0, qt * kRows, pol_q);
+          tok_load(qbuf + kBox, &p.mQ, &sh.q_full, p.g, qpos, 64, qt * kRows, pol_q);
+          ++q_issued;
+        }
         const KeyFrames kf = key_frames(t, p.T);
         const int J = key_tiles(p, kf);
         int cur = -2;
@@ -242,25 +252,18 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
             kpos = kt.text ? tok_pos(p.g, bh, true) : tok_pos(p.g, bh * p.T + kt.frame, false);
             cur = kt.frame;
           }
-          const int ks = it % kKStages, vs = it % kVStages;
-          if (!(ok = mbar_wait(&sh.k_empty[ks], ((it / kKStages) & 1) ^ 1))) break;
-          mbar_expect_tx(&sh.k_full[ks], kTile);
-          tok_load(kbuf + ks * kTile, kt.text ? &p.mKt : &p.mK, &sh.k_full[ks], p.g, kpos, 0, kt.y, pol_kv);
-          tok_load(kbuf + ks * kTile + kBox, kt.text ? &p.mKt : &p.mK, &sh.k_full[ks], p.g, kpos, 64, kt.y, pol_kv);
-          ++k_issued;
-          if (!(ok = mbar_wait(&sh.v_empty[vs], ((it / kVStages) & 1) ^ 1))) break;
-          mbar_expect_tx(&sh.v_full[vs], kTile);
-          tok_load(vbuf + vs * kTile, kt.text ? &p.mVt : &p.mV, &sh.v_full[vs], p.g, kpos, 0, kt.y, pol_kv);
-          tok_load(vbuf + vs * kTile + kBox, kt.text ? &p.mVt : &p.mV, &sh.v_full[vs], p.g, kpos, 64, kt.y, pol_kv);
-          ++v_issued;
+          const int st = it % stages;
+          if (!(ok = mbar_wait(&empty[st], ((it / stages) & 1) ^ 1))) break;
+          const CUtensorMap* map = kl ? (kt.text ? &p.mKt : &p.mK) : (kt.text ? &p.mVt : &p.mV);
+          mbar_expect_tx(&full[st], kTile);
+          tok_load(ring + st * kTile, map, &full[st], p.g, kpos, 0, kt.y, pol_kv);
+          tok_load(ring + st * kTile + kBox, map, &full[st], p.g, kpos, 64, kt.y, pol_kv);
+          ++issued;
         }
       }
       if (!ok) set_abort(sh, p.err);
       if (aborted(sh)) {   // the loads still in flight land before exit
-        for (int c = k_issued > kKStages ? k_issued - kKStages : 0; c < k_issued; ++c)
-          mbar_wait(&sh.k_full[c % kKStages], (c / kKStages) & 1);
-        for (int c = v_issued > kVStages ? v_issued - kVStages : 0; c < v_issued; ++c)
-          mbar_wait(&sh.v_full[c % kVStages], (c / kVStages) & 1);
+        for (int c = issued > stages ? issued - stages : 0; c < issued; ++c) mbar_wait(&full[c % stages], (c / stages) & 1);
         if (q_issued > 0) mbar_wait(&sh.q_full, (q_issued - 1) & 1);
       }
     }
@@ -291,11 +294,20 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
         const int t = (w / p.qtiles) % p.T;
         const int J = key_tiles(p, key_frames(t, p.T));
         if (!(ok = mbar_wait(&sh.q_full, ui & 1))) break;
-        if (!(ok = issue_s(it))) break;
+        // S runs two tiles ahead of P V (an MMA issue waits while the tensor
+        // pipe is busy, so S_{j+2} goes in before P_j V_j, not after it).
+        int ns = 0;                            // the unit's next S tile
+        auto next_s = [&]() -> bool {
+          if (!issue_s(it + ns)) return false;
+          if (++ns == J) mma_commit(&sh.q_empty);   // the unit's last S MMAs read Q before anything after
+          return true;
+        };
+        if (!(ok = next_s())) break;
+        if (ns < J && !(ok = next_s())) break;
         for (int j = 0; j < J && ok; ++j) {
           const int pos = it + j, s = pos & 1, vs = pos % kVStages;
-          if (j + 1 < J && !(ok = issue_s(pos + 1))) break;
-          if (j + 1 == J) mma_commit(&sh.q_empty);   // the unit's last S MMAs read Q before anything after
+          // S_{j+2}: its buffer is S_j's, free once the softmax has read S_j
+          if (ns < J && !(ok = next_s())) break;
           if (j == 0 && !(ok = mbar_wait(&sh.o_free, (ui & 1) ^ 1))) break;   // the previous unit's O is read
           if (!(ok = mbar_wait(&sh.p_full[s], (pos >> 1) & 1))) break;
           if (!(ok = mbar_wait(&sh.v_full[vs], (pos / kVStages) & 1))) break;
@@ -316,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
       mma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
     }
-  } else {
+  } else if (warp < kVWarp) {
     // ------------------------------------------------------------ softmax + epilogue
     // Two threads per query row: warps 2..5 take keys (and O columns) 0..63,
     // warps 6..9 keys 64..127, in the same TMEM lane quarter.  The partners
@@ -335,10 +347,18 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
       const int qt = w % p.qtiles, t = (w / p.qtiles) % p.T, bh = w / (p.qtiles * p.T);
       const KeyFrames kf = key_frames(t, p.T);
       const int J = key_tiles(p, kf);
+      const int nft = kf.count() * p.qtiles;   // the key frames' tiles (then the text's)
+      int fy = 0;                              // tile of the current key frame
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < J; ++j) {
         const int pos = it + j, s = pos & 1;
-        const KeyTile kt = key_tile(p, kf, j);
+        int kvalid;                            // keys in this tile
+        if (j < nft) {
+          kvalid = fy == p.qtiles - 1 ? p.n - fy * kRows : kRows;
+          if (++fy == p.qtiles) fy = 0;
+        } else {
+          kvalid = min(kRows, p.n_txt - (j - nft) * kRows);
+        }
         const bool stall = p.stall == VDA_TEST_STALL_SOFTMAX && blockIdx.x == 0 && pos == 0;
         ok = !aborted(sh) && mbar_wait_or_stall(&sh.s_full[s], (pos >> 1) & 1, &sh.never, stall);
         // P_j's slot is free once PV_{j-2} is done.
@@ -355,11 +375,16 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
           tmem_ld_wait();
           tc_fence_before();
           mbar_arrive(&sh.s_free[s]);          // the MMAs may write the next scores here
-          // scores in log2 units; keys past the tile's valid ones excluded
-          const int valid = kt.valid - half * 64;
+          // raw scores; keys past the tile's valid ones excluded
 #pragma unroll
-          for (int e = 0; e < 64; ++e) x[e] = e < valid ? __uint_as_float(xr[e]) * p.c : -INFINITY;
-          // the half row's maximum by a pairwise tree (depth 6, not a chain of 64)
+          for (int e = 0; e < 64; ++e) x[e] = __uint_as_float(xr[e]);
+          const int valid = kvalid - half * 64;
+          if (valid < 64) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) x[e] = e < valid ? x[e] : -INFINITY;
+          }
+          // the half row's maximum by a pairwise tree (depth 6, not a chain of
+          // 64), in log2 units (the scale is positive)
           float tm[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) tm[i] = fmaxf(x[2 * i], x[2 * i + 1]);
@@ -368,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
 #pragma unroll
             for (int i = 0; i < w2; ++i) tm[i] = fmaxf(tm[2 * i], tm[2 * i + 1]);
           }
-          mt = tm[0];
+          mt = tm[0] * p.c;
         }
         if (!ok) set_abort(sh, p.err);
         xmax[(s * 2 + half) * kRows + row] = mt;
@@ -406,14 +431,14 @@ __global__ void __launch_bounds__(kThreads, 1) local_softmax_tc_kernel(const __g
           }
           m = mn;
         }
-        // P = 2^(x - m) as bf16 pairs into the tile's P slot (keys 64 half ..
+        // P = 2^(c x - m) as bf16 pairs into the tile's P slot (keys 64 half ..
         // 64 half + 63 are columns 32 half .. 32 half + 31).
         {
           uint32_t pw[32];
           float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float v0 = ex2(x[2 * e] - m), v1 = ex2(x[2 * e + 1] - m);
+            const float v0 = ex2(fmaf(x[2 * e], p.c, -m)), v1 = ex2(fmaf(x[2 * e + 1], p.c, -m));
             lp[e & 3] += v0 + v1;
             pw[e] = pack_bf16(v0, v1);
           }
