@@ -135,13 +135,19 @@ def path_roofline(w, peaks):
                 bound="hbm" if t_hbm >= t_tc else "tensor")
 
 
+# The other lines' kernels (bf16 only).
+KERNEL_SOURCES = {"merge": "frame_wise_linear_b200/csrc/vda_merge_tc.cu",
+                  "softmax": "frame_wise_linear_b200/csrc/vda_local_softmax_tc.cu"}
+
+
 def traffic_lookup(stage, w):
     """DRAM bytes per launch of a stage's kernel on workload `w`, from the committed ncu summary,
     if the kernel's source is unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(path) or stage not in STAGE_SOURCES[w.dtype]:
+    srcs = dict(STAGE_SOURCES[w.dtype], **KERNEL_SOURCES)
+    if not os.path.exists(path) or stage not in srcs:
         return None
-    src = os.path.join(ROOT, STAGE_SOURCES[w.dtype][stage])
+    src = os.path.join(ROOT, srcs[stage])
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     with open(path) as fh:
         for line in fh:
@@ -758,8 +764,8 @@ def run_merge(args, w):
                    "tokens": tokens, "K": K, "D": D, "l2": "inputs larger than L2; no flush"},
         "roofline": {"kernel": "merge_tc_kernel", "bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
-                     "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json bf16_tflops)", "traffic": None,
-                     "algorithmic_bytes": bytes_},
+                     "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json bf16_tflops)",
+                     "traffic": traffic_lookup("merge", w), "algorithmic_bytes": bytes_},
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -830,8 +836,8 @@ def run_softmax(args, w):
         "config": config_of(w, 1),
         "roofline": {"kernel": "local_softmax_tc_kernel", "bound": "tensor", "achieved": tf,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
-                     "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json bf16_tflops)", "traffic": None,
-                     "flops": softmax_work(w)},
+                     "peak_source": f"{peaks_kind} (MEASURED_PEAKS.json bf16_tflops)",
+                     "traffic": traffic_lookup("softmax", w), "flops": softmax_work(w)},
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
