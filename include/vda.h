@@ -24,7 +24,7 @@
  * vda_problem.layout = VDA_LAYOUT_BHTND (0, the default):
  *     Q, K : [B, H, T, n, d_k]      V, G, O : [B, H, T, n, d_v]
  *     K_txt: [B, H, n_txt, d_k]     V_txt   : [B, H, n_txt, d_v]
- * With VDA_LAYOUT_BTNHD (1; bfloat16 only), the token-major layout of a
+ * With VDA_LAYOUT_BTNHD (1; bfloat16 or e4m3), the token-major layout of a
  * video transformer's attention, heads inside tokens:
  *     Q, K : [B, T*n, H, d_k]       V, G, O : [B, T*n, H, d_v]
  *     K_txt: [B, n_txt, H, d_k]     V_txt   : [B, n_txt, H, d_v]
@@ -93,7 +93,7 @@ typedef struct vda_problem {
   int32_t B, H, T, n, n_txt, d_k, d_v;
   int32_t dtype; /* vda_dtype */
   float lambda;
-  int32_t layout; /* vda_layout; VDA_LAYOUT_BTNHD needs bfloat16 */
+  int32_t layout; /* vda_layout; VDA_LAYOUT_BTNHD needs bfloat16 or e4m3 */
   int32_t test_stall; /* testing hook, VDA_TEST_STALL_*; 0 in normal use */
   /* e4m3 inputs only (ignored otherwise): the value an element stands for is
    * scale times its stored e4m3 value, one scale per tensor (K_txt takes
