@@ -25,15 +25,17 @@
 //     shared memory as hi / lo K-major images, and 48 MMAs (K = 256: G_0 S_0^T
 //     and S_0 G_0^T, three passes) give W1_0.  The text's rows are stored from
 //     registers.
-//   frames next, a contiguous range per CTA:
+//   frames next, a contiguous range per CTA (a CTA that ran a text chain
+//   takes about 8 frames fewer):
 //     warp 0     TMA producer: per frame two half-units, (Gf, S^f) and then
 //                (Gb, S^b), 64 KB each, through a 2-slot ring.
 //     warp 1     TMEM and the 32 MMAs of a frame (16 per half-unit) into one
 //                of two 128-column accumulators.
 //     warps 2..5 epilogue: W1 = -acc and dB = Gf + Gb (the bf16 adjoints, read
 //                from global memory, where the producer's loads have just
-//                brought them into L2) through two 32 KB staging boxes, TMA
-//                stores into the [frames][256][128] operand image.
+//                brought them into L2, before the wait for the frame's MMAs)
+//                through two 32 KB staging boxes, TMA stores into the
+//                [frames][256][128] operand image.
 // Every wait is bounded; a wait that runs out sets the timeout bit of the
 // error word and the CTA winds down.
 #include "sm100.cuh"
@@ -64,6 +66,7 @@ struct BwdOperandsParams {
   __nv_bfloat16* Wt;                // [heads][256][128] bf16: the text's W1_0 | dB_0 (NULL: no text)
   unsigned* err;
   int frames, heads, T;
+  int text_weight;                  // frames a head's text chain counts for in the frame split
   float inv_lam;
   int stall;                        // testing hook: a VDA_TEST_STALL_* site, 0 in normal use
 };
@@ -291,8 +294,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_operands_tc_kernel(const __gr
   }
 
   // ---------------------------------------------------------------- frames
-  const int f_begin = (int)((long long)p.frames * blockIdx.x / gridDim.x);
-  const int f_end = (int)((long long)p.frames * (blockIdx.x + 1) / gridDim.x);
+  // Contiguous frame ranges, with each text chain counted as text_weight
+  // frames of its CTA's share (the CTAs that ran a text chain take fewer
+  // frames).  Split points b(c) = V(c) - w * texts(< c), V(c) = total c / grid:
+  // b(0) = 0, b(grid) = frames, and the host keeps b non-decreasing.
+  auto split = [&](int c) -> int {
+    const long long w = p.Wt ? p.text_weight : 0;
+    const long long total = p.frames + w * p.heads;
+    const long long texts = min((long long)c, (long long)p.heads);   // heads of the CTAs before c (one each)
+    return (int)(total * c / gridDim.x - w * texts);
+  };
+  const int f_begin = split(blockIdx.x);
+  const int f_end = split(blockIdx.x + 1);
   const int J = f_end - f_begin;
   if (warp == 0) {
     if (lane == 0 && !aborted(sh)) {
@@ -328,7 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_operands_tc_kernel(const __gr
 #pragma unroll 1
         for (int h = 0; h < 2 && ok; ++h) {   // (Gf, S^f), then (Gb, S^b)
           const int hj = 2 * j + h;
-          const bool stall = p.stall == VDA_TEST_STALL_OPERANDS && blockIdx.x == 0 && hj == 0;
+          // (the last CTA: it runs no text chain and always has frames)
+          const bool stall = p.stall == VDA_TEST_STALL_OPERANDS && blockIdx.x == gridDim.x - 1 && hj == 0;
           if (!(ok = mbar_wait_or_stall(&sh.full[h], (hj >> 1) & 1, &sh.never, stall))) break;
           tc_fence_after();
           const uint32_t g = smem_u32(ring + h * kSlot), sv = g + kMat;
@@ -355,6 +369,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_operands_tc_kernel(const __gr
     for (int j = 0; j < J; ++j) {
       const int tb = j & 1;
       const int f = f_begin + j;
+      // dB's operands, the row of Gf and of Gb (bf16, just brought into L2 by
+      // the producer's loads), loaded before the wait so that their latency
+      // overlaps the frame's MMAs.
+      uint4 ga[16], gb[16];
+      {
+        const __nv_bfloat16* gf = p.Gf + ((size_t)f * 128 + row) * 128;
+        const __nv_bfloat16* gbp = p.Gb + ((size_t)f * 128 + row) * 128;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          ga[c] = *reinterpret_cast<const uint4*>(gf + 8 * c);
+          gb[c] = *reinterpret_cast<const uint4*>(gbp + 8 * c);
+        }
+      }
       bool ok = !aborted(sh) && mbar_wait(&sh.t_full[tb], (j >> 1) & 1);
       if (!ok) set_abort(sh, p.err);
       if (named_bar_or(kEpiBar, 128, !ok)) break;   // one decision for the four warps
@@ -376,14 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_operands_tc_kernel(const __gr
       }
       tc_fence_before();
       mbar_arrive(&sh.t_empty[tb]);
-      const __nv_bfloat16* gf = p.Gf + ((size_t)f * 128 + row) * 128;
-      const __nv_bfloat16* gb = p.Gb + ((size_t)f * 128 + row) * 128;
-#pragma unroll 4
+#pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const uint4 a = *reinterpret_cast<const uint4*>(gf + 8 * c);
-        const uint4 b = *reinterpret_cast<const uint4*>(gb + 8 * c);
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ga[c]);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&gb[c]);
         float v[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -442,6 +465,11 @@ cudaError_t launch_bwd_operands_tc(const vda_problem& p, const __nv_bfloat16* Gf
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = frames < sms ? frames : sms;
+  // A text chain costs about as much as 8 frames; the weight is capped so
+  // that every CTA's share of (frames + weight * heads) covers its text:
+  // (frames + w heads) / grid >= w, i.e. w <= frames / (grid - heads).
+  prm.text_weight = 0;
+  if (prm.Wt && grid > heads) prm.text_weight = min(8, frames / (grid - heads));
   // Programmatic dependent launch: the CTAs start as the adjoint scan's CTAs
   // finish; griddep_wait() holds them until the adjoints are written.
   cudaLaunchConfig_t cfg = {};

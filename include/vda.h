@@ -107,8 +107,9 @@ typedef struct vda_problem {
  * kernel winds down: its other warps stop at their next decision point, the
  * copies and MMAs it has issued complete, its tensor memory is released, and
  * the kernels after it on the stream still end.  A nonzero test_stall names
- * one wait below; in the first CTA of the kernel that holds it (and only
- * there), that wait is made on a barrier nothing ever signals, so it runs out
+ * one wait below; in one CTA of the kernel that holds it (the first, unless
+ * the site says otherwise), that wait is made on a barrier nothing ever
+ * signals, so it runs out
  * exactly as a wait on a lost signal would.  The call then returns VDA_OK
  * (enqueued), vda_sync_status() reports VDA_ERR_TIMEOUT, and later calls run
  * normally.  A site that the problem's sizes never reach (for example the
@@ -128,7 +129,8 @@ enum {
   VDA_TEST_STALL_RBWD_DQ = 10,       /* readout backward: the epilogue's wait for the first dQ         */
   VDA_TEST_STALL_GBWD_TILE = 11,     /* Gram backward: the MMA thread's wait for the first K, V tile   */
   VDA_TEST_STALL_GBWD_STORE = 12,    /* Gram backward: the epilogue's wait for the second dK, dV       */
-  VDA_TEST_STALL_OPERANDS = 13,      /* backward operands: the MMA thread's wait for its first frame   */
+  VDA_TEST_STALL_OPERANDS = 13,      /* backward operands: the MMA thread's wait for its first frame,
+                                        in the kernel's last CTA (the first may have no frames)       */
   VDA_TEST_STALL_MERGE = 14,         /* vda_merge_project: the MMA thread's wait for its first K block */
   VDA_TEST_STALL_SOFTMAX = 15,       /* vda_local_softmax: the softmax warps' wait for the first scores */
   VDA_TEST_STALL_MAX = 15

@@ -4,8 +4,9 @@ Every wait inside the tensor-core kernels gives up after 2 s of the GPU's
 global timer; the kernel then sets the timeout bit of the error word and
 winds down (its other warps stop at their next decision point, its copies and
 MMAs complete, its tensor memory is released).  The testing hook
-``vda_problem.test_stall`` makes one named wait, in the first CTA of its
-kernel, wait on a barrier that nothing signals, so it runs out exactly as a
+``vda_problem.test_stall`` makes one named wait, in one CTA of its kernel
+(the first, or for the operands site the last), wait on a barrier that nothing
+signals, so it runs out exactly as a
 wait on a lost signal would.  Nothing faults: the hook only chooses which
 barrier a bounded wait watches.
 
