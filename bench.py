@@ -221,6 +221,18 @@ def cpu_threads():
     return os.cpu_count() or 1
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), for the CPU legs' lines."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def blas_limits():
     """Fixes the BLAS thread count for the oracle's timing (both CPU legs use the same)."""
     from threadpoolctl import threadpool_limits
@@ -311,7 +323,7 @@ def run_reference(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -571,7 +583,7 @@ def finish(args, w, ws_n, rank, pg, value, ms_step, roof, path, e2e, clocks):
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         v, threads, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": desc}
+                                "sample": desc, "cpu": cpu_model()}
     if pg:
         pg.barrier()
         pg.destroy_process_group()
