@@ -68,6 +68,24 @@ def test_merge_bad_problem_rejected(lib):
     assert s == vda.VDA_ERR_INVALID_ARG, vda.vda_last_error()
 
 
+def test_local_softmax_bad_arguments_rejected(lib):
+    # rejected on the host before any CUDA call; lambda is not read by this branch
+    ok = 1 << 20
+    args = [ok] * 7
+    p = _p(lam=0.0)
+    assert vda.vda_local_softmax(p, *args, None, stream=0, workspace_bytes=256, check=False) == vda.VDA_ERR_WORKSPACE
+    assert vda.vda_local_softmax(_p(), *args, ok, stream=0, workspace_bytes=255, check=False) == vda.VDA_ERR_WORKSPACE
+    assert vda.vda_local_softmax(_p(), *args, ok + 16, stream=0, workspace_bytes=256, check=False) == vda.VDA_ERR_WORKSPACE
+    assert vda.vda_local_softmax(_p(dtype=vda.VDA_DTYPE_F32), *args, ok, stream=0, workspace_bytes=256,
+                                 check=False) == vda.VDA_ERR_UNSUPPORTED
+    assert vda.vda_local_softmax(_p(dtype=vda.VDA_DTYPE_E4M3), *args, ok, stream=0, workspace_bytes=256,
+                                 check=False) == vda.VDA_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[0] = 0
+    assert vda.vda_local_softmax(_p(), *bad, ok, stream=0, workspace_bytes=256, check=False) == vda.VDA_ERR_INVALID_ARG
+    assert vda.vda_local_softmax(_p(T=0), *args, ok, stream=0, workspace_bytes=256, check=False) == vda.VDA_ERR_INVALID_ARG
+
+
 def _p(**kw):
     base = dict(B=1, H=2, T=3, n=64, n_txt=8, d_k=128, d_v=128, dtype=vda.VDA_DTYPE_BF16, lam=1.0)
     base.update(kw)
