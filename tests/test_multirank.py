@@ -82,3 +82,45 @@ def test_backward_roofline_bytes_are_the_tensors():
         assert rf["bytes"] == want, name
     assert bench.backward_roofline(synth.WORKLOADS["768p"], {"hbm_gbs": 6549.1, "bf16_tflops": 1628.0})["bytes"] \
         == 3352690688
+
+
+def test_forward_roofline_arithmetic():
+    """The forward line's algorithmic bytes and path roofline at 768p (SURVEY's table: 1.862 GB, 284.3 us at
+    the measured 6549.1 GB/s) and the e4m3 line's (Q, K, V, G and the text at one byte, O at two)."""
+    import bench
+    from frame_wise_linear_b200 import synth
+    peaks = {"hbm_gbs": 6549.1, "bf16_tflops": 1628.3}
+    w = synth.WORKLOADS["768p"]
+    pr = bench.path_roofline(w, peaks)
+    units, n, d, nt = w.B * w.H * w.T, w.n, w.d_k, w.n_txt
+    want = 5 * units * n * d * 2 + 2 * w.B * w.H * nt * d * 2
+    assert pr["bytes"] == want == 1862139904
+    assert abs(pr["t_roof_s"] * 1e6 - 284.3) < 0.1
+    assert bench.stage_work(w)["readout"]["bytes"] == 3 * units * n * d * 2      # Q, G read, O written
+    w8 = synth.WORKLOADS["768p_fp8"]
+    assert bench.path_roofline(w8, peaks)["bytes"] == 4 * units * n * d + units * n * d * 2 + 2 * w.B * w.H * nt * d
+
+
+def test_softmax_work_counts_the_window():
+    """The local softmax line's flops: 4 n keys d per query frame, keys = n x (window frames + anchors) + n_txt;
+    at T = 45 the window and anchors allow 45 x 15 - 50 (the edge blocks have one neighbour) + 70 = 695 frame pairs."""
+    import bench
+    from frame_wise_linear_b200 import synth
+    from oracle import softmax_oracle as so
+    w = synth.WORKLOADS["768p"]
+    pairs = sum(len(so.key_frames(t, w.T)) for t in range(w.T))
+    assert pairs == 45 * 15 - 50 + 70
+    want = 4 * w.B * w.H * w.n * w.d_k * (w.T * w.n_txt + pairs * w.n)
+    assert bench.softmax_work(w) == want
+
+
+def test_committed_dram_traffic_describes_the_current_forward_kernels():
+    """profiles/dram_traffic.txt holds the ncu DRAM bytes of the 768p forward kernels for their current
+    source files (the bench reports roofline.traffic only while the digests match)."""
+    import bench
+    from frame_wise_linear_b200 import synth
+    w = synth.WORKLOADS["768p"]
+    for stage in ("readout", "gram+factor", "scan"):
+        assert bench.traffic_lookup(stage, w) is not None, stage
+    algo = bench.stage_work(w)["readout"]["bytes"]
+    assert 1.0 <= bench.traffic_lookup("readout", w) / algo < 1.2
