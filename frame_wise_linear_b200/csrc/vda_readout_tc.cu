@@ -3,9 +3,9 @@
 // ("VDN-MiniMax-H3" (aiezz.com), section 03, gate fusion item: a
 // content-dependent sigmoid gate on the branch output).  bfloat16 Q, G, O and
 // states, d = 128; or e4m3 Q and G with per-tensor scales (O and states
-// bfloat16): each Q tile is widened exactly to bfloat16 in shared memory for
-// the MMA (an MMA takes one element type for both operands, and the states
-// stay bfloat16), and G is widened in the epilogue.
+// bfloat16): each Q tile is widened exactly to bfloat16 into tensor memory,
+// where the MMA reads its A operand (an MMA takes one element type for both
+// operands, and the states stay bfloat16), and G is widened in the epilogue.
 //
 // Precision: Q is exact in bf16; the scan hands over S^f and S^b as bf16,
 // and O = sigmoid(G) * (Q S^f + Q S^b) takes two MMA passes accumulated in
@@ -28,10 +28,12 @@
 //               as the MMAs release it.
 //   e4m3 inputs: Q and G tiles are half the size, so their rings are 3 and
 //               4 deep (about the bytes in flight of bf16).  The epilogue warps
-//               also widen the next tile's Q to bf16, each thread its own row
-//               and column half, straight into tensor memory, where the MMAs
-//               read A from (two 64-column slots); O goes out through two
-//               8 KB staging boxes per column half (32-column TMA stores).
+//               form two groups that take alternate tiles over all 128
+//               columns (the tile's parity picks its accumulator and its
+//               64-column A slot); each group also widens its next tile's Q,
+//               each thread its own row, straight into its A slot, and sends
+//               O out through its two 8 KB staging boxes in turn (32-column
+//               TMA stores).
 // Every wait is bounded (see sm100.cuh); a wait that runs out sets the timeout
 // bit of the error word and the CTA winds down.
 #include "sm100.cuh"
