@@ -68,6 +68,17 @@ def test_merge_bad_problem_rejected(lib):
     assert s == vda.VDA_ERR_INVALID_ARG, vda.vda_last_error()
 
 
+def test_backward_refuses_e4m3_and_f32(lib):
+    # the backward is built for bf16 inputs (d = 128); other types are refused on the host
+    ok = 1 << 20
+    for kw in (dict(dtype=vda.VDA_DTYPE_E4M3), dict(dtype=vda.VDA_DTYPE_F32)):
+        p = _p(**kw)
+        out = ctypes.c_size_t(0)
+        assert lib.vda_backward_workspace_size(ctypes.byref(p), ctypes.byref(out)) == vda.VDA_ERR_UNSUPPORTED
+        s = vda.vda_backward(p, *([ok] * 7), *([ok] * 6), ok, stream=0, workspace_bytes=1 << 40, check=False)
+        assert s == vda.VDA_ERR_UNSUPPORTED, vda.vda_last_error()
+
+
 def test_local_softmax_bad_arguments_rejected(lib):
     # rejected on the host before any CUDA call; lambda is not read by this branch
     ok = 1 << 20
