@@ -275,7 +275,11 @@ vda_status vda_backward_from_forward(const vda_problem* p, const void* Q, const 
  * read.  Scores, softmax and accumulation in float32; O rounded to bf16.
  * workspace: at least 256 bytes of device memory (256-byte aligned) holding
  * the device error word, which the call clears and vda_sync_status() reads.
- * Asynchronous on `stream`. */
+ * Asynchronous on `stream`.  Errors on the host, before anything is enqueued:
+ * vda_forward's size and pointer checks (VDA_ERR_INVALID_ARG,
+ * VDA_ERR_UNSUPPORTED), VDA_ERR_UNSUPPORTED for float32 or e4m3 problems,
+ * VDA_ERR_WORKSPACE for a missing, misaligned or short workspace; on the
+ * device, VDA_ERR_TIMEOUT through vda_sync_status(). */
 vda_status vda_local_softmax(const vda_problem* p, const void* Q, const void* K, const void* V, const void* G,
                              const void* K_txt, const void* V_txt, void* O, void* workspace, size_t workspace_bytes,
                              void* stream);
@@ -294,7 +298,13 @@ vda_status vda_local_softmax(const vda_problem* p, const void* Q, const void* K,
  * tokens >= 1; K a multiple of 64; D a multiple of 8 (>= 8).  Device
  * pointers, 16-byte aligned.  workspace: at least 256 bytes of device memory
  * (256-byte aligned) holding the device error word, which the call clears
- * and vda_sync_status() reads.  Asynchronous on `stream`. */
+ * and vda_sync_status() reads.  Asynchronous on `stream`.  Errors on the host,
+ * before anything is enqueued: VDA_ERR_INVALID_ARG for a NULL problem, tokens
+ * out of [1, 2^31 - 256], a NULL or misaligned pointer, O_sm or W_sm given
+ * alone, an unknown test_stall or a nonzero reserved field;
+ * VDA_ERR_UNSUPPORTED for K or D off the grid above; VDA_ERR_WORKSPACE for a
+ * missing, misaligned or short workspace; on the device, VDA_ERR_TIMEOUT
+ * through vda_sync_status(). */
 typedef struct vda_merge_problem {
   int64_t tokens;
   int32_t K, D;
