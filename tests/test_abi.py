@@ -68,6 +68,19 @@ def test_merge_bad_problem_rejected(lib):
     assert s == vda.VDA_ERR_INVALID_ARG, vda.vda_last_error()
 
 
+def test_noalloc_refuses_problems_above_its_scratch(lib):
+    # the size check comes before anything touches the device: the 768p problem needs about 287 MB
+    from frame_wise_linear_b200 import synth
+    ok = 1 << 20
+    big = vda.make_problem(**synth.WORKLOADS["768p"].problem())
+    assert vda.vda_workspace_size(big) > 64 << 20
+    s = vda.vda_forward_noalloc(big, *([ok] * 7), stream=0, check=False)
+    assert s == vda.VDA_ERR_WORKSPACE
+    assert "scratch" in vda.vda_last_error()
+    bad = _p(lam=-1.0)
+    assert vda.vda_forward_noalloc(bad, *([ok] * 7), stream=0, check=False) == vda.VDA_ERR_INVALID_ARG
+
+
 def test_backward_refuses_e4m3_and_f32(lib):
     # the backward is built for bf16 inputs (d = 128); other types are refused on the host
     ok = 1 << 20
